@@ -1,0 +1,20 @@
+"""Float64 CPU oracle for one Psi-Spec decode step (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The CUDA library and its Python binding
+never import it, and it imports nothing from them.
+"""
+
+from .uno_oracle import (  # noqa: F401
+    PHILOX_WORD_ACCEPT,
+    PHILOX_WORD_SAMPLE,
+    bf16_bits_to_f64,
+    dualpath_linear,
+    philox4x32_10,
+    round_to_bf16,
+    softmax_rows,
+    uniforms_for_block,
+    verify_block,
+    verify_block_u,
+    word_to_uniform,
+)
