@@ -1,0 +1,163 @@
+/*
+ * uno.h -- C ABI of the B200 (sm_100a) hot path of one Psi-Spec decode step.
+ *
+ * Source of the operations: "Unlocking Lossless Speedups in LLMs via Discrete
+ * Diffusion" (Uno). The picx.dev summary page, "Methodology / Architecture",
+ * and the paperglide reader page, "The Uno Framework", define the dual-pathway
+ * linear; the reader's "The Psi-Speculative Sampler" and "Sampler Extensions"
+ * (linear sampler) define the verification step, with the standard speculative
+ * rejection-sampling rule the pages cite (Leviathan et al. 2023; Chen et al.
+ * 2023).
+ *
+ * Conventions shared by every entry point:
+ *  - Every buffer argument is a DEVICE pointer owned by the caller. The library
+ *    never allocates, frees or keeps a reference to caller memory after a call.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the host. The return value reports argument
+ *    errors (checked on the host before anything is launched) and launch errors.
+ *  - Matrices are dense and row-major with no padding between rows.
+ *  - Base pointers of logits, activations, weights and outputs must be 16-byte
+ *    aligned (cudaMalloc and PyTorch allocations are 256-byte aligned).
+ *  - On an error nothing is launched and no output is written.
+ */
+#ifndef UNO_H_
+#define UNO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of logits, activations and weights. */
+typedef enum {
+  UNO_BF16 = 0, /* bfloat16 storage, float32 arithmetic                       */
+  UNO_F32 = 1   /* float32 storage; the GEMM runs on the TF32 tensor-core path */
+} uno_dtype;
+
+/* Status codes (negative = error). */
+typedef enum {
+  UNO_OK = 0,
+  UNO_ERR_NULL = -1,      /* a required pointer is NULL                         */
+  UNO_ERR_SIZE = -2,      /* a size is negative or beyond a documented limit    */
+  UNO_ERR_ALIGN = -3,     /* a pointer or a row stride breaks the 16-byte rule  */
+  UNO_ERR_DTYPE = -4,     /* dtype is not a uno_dtype value                     */
+  UNO_ERR_WORKSPACE = -5, /* workspace is NULL or smaller than required         */
+  UNO_ERR_CUDA = -6,      /* a CUDA runtime/driver call or a launch failed      */
+  UNO_ERR_DEVICE = -7     /* the current device is not an sm_100 GPU            */
+} uno_status;
+
+/* Human-readable name of a status code. Never returns NULL. */
+const char* uno_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int uno_version(void);
+
+/* ------------------------------------------------------------------------ *
+ * Block verifier (linear Psi-Spec sampler, verification step)
+ *
+ * For each sequence b in [0, B) with drafted ids x_0..x_{K-1}:
+ *   p_i = softmax(p_logits[b, i, :]), q_i = softmax(q_logits[b, i, :])
+ *   (temperature 1, float32 arithmetic on device).
+ *   u_i, u'_i = uniforms of Philox4x32-10 (Salmon et al., SC'11) with
+ *   key = (seed lo32, seed hi32) and counter = (b, i, step lo32, step hi32);
+ *   u_i = (word0 >> 8) * 2^-24, u'_i = (word1 >> 8) * 2^-24.
+ *   accept_i  <=>  u_i * q_i(x_i) < p_i(x_i)
+ *   n = index of the first rejected position, or K when all are accepted.
+ *   n < K : y ~ max(0, p_n - q_n) (normalised; p_n if that is all zero)
+ *   n = K : y ~ p_K (the bonus row).
+ *   y is drawn by inverse CDF in index order: the smallest v whose running
+ *   weight sum exceeds u'_n times the total.
+ *   out_tokens[b] = (x_0, ..., x_{n-1}, y, -1, ..., -1); accepted_len[b] = n.
+ * A draft id outside [0, V) in sequence b is reported on the device:
+ * accepted_len[b] = -1 and out_tokens[b, :] = -1 (the call still returns
+ * UNO_OK; the caller reads accepted_len to see it).
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes uno_verify_block needs for (B, K, V, dtype); 0 on bad sizes. */
+size_t uno_verify_workspace_bytes(int B, int K, int V, int dtype);
+
+/*
+ * p_logits      [B, K+1, V] dtype  AR (verifier) logits; row K is the bonus row
+ * q_logits      [B, K,   V] dtype  draft logits
+ * draft_tokens  [B, K]      int32  drafted ids
+ * B             0 <= B <= 2^20     (B = 0 launches nothing and returns UNO_OK)
+ * K             1 <= K <= 256      drafted positions per sequence
+ * V             1 <= V <= 2^28     vocabulary size (any value; no alignment rule)
+ * seed, step    Philox key and counter words (see above)
+ * out_tokens    [B, K+1]    int32  emitted tokens, -1 padded        (required)
+ * accepted_len  [B]         int32  accepted draft count n (or -1)   (required)
+ * p_at_draft    [B, K]      float  p_i(x_i)                         (optional, NULL)
+ * q_at_draft    [B, K]      float  q_i(x_i)                         (optional, NULL)
+ * row_lse       [B, 2K+1]   float  log-sum-exp of every row: p rows 0..K,
+ *                                  then q rows 0..K-1               (optional, NULL)
+ * workspace     device scratch of at least uno_verify_workspace_bytes(B,K,V,dtype)
+ *               bytes, 16-byte aligned. It must be zero-filled before its FIRST
+ *               use; every call leaves it zero-filled again, so a workspace is
+ *               reused without clearing. Two calls that share a workspace must
+ *               be ordered on one stream.
+ * stream        cudaStream_t
+ * Returns UNO_OK or a negative uno_status.
+ */
+int uno_verify_block(const void* p_logits, const void* q_logits, const int32_t* draft_tokens,
+                     int B, int K, int V, int dtype, uint64_t seed, uint64_t step,
+                     int32_t* out_tokens, int32_t* accepted_len, float* p_at_draft,
+                     float* q_at_draft, float* row_lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * Dual-pathway linear (one pass over the frozen weight W)
+ *
+ *   y_ar    = x W^T                       (verification pathway, theta_AR)
+ *   T       = scale * x A^T               (LoRA down projection, scale = alpha/r)
+ *   y_draft = y_ar + T Bm^T               (drafting pathway, theta_AR + theta_Delta)
+ *
+ * Arithmetic: tcgen05 tensor cores, float32 accumulation. With UNO_BF16
+ * operands T is rounded to bfloat16 before the adapter product (it is a
+ * bfloat16 tensor-core operand); with UNO_F32 operands every product runs in
+ * TF32 and T stays float32. Outputs are stored in dtype, rounded to nearest.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes uno_dualpath_linear needs; 0 on bad sizes. */
+size_t uno_dualpath_workspace_bytes(int M, int d_in, int d_out, int r, int dtype);
+
+/*
+ * x        [M, d_in]      dtype  activations
+ * W        [d_out, d_in]  dtype  frozen AR weight (nn.Linear layout)
+ * A        [r, d_in]      dtype  LoRA down weight
+ * Bm       [d_out, r]     dtype  LoRA up weight
+ * scale    alpha / r
+ * y_ar     [M, d_out]     dtype  output, or NULL to skip it
+ * y_draft  [M, d_out]     dtype  output, or NULL to skip it (and the adapter)
+ * M        0 <= M <= 2^24 rows (M = 0 launches nothing)
+ * d_in     >= 1, multiple of 8 (bf16) / 4 (f32) so rows are 16-byte strided
+ * d_out    >= 1, multiple of 8 (bf16) / 4 (f32)
+ * r        1 <= r <= 256, multiple of 8 (bf16) / 4 (f32)
+ * workspace  device scratch of at least uno_dualpath_workspace_bytes(...) bytes,
+ *            16-byte aligned, contents irrelevant on entry. Two calls that
+ *            share a workspace must be ordered on one stream.
+ * Returns UNO_OK or a negative uno_status. At least one of y_ar / y_draft
+ * must be non-NULL.
+ */
+int uno_dualpath_linear(const void* x, const void* W, const void* A, const void* Bm,
+                        float scale, void* y_ar, void* y_draft, int M, int d_in, int d_out,
+                        int r, int dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * Device fault flags
+ *
+ * Every wait inside the kernels is bounded in time. A wait that gives up
+ * (which correct code never does) sets a bit here, abandons its work and lets
+ * the kernel exit instead of hanging the GPU: bit 0 TMA producer, bit 1 MMA
+ * issuer, bit 2 epilogue. This call synchronises the device, writes the
+ * current flags to *flags and clears them when `clear` is non-zero.
+ * ------------------------------------------------------------------------ */
+int uno_device_fault_flags(int clear, unsigned int* flags);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* UNO_H_ */

@@ -1,0 +1,191 @@
+"""PyTorch-facing binding of the Uno C ABI (argument marshalling only).
+
+Every step of the computation runs in libuno.so's sm_100a kernels; this
+module checks tensor devices, dtypes and shapes, allocates outputs and
+workspaces through PyTorch, and passes raw pointers and the current CUDA
+stream to the C entry points of the same names.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from ._lib import UNO_BF16, UNO_F32, UnoError, lib
+
+_DT = {torch.bfloat16: UNO_BF16, torch.float32: UNO_F32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32") from None
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_cuda(*ts: Optional[torch.Tensor]) -> torch.device:
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous (row-major, no padding)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("all tensors must live on the same device")
+    return dev
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+class _Workspaces:
+    """Grow-only device scratch buffers, one per (device, purpose).
+
+    The verifier's workspace must be zero on first use and is left zeroed by
+    every call, so it is allocated with zeros and reused as is. Calls that use
+    one cached workspace are ordered on the current stream of the caller.
+    """
+
+    def __init__(self):
+        self._bufs: dict = {}
+
+    def get(self, device: torch.device, purpose: str, nbytes: int) -> torch.Tensor:
+        key = (device.index, purpose)
+        buf = self._bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self._bufs[key] = buf
+        return buf
+
+
+_ws = _Workspaces()
+
+
+# ---------------------------------------------------------------------------
+# block verifier
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class VerifyResult:
+    out_tokens: torch.Tensor            # [B, K+1] int32, -1 padded
+    accepted_len: torch.Tensor          # [B] int32 (-1 marks an invalid draft id)
+    p_at_draft: Optional[torch.Tensor]  # [B, K] float32
+    q_at_draft: Optional[torch.Tensor]  # [B, K] float32
+    row_lse: Optional[torch.Tensor]     # [B, 2K+1] float32
+
+
+def verify_workspace_bytes(B: int, K: int, V: int, dtype: torch.dtype) -> int:
+    return int(lib.uno_verify_workspace_bytes(B, K, V, _DT[dtype]))
+
+
+def verify_block(p_logits: torch.Tensor, q_logits: torch.Tensor, draft_tokens: torch.Tensor,
+                 seed: int, step: int, *, want_probs: bool = False, want_lse: bool = False,
+                 out: Optional[VerifyResult] = None,
+                 workspace: Optional[torch.Tensor] = None) -> VerifyResult:
+    """Verify one drafted block per sequence (see ``uno_verify_block`` in uno.h).
+
+    p_logits [B, K+1, V] and q_logits [B, K, V] (bfloat16 or float32, same
+    dtype), draft_tokens [B, K] int32. Runs asynchronously on the current
+    stream.
+    """
+    if p_logits.dim() != 3 or q_logits.dim() != 3 or draft_tokens.dim() != 2:
+        raise ValueError("expected p [B,K+1,V], q [B,K,V], drafts [B,K]")
+    B, K1, V = p_logits.shape
+    K = K1 - 1
+    if tuple(q_logits.shape) != (B, K, V) or tuple(draft_tokens.shape) != (B, K):
+        raise ValueError("shape mismatch: p [B,K+1,V], q [B,K,V], drafts [B,K]")
+    if q_logits.dtype != p_logits.dtype:
+        raise TypeError("p_logits and q_logits must share a dtype")
+    if draft_tokens.dtype != torch.int32:
+        raise TypeError("draft_tokens must be int32")
+    dt = _dtype_code(p_logits)
+    dev = _check_cuda(p_logits, q_logits, draft_tokens)
+    if out is None:
+        out = VerifyResult(
+            torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+            torch.empty((B,), dtype=torch.int32, device=dev),
+            torch.empty((B, K), dtype=torch.float32, device=dev) if want_probs else None,
+            torch.empty((B, K), dtype=torch.float32, device=dev) if want_probs else None,
+            torch.empty((B, 2 * K + 1), dtype=torch.float32, device=dev) if want_lse else None,
+        )
+    _check_cuda(out.out_tokens, out.accepted_len, out.p_at_draft, out.q_at_draft, out.row_lse)
+    need = int(lib.uno_verify_workspace_bytes(B, K, V, dt))
+    ws = workspace if workspace is not None else _ws.get(dev, "verify", need)
+    st = lib.uno_verify_block(
+        _ptr(p_logits), _ptr(q_logits), _ptr(draft_tokens), B, K, V, dt,
+        ctypes.c_uint64(int(seed) & (2**64 - 1)), ctypes.c_uint64(int(step) & (2**64 - 1)),
+        _ptr(out.out_tokens), _ptr(out.accepted_len), _ptr(out.p_at_draft),
+        _ptr(out.q_at_draft), _ptr(out.row_lse), _ptr(ws), ws.numel(), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_verify_block")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# dual-pathway linear
+# ---------------------------------------------------------------------------
+
+
+def dualpath_workspace_bytes(M: int, d_in: int, d_out: int, r: int, dtype: torch.dtype) -> int:
+    return int(lib.uno_dualpath_workspace_bytes(M, d_in, d_out, r, _DT[dtype]))
+
+
+def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor,
+                    scale: float, *, want_ar: bool = True, want_draft: bool = True,
+                    y_ar: Optional[torch.Tensor] = None, y_draft: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None):
+    """y_ar = x W^T and y_draft = y_ar + scale (x A^T) Bm^T in one pass over W.
+
+    x [M, d_in], W [d_out, d_in], A [r, d_in], Bm [d_out, r], all bfloat16 or
+    all float32. Returns (y_ar, y_draft); an output not wanted is None.
+    """
+    if x.dim() != 2 or W.dim() != 2 or A.dim() != 2 or Bm.dim() != 2:
+        raise ValueError("expected 2-D x, W, A, Bm")
+    M, d_in = x.shape
+    d_out = W.shape[0]
+    r = A.shape[0]
+    if W.shape[1] != d_in or A.shape[1] != d_in or tuple(Bm.shape) != (d_out, r):
+        raise ValueError("shape mismatch: x [M,d_in], W [d_out,d_in], A [r,d_in], Bm [d_out,r]")
+    if not (x.dtype == W.dtype == A.dtype == Bm.dtype):
+        raise TypeError("x, W, A and Bm must share a dtype")
+    dt = _dtype_code(x)
+    dev = _check_cuda(x, W, A, Bm)
+    if want_ar and y_ar is None:
+        y_ar = torch.empty((M, d_out), dtype=x.dtype, device=dev)
+    if want_draft and y_draft is None:
+        y_draft = torch.empty((M, d_out), dtype=x.dtype, device=dev)
+    if not want_ar:
+        y_ar = None
+    if not want_draft:
+        y_draft = None
+    _check_cuda(y_ar, y_draft)
+    need = int(lib.uno_dualpath_workspace_bytes(M, d_in, d_out, r, dt))
+    ws = workspace if workspace is not None else _ws.get(dev, "dualpath", need)
+    st = lib.uno_dualpath_linear(_ptr(x), _ptr(W), _ptr(A), _ptr(Bm), ctypes.c_float(scale),
+                                 _ptr(y_ar), _ptr(y_draft), M, d_in, d_out, r, dt, _ptr(ws),
+                                 ws.numel(), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_dualpath_linear")
+    return y_ar, y_draft
+
+
+def device_fault_flags(clear: bool = True) -> int:
+    """Fault bits set by a kernel wait that gave up (0 = none). Synchronises."""
+    flags = ctypes.c_uint(0)
+    st = lib.uno_device_fault_flags(1 if clear else 0, ctypes.byref(flags))
+    if st != 0:
+        raise UnoError(st, "uno_device_fault_flags")
+    return int(flags.value)

@@ -1,0 +1,62 @@
+// Device-side helpers shared by the Uno sm_100a kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace uno {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and Shaw,
+// "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11). Ten rounds; each
+// round multiplies counter words 0 and 2 by the two Philox multipliers, takes
+// the high and low halves of the 64-bit products, and mixes in the key, which
+// is bumped by the two Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t m0 = 0xD2511F53u, m1 = 0xCD9E8D57u;
+    const uint32_t lo0 = m0 * c.x, hi0 = __umulhi(m0, c.x);
+    const uint32_t lo1 = m1 * c.z, hi1 = __umulhi(m1, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+    k.x += 0x9E3779B9u;
+    k.y += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Top 24 bits of a Philox word as a float in [0, 1): exact in float32.
+__device__ __forceinline__ float uniform24(uint32_t w) {
+  return static_cast<float>(w >> 8) * 5.9604644775390625e-08f;  // 2^-24
+}
+
+// Uniforms of sequence b, position i: counter (b, i, step lo, step hi),
+// key (seed lo, seed hi). Word 0 -> accept test, word 1 -> token draw.
+__device__ __forceinline__ uint4 verify_block_words(uint64_t seed, uint64_t step, uint32_t b,
+                                                    uint32_t i) {
+  return philox4x32_10(make_uint4(b, i, static_cast<uint32_t>(step),
+                                  static_cast<uint32_t>(step >> 32)),
+                       make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)));
+}
+
+// 2^x on the SFU (PTX ex2.approx, flush-to-zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) {
+  return __uint_as_float(h16 << 16);
+}
+
+// Round-to-nearest-even float -> bfloat16 bits (finite inputs; NaN kept NaN).
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0x7FC0;
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+}  // namespace uno

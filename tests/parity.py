@@ -1,0 +1,104 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+Token ids and accepted lengths must match exactly, except where the oracle's
+decision lies within a near-tie band (float32 on the device cannot decide it
+the same way for certain):
+  * an accept test with |u - p/q| < 1e-5 (the stated criterion); the row is
+    not compared from that position on;
+  * a token draw whose threshold u' * total lies within
+    TAU_ABS + TAU_REL * total of a CDF boundary of the oracle.
+Probabilities must match within 1e-5 absolute.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+ACCEPT_TIE = 1e-5
+TAU_ABS = 2e-6
+TAU_REL = 1e-5
+PROB_ATOL = 1e-5
+
+
+def widen(t: torch.Tensor) -> np.ndarray:
+    """Exact float64 copy of a bf16/f32 tensor (CPU)."""
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+@dataclass
+class VerifyReport:
+    rows: int
+    compared: int
+    accept_ties: int
+    draw_ties: int
+    invalid: int
+
+
+def compare_verify(gpu, ref, check_probs: bool = True) -> VerifyReport:
+    """Assert the CUDA verifier agrees with the oracle; return tie counts."""
+    n_g = gpu.accepted_len.cpu().numpy()
+    out_g = gpu.out_tokens.cpu().numpy()
+    n_o = ref["accepted_len"]
+    out_o = ref["out_tokens"]
+    B, K1 = out_o.shape
+    K = K1 - 1
+    ratio, u = ref["ratio"], ref["u_acc"]
+    acc_ties = draw_ties = compared = invalid = 0
+    for b in range(B):
+        if n_o[b] < 0:
+            invalid += 1
+            assert n_g[b] == -1 and np.all(out_g[b] == -1), f"row {b}: invalid drafts not flagged"
+            continue
+        last = min(n_o[b], K - 1)
+        tie = np.abs(u[b, : last + 1] - ratio[b, : last + 1]) < ACCEPT_TIE
+        if tie.any():
+            acc_ties += 1
+            first = int(np.argmax(tie))
+            # decisions before the tie must still agree
+            assert n_g[b] >= first, f"row {b}: rejected at {n_g[b]} before tie at {first}"
+            assert np.array_equal(out_g[b, :first], out_o[b, :first])
+            continue
+        assert n_g[b] == n_o[b], f"row {b}: accepted {n_g[b]} vs oracle {n_o[b]}"
+        n = n_o[b]
+        assert np.array_equal(out_g[b, :n], out_o[b, :n])
+        assert np.all(out_g[b, n + 1:] == -1)
+        t, lo, hi, tot = ref["cdf_t"][b], ref["cdf_prev"][b], ref["cdf_at"][b], ref["cdf_total"][b]
+        tau = TAU_ABS + TAU_REL * tot
+        if min(t - lo, hi - t) < tau:
+            draw_ties += 1
+            continue
+        assert out_g[b, n] == out_o[b, n], f"row {b}: token {out_g[b, n]} vs oracle {out_o[b, n]}"
+        compared += 1
+    if check_probs and gpu.p_at_draft is not None:
+        valid = n_o >= 0
+        for name in ("p_at_draft", "q_at_draft"):
+            g = getattr(gpu, name).cpu().numpy()[valid]
+            err = np.abs(g - ref[name][valid]).max() if valid.any() else 0.0
+            assert err < PROB_ATOL, f"{name} max abs error {err}"
+    if gpu.row_lse is not None:
+        g = gpu.row_lse.cpu().numpy()
+        err = np.abs(g - ref["row_lse"]).max()
+        # lse = log Z: an absolute error of e in lse is a relative error e in Z.
+        assert err < 2e-5 * max(1.0, np.abs(ref["row_lse"]).max()), f"row_lse error {err}"
+    return VerifyReport(B, compared, acc_ties, draw_ties, invalid)
+
+
+def rel_err_normwise(got: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+def assert_dualpath_close(got: torch.Tensor, ref: np.ndarray, tol: float = 2e-2):
+    """Normwise max relative error (the stated criterion) plus an elementwise
+    bound |y - ref| <= tol*|ref| + tol*rms(ref)."""
+    g = widen(got)
+    assert g.shape == ref.shape
+    assert np.all(np.isfinite(g))
+    e = rel_err_normwise(g, ref)
+    assert e < tol, f"normwise relative error {e}"
+    rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
+    bad = np.abs(g - ref) > tol * np.abs(ref) + tol * rms
+    assert not bad.any(), f"{int(bad.sum())} elements outside the elementwise bound"
+    return e

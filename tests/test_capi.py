@@ -1,0 +1,116 @@
+"""The C ABI library loads and exports every function include/uno.h declares.
+
+Runs without a GPU: only host-side entry points and argument validation are
+called (validation happens before any CUDA call, so bad arguments are
+reported on any machine).
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "uno.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lossless_decoding_b200.build import build_library
+    build_library()
+    from lossless_decoding_b200._lib import lib as L
+    return L
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(uno_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("uno_verify_block", "uno_dualpath_linear", "uno_verify_workspace_bytes",
+                     "uno_dualpath_workspace_bytes", "uno_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(os.path.join(ROOT, "lossless_decoding_b200", "libuno.so"))
+    for name in _declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    for code in range(-7, 1):
+        s = lib.uno_status_string(code).decode()
+        assert s.startswith("UNO_")
+    assert lib.uno_status_string(-99).decode() == "UNO_ERR_UNKNOWN"
+    assert lib.uno_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    assert lib.uno_verify_workspace_bytes(64, 16, 151936, 0) > 0
+    assert lib.uno_verify_workspace_bytes(-1, 16, 100, 0) == 0
+    assert lib.uno_verify_workspace_bytes(1, 0, 100, 0) == 0
+    assert lib.uno_verify_workspace_bytes(1, 257, 100, 0) == 0
+    assert lib.uno_verify_workspace_bytes(1, 4, 100, 7) == 0
+    assert lib.uno_dualpath_workspace_bytes(1024, 4096, 4096, 128, 0) >= 1024 * 128 * 2
+    assert lib.uno_dualpath_workspace_bytes(16, 4096, 151936, 128, 0) > 0
+    assert lib.uno_dualpath_workspace_bytes(16, 4100, 4096, 128, 0) == 0   # d_in % 8
+    assert lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 257, 0) == 0   # r > 256
+    assert lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 12, 0) == 0    # r % 8 (bf16)
+    assert lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 12, 1) > 0     # r % 4 (f32)
+
+
+def test_argument_errors_need_no_gpu(lib):
+    from lossless_decoding_b200._lib import STATUS
+    fake = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(4096 + 2)
+    u64 = ctypes.c_uint64
+    # verify: dtype, size, null, alignment, workspace
+    call = lib.uno_verify_block
+    assert STATUS[call(fake, fake, fake, 1, 4, 10, 9, u64(0), u64(0), fake, fake, None, None,
+                       None, fake, 1 << 20, None)] == "UNO_ERR_DTYPE"
+    assert STATUS[call(fake, fake, fake, 1, 0, 10, 0, u64(0), u64(0), fake, fake, None, None,
+                       None, fake, 1 << 20, None)] == "UNO_ERR_SIZE"
+    assert STATUS[call(None, fake, fake, 1, 4, 10, 0, u64(0), u64(0), fake, fake, None, None,
+                       None, fake, 1 << 20, None)] == "UNO_ERR_NULL"
+    assert STATUS[call(odd, fake, fake, 1, 4, 10, 0, u64(0), u64(0), fake, fake, None, None,
+                       None, fake, 1 << 20, None)] == "UNO_ERR_ALIGN"
+    assert STATUS[call(fake, fake, fake, 1, 4, 10, 0, u64(0), u64(0), fake, fake, None, None,
+                       None, fake, 8, None)] == "UNO_ERR_WORKSPACE"
+    assert STATUS[call(fake, fake, fake, 1, 4, 10, 0, u64(0), u64(0), fake, fake, None, None,
+                       None, None, 1 << 20, None)] == "UNO_ERR_WORKSPACE"
+    # B = 0 is an empty, valid call
+    assert call(None, None, None, 0, 4, 10, 0, u64(0), u64(0), None, None, None, None, None,
+                None, 0, None) == 0
+    # dual path
+    dual = lib.uno_dualpath_linear
+    assert STATUS[dual(fake, fake, fake, fake, 2.0, fake, fake, 16, 4096, 4096, 128, 5, fake,
+                       1 << 30, None)] == "UNO_ERR_DTYPE"
+    assert STATUS[dual(fake, fake, fake, fake, 2.0, fake, fake, 16, 4095, 4096, 128, 0, fake,
+                       1 << 30, None)] == "UNO_ERR_SIZE"
+    assert STATUS[dual(fake, fake, fake, fake, 2.0, None, None, 16, 4096, 4096, 128, 0, fake,
+                       1 << 30, None)] == "UNO_ERR_NULL"
+    assert STATUS[dual(fake, fake, None, fake, 2.0, fake, fake, 16, 4096, 4096, 128, 0, fake,
+                       1 << 30, None)] == "UNO_ERR_NULL"
+    assert STATUS[dual(fake, odd, fake, fake, 2.0, fake, fake, 16, 4096, 4096, 128, 0, fake,
+                       1 << 30, None)] == "UNO_ERR_ALIGN"
+    assert STATUS[dual(fake, fake, fake, fake, 2.0, fake, fake, 16, 4096, 4096, 128, 0, fake,
+                       16, None)] == "UNO_ERR_WORKSPACE"
+    assert dual(None, None, None, None, 2.0, None, None, 0, 4096, 4096, 128, 0, None, 0,
+                None) == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    from lossless_decoding_b200 import api
+    p = torch.zeros(1, 3, 8)
+    with pytest.raises(ValueError):
+        api.verify_block(p, torch.zeros(1, 2, 8), torch.zeros(1, 2, dtype=torch.int32), 0, 0)
+    x = torch.zeros(4, 8)
+    with pytest.raises(ValueError):
+        api.dualpath_linear(x, torch.zeros(8, 8), torch.zeros(8, 8), torch.zeros(8, 8), 1.0)

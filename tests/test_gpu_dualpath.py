@@ -1,0 +1,152 @@
+"""Parity of the CUDA dual-pathway linear with the float64 oracle (needs a B200).
+
+Criterion: normwise max relative error below 2e-2 per output (bf16 operands,
+float32 accumulation; float32 operands run on the TF32 path), plus an
+elementwise bound (tests/parity.py). Large shapes compare a seeded sample of
+rows or columns, which the oracle computes directly (every output element is
+an independent dot product).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lossless_decoding_b200.inputs import QWEN3_8B_PROJECTIONS, dualpath_inputs
+from tests.parity import assert_dualpath_close, widen
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lossless_decoding_b200 import api as A
+    return A
+
+
+def _ref(d, rows=None, cols=None):
+    """Oracle on a subset: rows of x and/or output columns (rows of W and Bm)."""
+    x, W, Bm = d.x, d.W, d.Bm
+    if rows is not None:
+        x = x[torch.as_tensor(rows, device=x.device)]
+    if cols is not None:
+        ci = torch.as_tensor(cols, device=W.device)
+        W, Bm = W[ci], Bm[ci]
+    return oracle.dualpath_linear(widen(x), widen(W), widen(d.A), widen(Bm), d.scale,
+                                  round_t_to_bf16=(d.x.dtype == torch.bfloat16))
+
+
+def _run(api, d, **kw):
+    y = api.dualpath_linear(d.x.to(DEV), d.W.to(DEV), d.A.to(DEV), d.Bm.to(DEV), d.scale, **kw)
+    torch.cuda.synchronize()
+    return y
+
+
+def test_tiny_configuration_tf32(api):
+    d = dualpath_inputs(M=8, d_in=512, d_out=512, r=16, alpha=32.0, dtype="f32", b_std=0.01,
+                        seed=0)
+    y_ar, y_dr = _run(api, d)
+    ref_ar, ref_dr, _ = _ref(d)
+    assert_dualpath_close(y_ar, ref_ar)
+    assert_dualpath_close(y_dr, ref_dr)
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,dtype", [
+    (1, 64, 8, 8, "bf16"),
+    (8, 512, 136, 16, "bf16"),
+    (16, 520, 1000, 128, "bf16"),
+    (17, 4096, 1024, 128, "bf16"),       # K+1 = 17 rows (bonus row)
+    (100, 1024, 776, 64, "bf16"),
+    (256, 256, 384, 256, "bf16"),
+    (257, 512, 264, 128, "bf16"),         # first non-swapped size, ragged everything
+    (300, 1032, 520, 24, "bf16"),
+    (1024, 2048, 1024, 128, "bf16"),
+    (40, 300, 100, 20, "f32"),
+    (520, 260, 300, 36, "f32"),
+])
+def test_parity_shapes(api, M, d_in, d_out, r, dtype):
+    d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=r, alpha=2.0 * r, dtype=dtype,
+                        seed=M + d_in)
+    y_ar, y_dr = _run(api, d)
+    ref_ar, ref_dr, _ = _ref(d)
+    assert_dualpath_close(y_ar, ref_ar)
+    assert_dualpath_close(y_dr, ref_dr)
+    # the adapter term itself is resolved, not swamped by y_ar
+    delta = widen(y_dr) - widen(y_ar)
+    ref_delta = ref_dr - ref_ar
+    if np.abs(ref_delta).max() > 0:
+        rel = np.abs(delta - ref_delta).max() / np.abs(ref_delta).max()
+        assert rel < 0.1, f"adapter term relative error {rel}"
+    assert api.device_fault_flags() == 0
+
+
+def test_outputs_are_optional_and_adapter_zero_is_exact(api):
+    d = dualpath_inputs(M=64, d_in=512, d_out=512, r=32, alpha=64.0, seed=3)
+    y_ar, y_dr = _run(api, d)
+    a_only, none = _run(api, d, want_draft=False)
+    assert none is None and torch.equal(a_only, y_ar)
+    none, d_only = _run(api, d, want_ar=False)
+    assert none is None and torch.equal(d_only, y_dr)
+    d.Bm.zero_()
+    y_ar0, y_dr0 = _run(api, d)
+    assert torch.equal(y_ar0, y_dr0)
+    for M in (300, 1024):  # non-swapped tiles as well
+        d2 = dualpath_inputs(M=M, d_in=256, d_out=512, r=16, alpha=32.0, seed=M)
+        d2.Bm.zero_()
+        a, b = _run(api, d2)
+        assert torch.equal(a, b)
+
+
+def test_workspace_contents_do_not_matter(api):
+    d = dualpath_inputs(M=300, d_in=1024, d_out=512, r=128, alpha=256.0, seed=11)
+    need = api.dualpath_workspace_bytes(300, 1024, 512, 128, torch.bfloat16)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)  # NaN bit patterns
+    y1 = _run(api, d, workspace=ws)
+    y2 = _run(api, d)
+    assert torch.equal(y1[0], y2[0]) and torch.equal(y1[1], y2[1])
+
+
+def test_outputs_stay_in_bounds(api):
+    M, d_in, d_out, r = 33, 256, 136, 16
+    d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=r, alpha=32.0, seed=4)
+    big_a = torch.full((M * d_out + 4096,), 7.0, dtype=torch.bfloat16, device=DEV)
+    big_d = torch.full((M * d_out + 4096,), 7.0, dtype=torch.bfloat16, device=DEV)
+    _run(api, d, y_ar=big_a[: M * d_out].view(M, d_out), y_draft=big_d[: M * d_out].view(M, d_out))
+    assert torch.all(big_a[M * d_out:] == 7.0) and torch.all(big_d[M * d_out:] == 7.0)
+
+
+def test_lm_head_single_sequence_sampled_columns(api):
+    # Qwen3-8B-shaped LM head 4096 -> 151936 at M = 16 (K drafts) and 17 (+ bonus row)
+    for M in (16, 17):
+        d = dualpath_inputs(M=M, d_in=4096, d_out=151936, r=128, alpha=256.0, seed=M,
+                            device=DEV)
+        y_ar, y_dr = api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale)
+        torch.cuda.synchronize()
+        cols = np.sort(np.random.default_rng(M).choice(151936, size=2048, replace=False))
+        cols = np.concatenate([cols, np.arange(151936 - 64, 151936)])  # the last, ragged tile
+        ref_ar, ref_dr, _ = _ref(d, cols=cols)
+        ci = torch.from_numpy(cols).to(DEV)
+        assert_dualpath_close(y_ar[:, ci], ref_ar)
+        assert_dualpath_close(y_dr[:, ci], ref_dr)
+        del d, y_ar, y_dr
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,d_in,d_out", QWEN3_8B_PROJECTIONS)
+def test_batched_decode_projections_sampled_rows(api, name, d_in, d_out):
+    # B=64 sequences x K=16 drafts = 1024 rows, rank-128 adapters with alpha 256
+    d = dualpath_inputs(M=1024, d_in=d_in, d_out=d_out, r=128, alpha=256.0, seed=d_in + d_out,
+                        device=DEV)
+    y_ar, y_dr = api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(1).choice(1024, size=48, replace=False))
+    rows = np.concatenate([rows, np.arange(1024 - 16, 1024)])
+    ref_ar, ref_dr, _ = _ref(d, rows=rows)
+    ri = torch.from_numpy(rows).to(DEV)
+    assert_dualpath_close(y_ar[ri], ref_ar)
+    assert_dualpath_close(y_dr[ri], ref_dr)
+    assert api.device_fault_flags() == 0
