@@ -1,0 +1,530 @@
+"""Benchmark of one Psi-Spec decode step's hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batched_decode_b64_k16|qwen3_8b_b1]
+
+A step is one pass over the whole hot path for one batch:
+  batched_decode_b64_k16 (default): B = 64 sequences x K = 16 drafted positions
+      = 1024 rows; the dual-pathway linear of every projection of one
+      Qwen3-8B-shaped layer (q, k, v, o, gate, up, down; rank-128 LoRA,
+      alpha 256, bf16) over the 1024 rows, then the block verifier over
+      64 x (2*16+1) rows of 151936 bf16 logits.
+  qwen3_8b_b1: one sequence, K = 16: the dual-path LM head 4096 -> 151936 over
+      the 17 rows (16 drafts + the bonus row), then the verifier on its logits
+      (p = y_AR rows, q = y_draft rows).
+
+The metric is verified draft rows per second (B*K per step); emitted tokens
+per second is reported beside it. Inputs are synthetic and seeded (random
+weights; no checkpoint or dataset) and larger than L2 per step. Timing: W
+warm-up steps, then K steps bracketed by a barrier and device syncs, CUDA
+events on the launching stream, max over ranks. One JSON line on rank 0.
+
+--impl reference runs the float64 CPU oracle (the only other implementation
+there is) on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from lossless_decoding_b200.inputs import (QWEN3_8B_HIDDEN, QWEN3_8B_PROJECTIONS,  # noqa: E402
+                                           QWEN3_8B_VOCAB)
+
+B64, K16, RANK, ALPHA = 64, 16, 128, 256.0
+METRIC = "verified draft rows/s"
+UNIT = "rows/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained"), "src": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workloads on the device
+# ---------------------------------------------------------------------------
+
+
+def _dual_flops(M, d_in, d_out, r):
+    return 2.0 * M * d_in * d_out + 2.0 * M * r * (d_in + d_out)
+
+
+class BatchedDecode:
+    """64 sequences x 16 drafts: 7 dual-path projections + verify."""
+
+    name = "batched_decode_b64_k16"
+
+    def __init__(self, dev, seed):
+        from lossless_decoding_b200 import api
+        from lossless_decoding_b200.inputs import dualpath_inputs, verify_inputs
+        self.api = api
+        self.B, self.K, self.V = B64, K16, QWEN3_8B_VOCAB
+        self.M = self.B * self.K
+        self.layers = []
+        for i, (name, d_in, d_out) in enumerate(QWEN3_8B_PROJECTIONS):
+            d = dualpath_inputs(M=self.M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA,
+                                seed=seed * 100 + i, device=dev)
+            y_ar = torch.empty((self.M, d_out), dtype=torch.bfloat16, device=dev)
+            y_dr = torch.empty_like(y_ar)
+            ws = torch.empty(api.dualpath_workspace_bytes(self.M, d_in, d_out, RANK,
+                                                          torch.bfloat16),
+                             dtype=torch.uint8, device=dev)
+            self.layers.append((name, d, y_ar, y_dr, ws))
+        self.v = verify_inputs(self.B, self.K, self.V, dtype="bf16", dist="normal", p_std=2.0,
+                               sigma=1.0, seed=seed, device=dev)
+        self.vws = torch.zeros(api.verify_workspace_bytes(self.B, self.K, self.V,
+                                                          torch.bfloat16),
+                               dtype=torch.uint8, device=dev)
+        self.out = api.VerifyResult(
+            torch.empty((self.B, self.K + 1), dtype=torch.int32, device=dev),
+            torch.empty((self.B,), dtype=torch.int32, device=dev), None, None, None)
+        self.gemm_flops = sum(_dual_flops(self.M, d.x.shape[1], d.W.shape[0], RANK)
+                              for _, d, *_ in self.layers)
+        self.verify_bytes = (self.B * (2 * self.K + 1) * self.V * 2 + self.B * self.K * 4
+                             + self.B * (self.K + 2) * 4)
+        self.launches_per_step = 3 * len(self.layers) + 1
+        # bytes a step reads at least once (all distinct, so L2 cannot carry them)
+        self.step_bytes = sum(d.x.numel() * 2 + d.W.numel() * 2 + d.A.numel() * 2
+                              + d.Bm.numel() * 2 for _, d, *_ in self.layers) + self.verify_bytes
+
+    def step(self, seed_step, ev=None):
+        api = self.api
+        for i, (_, d, y_ar, y_dr, ws) in enumerate(self.layers):
+            if ev is not None:
+                ev[0][i].record()
+            api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale, y_ar=y_ar, y_draft=y_dr,
+                                workspace=ws)
+            if ev is not None:
+                ev[1][i].record()
+        if ev is not None:
+            ev[2].record()
+        api.verify_block(self.v.p_logits, self.v.q_logits, self.v.draft_tokens, seed=1234,
+                         step=seed_step, out=self.out, workspace=self.vws)
+        if ev is not None:
+            ev[3].record()
+
+    def make_events(self):
+        n = len(self.layers)
+        mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        return ([mk() for _ in range(n)], [mk() for _ in range(n)], mk(), mk())
+
+    def op_times(self, ev):
+        gemm = sum(a.elapsed_time(b) for a, b in zip(ev[0], ev[1]))
+        return gemm, ev[2].elapsed_time(ev[3])
+
+    # host-resident inputs for the end-to-end measurement
+    def host_inputs(self):
+        pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+        xs = [pin(d.x) for _, d, *_ in self.layers]
+        return xs, pin(self.v.p_logits), pin(self.v.q_logits), pin(self.v.draft_tokens)
+
+    def e2e_step(self, host, step):
+        xs, hp, hq, hx = host
+        for (_, d, *_), hxv in zip(self.layers, xs):
+            d.x.copy_(hxv, non_blocking=True)
+        self.v.p_logits.copy_(hp, non_blocking=True)
+        self.v.q_logits.copy_(hq, non_blocking=True)
+        self.v.draft_tokens.copy_(hx, non_blocking=True)
+        self.step(step)
+        self.h_tok.copy_(self.out.out_tokens, non_blocking=True)
+        self.h_len.copy_(self.out.accepted_len, non_blocking=True)
+
+    def e2e_bytes(self, host):
+        xs, hp, hq, hx = host
+        h2d = sum(t.numel() * t.element_size() for t in xs) + sum(
+            t.numel() * t.element_size() for t in (hp, hq, hx))
+        d2h = self.out.out_tokens.numel() * 4 + self.out.accepted_len.numel() * 4
+        self.h_tok = torch.empty_like(self.out.out_tokens, device="cpu").pin_memory()
+        self.h_len = torch.empty_like(self.out.accepted_len, device="cpu").pin_memory()
+        return h2d, d2h
+
+    def emitted(self):
+        return int((self.out.accepted_len.clamp(min=0) + 1).sum().item())
+
+    def config(self):
+        return {"workload": self.name, "B": self.B, "K": self.K, "V": self.V,
+                "rows_M": self.M, "projections": [f"{n}:{d.x.shape[1]}->{d.W.shape[0]}"
+                                                  for n, d, *_ in self.layers],
+                "lora_rank": RANK, "lora_alpha": ALPHA, "logits": "bf16",
+                "l2": f"inputs larger than L2: {self.step_bytes / 1e9:.2f} GB distinct per step",
+                "seq_len": None, "global_batch": self.B, "parallelism": "replicas"}
+
+
+class SingleSequence(BatchedDecode):
+    """B = 1, K = 16: dual-path LM head over 17 rows, then verify its logits."""
+
+    name = "qwen3_8b_b1"
+
+    def __init__(self, dev, seed):
+        from lossless_decoding_b200 import api
+        from lossless_decoding_b200.inputs import dualpath_inputs
+        self.api = api
+        self.B, self.K, self.V = 1, K16, QWEN3_8B_VOCAB
+        self.M = self.K + 1
+        d = dualpath_inputs(M=self.M, d_in=QWEN3_8B_HIDDEN, d_out=self.V, r=RANK, alpha=ALPHA,
+                            seed=seed, device=dev)
+        y_ar = torch.empty((self.M, self.V), dtype=torch.bfloat16, device=dev)
+        y_dr = torch.empty_like(y_ar)
+        ws = torch.empty(api.dualpath_workspace_bytes(self.M, QWEN3_8B_HIDDEN, self.V, RANK,
+                                                      torch.bfloat16), dtype=torch.uint8,
+                         device=dev)
+        self.layers = [("lm_head", d, y_ar, y_dr, ws)]
+        g = torch.Generator(device=dev).manual_seed(seed)
+        self.drafts = torch.randint(0, self.V, (1, self.K), generator=g, device=dev,
+                                    dtype=torch.int32)
+        self.vws = torch.zeros(api.verify_workspace_bytes(1, self.K, self.V, torch.bfloat16),
+                               dtype=torch.uint8, device=dev)
+        self.out = api.VerifyResult(torch.empty((1, self.K + 1), dtype=torch.int32, device=dev),
+                                    torch.empty((1,), dtype=torch.int32, device=dev), None, None,
+                                    None)
+        self.gemm_flops = _dual_flops(self.M, QWEN3_8B_HIDDEN, self.V, RANK)
+        self.verify_bytes = (2 * self.K + 1) * self.V * 2 + self.K * 4 + (self.K + 2) * 4
+        self.launches_per_step = 4
+        self.step_bytes = (d.x.numel() + d.W.numel() + d.A.numel() + d.Bm.numel()) * 2
+
+    def step(self, seed_step, ev=None):
+        api = self.api
+        _, d, y_ar, y_dr, ws = self.layers[0]
+        if ev is not None:
+            ev[0][0].record()
+        api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale, y_ar=y_ar, y_draft=y_dr, workspace=ws)
+        if ev is not None:
+            ev[1][0].record()
+            ev[2].record()
+        p = y_ar.view(1, self.M, self.V)
+        q = y_dr[: self.K].view(1, self.K, self.V)
+        api.verify_block(p, q, self.drafts, seed=1234, step=seed_step, out=self.out,
+                         workspace=self.vws)
+        if ev is not None:
+            ev[3].record()
+
+    def host_inputs(self):
+        _, d, *_ = self.layers[0]
+        return [d.x.cpu().pin_memory()], self.drafts.cpu().pin_memory()
+
+    def e2e_step(self, host, step):
+        xs, hx = host
+        self.layers[0][1].x.copy_(xs[0], non_blocking=True)
+        self.drafts.copy_(hx, non_blocking=True)
+        self.step(step)
+        self.h_tok.copy_(self.out.out_tokens, non_blocking=True)
+        self.h_len.copy_(self.out.accepted_len, non_blocking=True)
+
+    def e2e_bytes(self, host):
+        xs, hx = host
+        h2d = xs[0].numel() * 2 + hx.numel() * 4
+        self.h_tok = torch.empty_like(self.out.out_tokens, device="cpu").pin_memory()
+        self.h_len = torch.empty_like(self.out.accepted_len, device="cpu").pin_memory()
+        return h2d, (self.K + 2) * 4
+
+    def config(self):
+        c = super().config()
+        c.update({"projections": [f"lm_head:{QWEN3_8B_HIDDEN}->{self.V}"], "rows_M": self.M,
+                  "l2": "W of the LM head (1.24 GB) is larger than L2"})
+        return c
+
+
+WORKLOADS = {c.name: c for c in (BatchedDecode, SingleSequence)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(workload: str, n_seq: int, seed: int = 0):
+    """Time the float64 oracle on n_seq sequences of the workload.
+
+    Returns (seconds, rows): the oracle's dual-path linear over the sample's
+    n_seq*K rows of every projection, then its verifier over the sample's
+    logits. Inputs are generated outside the timed part.
+    """
+    import oracle
+    from lossless_decoding_b200.inputs import dualpath_inputs, verify_inputs
+    K, V = K16, QWEN3_8B_VOCAB
+    M = n_seq * K
+    if workload == "qwen3_8b_b1":
+        projs = [("lm_head", QWEN3_8B_HIDDEN, V)]
+        M = K + 1
+    else:
+        projs = list(QWEN3_8B_PROJECTIONS)
+    dual = []
+    for i, (_, d_in, d_out) in enumerate(projs):
+        d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA, seed=seed + i)
+        dual.append((d.x.double().numpy(), d.W.double().numpy(), d.A.double().numpy(),
+                     d.Bm.double().numpy(), d.scale))
+    v = verify_inputs(n_seq, K, V, dtype="bf16", seed=seed)
+    p, q, x = v.p_logits.double().numpy(), v.q_logits.double().numpy(), v.draft_tokens.numpy()
+    t0 = time.perf_counter()
+    for (xx, W, A, Bm, s) in dual:
+        oracle.dualpath_linear(xx, W, A, Bm, s, round_t_to_bf16=True)
+    oracle.verify_block(p, q, x, seed=1234, step=0)
+    return time.perf_counter() - t0, n_seq * K
+
+
+def cpu_baseline(workload: str):
+    n_seq = 1 if workload == "qwen3_8b_b1" else 2
+    secs, rows = oracle_sample(workload, n_seq)
+    return {"value": rows / secs, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"{n_seq} sequence(s) x K={K16}: float64 oracle dual-path linear of "
+                       f"every projection over {rows if workload != 'qwen3_8b_b1' else K16 + 1} "
+                       f"rows + verifier over {n_seq}x{2 * K16 + 1} rows of {QWEN3_8B_VOCAB} "
+                       f"logits; {secs:.2f} s")}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    n_seq = 1
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, n_seq)
+    times = []
+    rows = 0
+    for i in range(args.steps):
+        s, rows = oracle_sample(args.workload, n_seq, seed=i)
+        times.append(s)
+    t = sum(times) / len(times)
+    value = rows / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_sequences": n_seq,
+                       "note": "float64 CPU oracle on host cores, one bounded sample per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{n_seq} sequence x K={K16} of {args.workload} per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+
+def run_ours(args):
+    world, rank, local = _dist()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    from lossless_decoding_b200 import api
+
+    wl = WORKLOADS[args.workload](dev, seed=17 + rank)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        wl.step(i)
+    api.device_fault_flags(clear=True)
+    barrier()
+
+    # ---- timed region: K steps, per-op events on the launching stream ----
+    events = [wl.make_events() for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    clocks.start()
+    barrier()
+    t0.record(stream)
+    for i in range(args.steps):
+        wl.step(args.warmup + i, events[i])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_step = max_over_ranks(ms_total / args.steps)
+    gemm_ms = [wl.op_times(e)[0] for e in events]
+    ver_ms = [wl.op_times(e)[1] for e in events]
+    emitted = wl.emitted()
+    faults = api.device_fault_flags(clear=True)
+
+    rows_per_step = wl.B * wl.K
+    value = world * rows_per_step / (ms_step / 1e3)
+    peaks = _peaks()
+    gemm_avg = sum(gemm_ms) / len(gemm_ms)
+    ver_avg = sum(ver_ms) / len(ver_ms)
+    gemm_tflops = wl.gemm_flops / (gemm_avg / 1e3) / 1e12
+    ver_gbs = wl.verify_bytes / (ver_avg / 1e3) / 1e9
+    dominant_gemm = gemm_avg >= ver_avg
+    roof_gemm = {"kernel": "dual-path linear (T split-K + reduce + dual tcgen05 GEMM)",
+                 "bound": "tensor", "achieved": gemm_tflops, "peak": peaks["bf16"],
+                 "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16"], "traffic": None,
+                 "peak_kind": f"bf16 dense burst, {peaks['src']}",
+                 "algorithmic_per_launch": wl.gemm_flops / len(wl.layers),
+                 "ms_per_step": gemm_avg}
+    roof_ver = {"kernel": "verify_kernel", "bound": "hbm", "achieved": ver_gbs,
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": ver_gbs / peaks["hbm"],
+                "traffic": None, "peak_kind": f"HBM copy, {peaks['src']}",
+                "algorithmic_per_launch": wl.verify_bytes, "ms_per_step": ver_avg}
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    host = wl.host_inputs()
+    h2d, d2h = wl.e2e_bytes(host)
+    e_steps = max(2, min(args.steps, 10))
+    for i in range(2):
+        wl.e2e_step(host, i)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e_steps):
+        wl.e2e_step(host, 100 + i)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps)
+    e2e_value = world * rows_per_step / (e2e_ms / 1e3)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded random weights, activations, logits)",
+            "config": wl.config(),
+            "emitted_tokens_per_s": world * emitted / (ms_step / 1e3),
+            "gemm_tflops": gemm_tflops, "verify_gbs": ver_gbs,
+            "roofline": roof_gemm if dominant_gemm else roof_ver,
+            "roofline_verify" if dominant_gemm else "roofline_gemm":
+                roof_ver if dominant_gemm else roof_gemm,
+            "gpu_launches": wl.launches_per_step * args.steps,
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "device_fault_flags": faults,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_decode_b64_k16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

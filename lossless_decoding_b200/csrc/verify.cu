@@ -18,7 +18,8 @@
 // sequence's 2K+1 rows, evaluates the accept tests, finds the first rejection
 // with a warp ballot, draws the residual (or bonus) token by inverse CDF over
 // one or two rows that were just streamed (mostly still in L2), writes the
-// outputs and resets the counter so the workspace can be reused.
+// outputs, and clears the partials and the counter it used, so the workspace
+// is zero-filled again when the call completes.
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -302,13 +303,15 @@ __device__ void finalize_sequence(const VerifyParams& P, int b, FinalShared& sh)
     sh.first_reject = K;
     sh.invalid = 0;
   }
-  // 1. merge slab partials of every row, slabs in index order.
+  // 1. merge slab partials of every row, slabs in index order, and clear them
+  //    so the workspace is zero-filled again when the call completes.
   for (int j = tid; j < R; j += kThreads) {
-    const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
+    Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
     float m = -INFINITY, z = 0.f;
     for (int s = 0; s < S; ++s) {
       const float2 v = __ldcg(reinterpret_cast<const float2*>(pp + s));
       merge(m, z, v.x, v.y);
+      pp[s] = Partial{0.f, 0.f};
     }
     sh.m[j] = m;
     sh.z[j] = z;
