@@ -106,6 +106,34 @@ int uno_verify_block(const void* p_logits, const void* q_logits, const int32_t* 
                      float* q_at_draft, float* row_lse, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/*
+ * uno_verify_block_noalloc -- the same verification, with no workspace
+ * argument and no allocation. The paper has no counterpart to this entry
+ * point; it exists for callers that cannot allocate device memory when they
+ * call, such as a plug-in whose host engine owns all device memory through its
+ * own pool, a latency-critical path that cannot afford cudaMalloc (it may
+ * synchronise the device), or a caller from another language with no device
+ * allocator at hand.
+ *
+ * Scratch: one fixed 4 MiB array in the library's device memory, reserved on
+ * every GPU that loads the library until the process exits. Calls whose
+ * uno_verify_workspace_bytes(B, K, V, dtype) exceeds 4 MiB are rejected with
+ * UNO_ERR_SIZE (for example B = 64, K = 16, V = 151936 needs about 51 KB).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call clears the part of the array it uses on `stream` before the
+ * kernel runs. All calls on a device share the array, so calls that may
+ * overlap on the GPU (different streams, or different host threads without
+ * ordering) race and corrupt each other's results: order them on one stream.
+ * The library calls no cudaMalloc, cudaFree or other allocating routine here.
+ * Arguments, outputs and errors are those of uno_verify_block.
+ */
+int uno_verify_block_noalloc(const void* p_logits, const void* q_logits,
+                             const int32_t* draft_tokens, int B, int K, int V, int dtype,
+                             uint64_t seed, uint64_t step, int32_t* out_tokens,
+                             int32_t* accepted_len, float* p_at_draft, float* q_at_draft,
+                             float* row_lse, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Dual-pathway linear (one pass over the frozen weight W)
  *

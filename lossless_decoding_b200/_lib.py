@@ -48,6 +48,9 @@ def _load() -> ctypes.CDLL:
     L.uno_verify_block.argtypes = [vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp, vp, vp, vp,
                                    vp, sz, vp]
     L.uno_verify_block.restype = i32
+    L.uno_verify_block_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp, vp,
+                                           vp, vp, vp]
+    L.uno_verify_block_noalloc.restype = i32
     L.uno_dualpath_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     L.uno_dualpath_workspace_bytes.restype = sz
     L.uno_dualpath_linear.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, vp, i32, i32, i32, i32,

@@ -134,6 +134,32 @@ def verify_block(p_logits: torch.Tensor, q_logits: torch.Tensor, draft_tokens: t
     return out
 
 
+def verify_block_noalloc(p_logits: torch.Tensor, q_logits: torch.Tensor,
+                         draft_tokens: torch.Tensor, seed: int, step: int, *,
+                         out: VerifyResult) -> VerifyResult:
+    """``uno_verify_block_noalloc``: the verifier without a workspace.
+
+    For callers that cannot allocate device memory at call time: the library
+    uses its own fixed 4 MiB scratch array and the caller supplies every
+    output buffer in ``out``. Calls on one device share that scratch, so keep
+    them on one stream. Problems needing more than 4 MiB of scratch raise
+    UnoError (UNO_ERR_SIZE).
+    """
+    B, K1, V = p_logits.shape
+    K = K1 - 1
+    dt = _dtype_code(p_logits)
+    dev = _check_cuda(p_logits, q_logits, draft_tokens, out.out_tokens, out.accepted_len,
+                      out.p_at_draft, out.q_at_draft, out.row_lse)
+    st = lib.uno_verify_block_noalloc(
+        _ptr(p_logits), _ptr(q_logits), _ptr(draft_tokens), B, K, V, dt,
+        ctypes.c_uint64(int(seed) & (2**64 - 1)), ctypes.c_uint64(int(step) & (2**64 - 1)),
+        _ptr(out.out_tokens), _ptr(out.accepted_len), _ptr(out.p_at_draft),
+        _ptr(out.q_at_draft), _ptr(out.row_lse), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_verify_block_noalloc")
+    return out
+
+
 # ---------------------------------------------------------------------------
 # dual-pathway linear
 # ---------------------------------------------------------------------------
