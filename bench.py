@@ -29,7 +29,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -71,53 +70,61 @@ def _dist():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls SM clock and clock-event reasons through NVML in a thread while
+    the timed region runs (read-only queries)."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device: torch.device, period_s: float = 0.002):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.err = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.nvml = None
+            self.err = f"NVML unavailable: {e}"
+
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                rs = get(self.h)
+                self.samples.append((sm, rs))
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(self.period)
 
     def start(self):
-        try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        import threading
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "NVML, polled during the timed region"}
 
 
 # ---------------------------------------------------------------------------
@@ -227,7 +234,7 @@ class BatchedDecode:
                                                   for n, d, *_ in self.layers],
                 "lora_rank": RANK, "lora_alpha": ALPHA, "logits": "bf16",
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e9:.2f} GB distinct per step",
-                "seq_len": None, "global_batch": self.B, "parallelism": "replicas"}
+                "global_batch": self.B, "parallelism": "replicas (one batch per GPU)"}
 
 
 class SingleSequence(BatchedDecode):
@@ -321,44 +328,58 @@ def _blas_threads():
         return 1
 
 
-def oracle_sample(workload: str, n_seq: int, seed: int = 0):
-    """Time the float64 oracle on n_seq sequences of the workload.
+_SAMPLES = {}
 
-    Returns (seconds, rows): the oracle's dual-path linear over the sample's
-    n_seq*K rows of every projection, then its verifier over the sample's
-    logits. Inputs are generated outside the timed part.
-    """
-    import oracle
+
+def _oracle_inputs(workload: str, n_seq: int):
+    """float64 inputs of a bounded sample (cached: generation is not timed)."""
+    key = (workload, n_seq)
+    if key in _SAMPLES:
+        return _SAMPLES[key]
     from lossless_decoding_b200.inputs import dualpath_inputs, verify_inputs
     K, V = K16, QWEN3_8B_VOCAB
-    M = n_seq * K
     if workload == "qwen3_8b_b1":
-        projs = [("lm_head", QWEN3_8B_HIDDEN, V)]
-        M = K + 1
+        projs, M = [("lm_head", QWEN3_8B_HIDDEN, V)], K + 1
     else:
-        projs = list(QWEN3_8B_PROJECTIONS)
+        projs, M = list(QWEN3_8B_PROJECTIONS), n_seq * K
     dual = []
     for i, (_, d_in, d_out) in enumerate(projs):
-        d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA, seed=seed + i)
+        d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA, seed=i)
         dual.append((d.x.double().numpy(), d.W.double().numpy(), d.A.double().numpy(),
                      d.Bm.double().numpy(), d.scale))
-    v = verify_inputs(n_seq, K, V, dtype="bf16", seed=seed)
-    p, q, x = v.p_logits.double().numpy(), v.q_logits.double().numpy(), v.draft_tokens.numpy()
+    v = verify_inputs(n_seq, K, V, dtype="bf16", seed=0)
+    _SAMPLES[key] = (dual, v.p_logits.double().numpy(), v.q_logits.double().numpy(),
+                     v.draft_tokens.numpy())
+    return _SAMPLES[key]
+
+
+def oracle_sample(workload: str, n_seq: int, step: int = 0):
+    """Time the float64 oracle on n_seq sequences of the workload.
+
+    The oracle's dual-path linear over the sample's rows of every projection,
+    then its verifier over the sample's 2K+1 logit rows per sequence. Returns
+    (seconds, verified rows).
+    """
+    import oracle
+    dual, p, q, x = _oracle_inputs(workload, n_seq)
     t0 = time.perf_counter()
     for (xx, W, A, Bm, s) in dual:
         oracle.dualpath_linear(xx, W, A, Bm, s, round_t_to_bf16=True)
-    oracle.verify_block(p, q, x, seed=1234, step=0)
-    return time.perf_counter() - t0, n_seq * K
+    oracle.verify_block(p, q, x, seed=1234, step=step)
+    return time.perf_counter() - t0, n_seq * K16
 
 
-def cpu_baseline(workload: str):
-    n_seq = 1 if workload == "qwen3_8b_b1" else 2
-    secs, rows = oracle_sample(workload, n_seq)
+def cpu_baseline(workload: str, min_seconds: float = 10.0, max_reps: int = 40):
+    n_seq = 1 if workload == "qwen3_8b_b1" else 8
+    secs = rows = reps = 0
+    while reps < max_reps and (secs < min_seconds or reps == 0):
+        s, r = oracle_sample(workload, n_seq, step=reps)
+        secs, rows, reps = secs + s, rows + r, reps + 1
     return {"value": rows / secs, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": (f"{n_seq} sequence(s) x K={K16}: float64 oracle dual-path linear of "
-                       f"every projection over {rows if workload != 'qwen3_8b_b1' else K16 + 1} "
-                       f"rows + verifier over {n_seq}x{2 * K16 + 1} rows of {QWEN3_8B_VOCAB} "
-                       f"logits; {secs:.2f} s")}
+            "sample": (f"{reps} x {n_seq} sequence(s), K={K16}: float64 oracle dual-path linear "
+                       f"of every projection over the sample's rows, then the verifier over "
+                       f"{n_seq}x{2 * K16 + 1} rows of {QWEN3_8B_VOCAB} logits; "
+                       f"{secs:.1f} s of oracle time")}
 
 
 def run_reference(args):
@@ -366,12 +387,12 @@ def run_reference(args):
     if rank != 0:
         return 0
     n_seq = 1
-    for _ in range(args.warmup):
-        oracle_sample(args.workload, n_seq)
+    for i in range(args.warmup):
+        oracle_sample(args.workload, n_seq, step=i)
     times = []
     rows = 0
     for i in range(args.steps):
-        s, rows = oracle_sample(args.workload, n_seq, seed=i)
+        s, rows = oracle_sample(args.workload, n_seq, step=args.warmup + i)
         times.append(s)
     t = sum(times) / len(times)
     value = rows / t
@@ -431,8 +452,7 @@ def run_ours(args):
     events = [wl.make_events() for _ in range(args.steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    clocks = ClockSampler(dev)
     clocks.start()
     barrier()
     t0.record(stream)
@@ -513,7 +533,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_decode_b64_k16")
