@@ -93,10 +93,8 @@ size_t uno_verify_workspace_bytes(int B, int K, int V, int dtype);
  * row_lse       [B, 2K+1]   float  log-sum-exp of every row: p rows 0..K,
  *                                  then q rows 0..K-1               (optional, NULL)
  * workspace     device scratch of at least uno_verify_workspace_bytes(B,K,V,dtype)
- *               bytes, 16-byte aligned. It must be zero-filled before its FIRST
- *               use; every call leaves it zero-filled again, so a workspace is
- *               reused without clearing. Two calls that share a workspace must
- *               be ordered on one stream.
+ *               bytes, 16-byte aligned; its contents on entry do not matter.
+ *               Two calls that share a workspace must be ordered on one stream.
  * stream        cudaStream_t
  * Returns UNO_OK or a negative uno_status.
  */
@@ -121,8 +119,8 @@ int uno_verify_block(const void* p_logits, const void* q_logits, const int32_t* 
  * UNO_ERR_SIZE (for example B = 64, K = 16, V = 151936 needs about 51 KB).
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
- * Every call clears the part of the array it uses on `stream` before the
- * kernel runs. All calls on a device share the array, so calls that may
+ * Every call clears the part of the array it uses on `stream` before its
+ * kernels run. All calls on a device share the array, so calls that may
  * overlap on the GPU (different streams, or different host threads without
  * ordering) race and corrupt each other's results: order them on one stream.
  * The library calls no cudaMalloc, cudaFree or other allocating routine here.

@@ -53,9 +53,8 @@ def _stream_handle(device: torch.device) -> int:
 class _Workspaces:
     """Grow-only device scratch buffers, one per (device, purpose).
 
-    The verifier's workspace must be zero on first use and is left zeroed by
-    every call, so it is allocated with zeros and reused as is. Calls that use
-    one cached workspace are ordered on the current stream of the caller.
+    The kernels do not depend on a workspace's previous contents. Calls that
+    use one cached workspace are ordered on the current stream of the caller.
     """
 
     def __init__(self):

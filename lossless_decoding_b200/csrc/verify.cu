@@ -8,18 +8,24 @@
 // from the verifier), with the standard speculative accept rule
 // u < p(x)/q(x) and residual max(0, p - q) that the pages cite.
 //
-// One launch does the whole step. Work unit = (sequence b, row j, slab s):
-// rows j = 0..K are the AR rows p_0..p_K, rows K+1..2K the draft rows
-// q_0..q_{K-1}; a slab is a contiguous stretch of one row's vocabulary. Each
-// CTA streams its slab once with 16-byte loads and keeps a running
-// (max, sum of exponentials) per thread, merged by warp shuffles and then
-// across warps. The CTA that completes a sequence's last unit (an atomic
-// counter per sequence, no waiting) merges the slab partials of the
-// sequence's 2K+1 rows, evaluates the accept tests, finds the first rejection
-// with a warp ballot, draws the residual (or bonus) token by inverse CDF over
-// one or two rows that were just streamed (mostly still in L2), writes the
-// outputs, and clears the partials and the counter it used, so the workspace
-// is zero-filled again when the call completes.
+// Two launches per call, with no waiting between CTAs:
+//  1. verify_stream_kernel streams every logit row once. One CTA per slab
+//     (about 64 KB of one row) issues 16-byte loads, four per thread in flight
+//     plus the next four prefetched, folds them into a running
+//     (reference, sum of 2^(x - reference)) in the log2 domain and writes one
+//     partial per slab.
+//     Nothing else happens on this path, so it runs at the speed of HBM.
+//  2. verify_draw_kernel runs SD CTAs per sequence. Each CTA merges the slab
+//     partials of the sequence's 2K+1 rows in a fixed order, evaluates the
+//     accept tests with Philox uniforms and finds the first rejection by
+//     ballot -- every CTA of a sequence computes the same decision from the
+//     same data, so none waits for another -- then sums the residual weights
+//     max(0, p_n - q_n) (or the bonus row p_K) over its range of fixed-size
+//     vocabulary chunks. The CTA that completes a sequence (atomic counter)
+//     takes the float64 running sum of the chunk sums, finds the chunk where
+//     u' * total is crossed, scans it with warp prefix sums to pick the token
+//     and writes the outputs.
+#include <atomic>
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -35,16 +41,21 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;            // 16-byte vectors per thread per iteration
+constexpr int kStreamCtasPerSm = 4;
+constexpr int kRound = 4;                 // 16-byte vectors per thread per round
+constexpr int kSlabBytes = 65536;         // target bytes streamed by one CTA
+constexpr int kMinSlabBytes = kThreads * 16;
 constexpr int kMaxK = 256;
 constexpr int kMaxRows = 2 * kMaxK + 1;
-constexpr int kMaxChunks = 2048;      // inverse-CDF chunk sums held in shared memory
-constexpr int kMinVecPerSlab = kThreads * kUnroll;  // at least one full iteration
+constexpr int kChunkMin = 256;            // vocabulary entries per inverse-CDF chunk
+constexpr int kMaxChunks = 4096;          // chunks per row (the chunk length grows beyond)
+constexpr int kChunksPerDrawCta = 16;
+constexpr int kSizingSms = 148;           // fixed, so the workspace size is device-independent
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct Partial {
-  float m;  // max over the slab of l * log2(e)
+  float m;  // reference in the log2 domain (see fold)
   float z;  // sum over the slab of 2^(l * log2(e) - m)
 };
 
@@ -52,7 +63,11 @@ struct VerifyParams {
   const void* p_logits;
   const void* q_logits;
   const int32_t* draft;
-  int B, K, V, S;
+  int B, K, V;
+  int S;          // slabs per row
+  int nchunks;    // inverse-CDF chunks per row
+  int chunk_len;  // vocabulary entries per chunk
+  int SD;         // draw CTAs per sequence
   uint64_t seed, step;
   int32_t* out_tokens;
   int32_t* accepted_len;
@@ -60,10 +75,12 @@ struct VerifyParams {
   float* q_at_draft;
   float* row_lse;
   Partial* partials;  // [B][2K+1][S]
-  int* counters;      // [B]
+  float* chunk_sums;  // [B][nchunks]
+  int* draw_count;    // [B], set to 0 by the streaming launch
+  int* max_pos;       // [B], 1 + largest positive-weight index; set to 0 likewise
 };
 
-// ---- element access --------------------------------------------------------
+// ---- element access -----------------------------------------------------------
 
 template <typename T>
 struct Elem;
@@ -96,7 +113,7 @@ struct Elem<float> {
   }
 };
 
-// ---- (max, sum-exp) algebra in the log2 domain ------------------------------
+// ---- (max, sum-exp) algebra in the log2 domain ----------------------------------
 
 __device__ __forceinline__ void merge(float& m, float& z, float m2, float z2) {
   const float mm = fmaxf(m, m2);
@@ -107,32 +124,58 @@ __device__ __forceinline__ void merge(float& m, float& z, float m2, float z2) {
   z = a + b;
 }
 
-// Fold n values (natural-log logits) into the running (m, z).
+// Fold N natural-log logits into the running (m, z). m is a reference, not
+// necessarily the running maximum: z = sum of 2^(x - m) over the values seen,
+// x = l * log2(e). The common path adds the group's sum against the current
+// reference; only when that sum reaches 2^70 (or is not finite, e.g. while m
+// is still -inf) does the group move the reference to its own maximum. So every
+// term stays below 2^70 and z below 2^84, and a term that underflows against
+// the reference is below 2^-126 of it, hence negligible against the true
+// maximum. Merges and p = 2^(x - m) / z do not depend on which reference is
+// kept.
 template <int N>
-__device__ __forceinline__ void fold(float& m, float& z, const float* v) {
-  float cm = v[0];
-#pragma unroll
-  for (int e = 1; e < N; ++e) cm = fmaxf(cm, v[e]);
-  if (cm == -INFINITY) return;
-  const float cm2 = cm * kLog2e;
-  if (cm2 > m) {
-    z *= uno::ex2(m - cm2);  // m = -inf gives 0
-    m = cm2;
-  }
+__device__ __forceinline__ float sum_ex2(const float* v, float m) {
   float t[N];
 #pragma unroll
   for (int e = 0; e < N; ++e) t[e] = uno::ex2(fmaf(v[e], kLog2e, -m));
-  // pairwise sum of the chunk, then one add into the running total
 #pragma unroll
   for (int w = 1; w < N; w *= 2) {
 #pragma unroll
     for (int e = 0; e + w < N; e += 2 * w) t[e] += t[e + w];
   }
-  z += t[0];
+  return t[0];
 }
 
-// Geometry of one row: a scalar head up to the first 16-byte boundary, then
-// nvec full vectors, then a scalar tail.
+template <int N>
+__device__ __forceinline__ void fold(float& m, float& z, const float* v) {
+  const float s = sum_ex2<N>(v, m);
+  if (s < 0x1p70f) {  // false for inf and NaN
+    z += s;
+    return;
+  }
+  float gm = v[0];
+#pragma unroll
+  for (int e = 1; e < N; ++e) gm = fmaxf(gm, v[e]);
+  if (gm == -INFINITY) return;
+  gm *= kLog2e;
+  if (gm > m) {
+    z = (m == -INFINITY) ? 0.f : z * uno::ex2(m - gm);
+    m = gm;
+  }
+  z += sum_ex2<N>(v, m);
+}
+
+__device__ __forceinline__ void warp_merge(float& m, float& z) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+    const float z2 = __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    merge(m, z, m2, z2);
+  }
+}
+
+// A row is a scalar head up to the first 16-byte boundary, nvec full 16-byte
+// vectors, then a scalar tail.
 struct RowGeom {
   int head, nvec, tail;
 };
@@ -147,6 +190,8 @@ __device__ __forceinline__ RowGeom row_geom(size_t elem_offset, int V) {
   return {head, nvec, V - head - nvec * kVec};
 }
 
+// Row j of sequence b: j = 0..K are the AR rows p_0..p_K, j = K+1..2K the draft
+// rows q_0..q_{K-1}.
 template <typename T>
 __device__ __forceinline__ const T* row_ptr(const VerifyParams& P, int b, int j, size_t* off) {
   const int K = P.K;
@@ -163,163 +208,318 @@ __device__ __forceinline__ const T* row_ptr(const VerifyParams& P, int b, int j,
   return base + *off;
 }
 
-// ---- block reductions -------------------------------------------------------
+// ---- launch 1: streaming ----------------------------------------------------------------
 
-__device__ __forceinline__ void warp_merge(float& m, float& z) {
+template <typename T>
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
+    verify_stream_kernel(const VerifyParams P) {
+  constexpr int kVec = Elem<T>::kVec;
+  __shared__ float red_m[kWarps], red_z[kWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = 2 * P.K + 1;
+  const int s = blockIdx.x % P.S;
+  const int rj = blockIdx.x / P.S;
+  const int j = rj % R, b = rj / R;
+
+  if (s == 0 && j == 0 && tid == 0) {  // counters the draw launch relies on
+    P.draw_count[b] = 0;
+    P.max_pos[b] = 0;
+  }
+
+  size_t off;
+  const T* row = row_ptr<T>(P, b, j, &off);
+  const RowGeom g = row_geom<T>(off, P.V);
+  const int per = (g.nvec + P.S - 1) / P.S;
+  const int v0 = min(s * per, g.nvec), v1 = min(v0 + per, g.nvec);
+  const uint4* vrow = reinterpret_cast<const uint4*>(row + g.head);
+
+  float m = -INFINITY, z = 0.f;
+  constexpr int kStep = kRound * kThreads;
+  const int full = (v1 - v0) / kStep;  // rounds in which every thread has kRound vectors
+  uint4 cur[kRound], nxt[kRound];
+  if (full > 0) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-    const float z2 = __shfl_xor_sync(0xFFFFFFFFu, z, o);
-    merge(m, z, m2, z2);
+    for (int k = 0; k < kRound; ++k) cur[k] = __ldg(vrow + v0 + k * kThreads + tid);
+  }
+  for (int r = 0; r < full; ++r) {
+    const int nb = v0 + (r + 1) * kStep;
+    if (r + 1 < full) {
+#pragma unroll
+      for (int k = 0; k < kRound; ++k) nxt[k] = __ldg(vrow + nb + k * kThreads + tid);
+    }
+#pragma unroll
+    for (int k = 0; k < kRound; k += 2) {
+      float f[2 * kVec];
+      Elem<T>::unpack(cur[k], f);
+      Elem<T>::unpack(cur[k + 1], f + kVec);
+      fold<2 * kVec>(m, z, f);
+    }
+#pragma unroll
+    for (int k = 0; k < kRound; ++k) cur[k] = nxt[k];
+  }
+  // remainder: fewer than kRound vectors per thread
+  for (int idx = v0 + full * kStep + tid; idx < v1; idx += kThreads) {
+    float f[kVec];
+    Elem<T>::unpack(__ldg(vrow + idx), f);
+    fold<kVec>(m, z, f);
+  }
+  if (s == 0 && tid < g.head) {
+    const float v = Elem<T>::at(row, tid);
+    fold<1>(m, z, &v);
+  }
+  if (s == P.S - 1 && tid < g.tail) {
+    const float v =
+        Elem<T>::at(row, static_cast<size_t>(g.head) + static_cast<size_t>(g.nvec) * kVec + tid);
+    fold<1>(m, z, &v);
+  }
+  warp_merge(m, z);
+  if (lane == 0) {
+    red_m[warp] = m;
+    red_z[warp] = z;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    m = (lane < kWarps) ? red_m[lane] : -INFINITY;
+    z = (lane < kWarps) ? red_z[lane] : 0.f;
+    warp_merge(m, z);
+    if (lane == 0) P.partials[static_cast<size_t>(blockIdx.x)] = Partial{m, z};
   }
 }
 
-// ---- the draw: inverse CDF over one row's weights ---------------------------
+// ---- launch 2: decision and draw ----------------------------------------------------------
 
 struct DrawShared {
-  float chunk_sum[kMaxChunks];
-  double t;          // threshold u' * total
-  int chunk;         // chunk where the running sum crosses t
-  int last_pos;      // largest index with positive weight
-  int token;
+  float row_m[kMaxRows], row_z[kMaxRows];
+  double scan[kThreads];
+  double total;
+  int first_reject, invalid, last_pos, is_last, chunk, token;
 };
 
-// Weight of token v. mode 0: max(0, p(v) - q(v)); mode 1: p(v).
+struct DrawRows {
+  int mode;  // 0: residual max(0, p_n - q_n); 1: the row p_n itself
+  float mp, izp, mq, izq;
+  float c;   // residual sign threshold (log2 domain)
+};
+
+// Weight of token v. mode 0: max(0, p(v) - q(v)), skipping both exponentials
+// where the log-domain test shows p(v) < q(v) by a clear margin; mode 1: p(v).
 template <typename T>
-__device__ __forceinline__ float weight(int mode, const T* rp, const T* rq, int v, float mp,
-                                        float izp, float mq, float izq) {
-  const float pv = uno::ex2(fmaf(Elem<T>::at(rp, v), kLog2e, -mp)) * izp;
-  if (mode) return pv;
-  const float qv = uno::ex2(fmaf(Elem<T>::at(rq, v), kLog2e, -mq)) * izq;
+__device__ __forceinline__ float weight(const DrawRows& d, const T* rp, const T* rq, int v) {
+  const float lp = Elem<T>::at(rp, v) * kLog2e;
+  if (d.mode) return uno::ex2(lp - d.mp) * d.izp;
+  const float lq = Elem<T>::at(rq, v) * kLog2e;
+  if (lp - lq < d.c - 1e-3f) return 0.f;
+  const float pv = uno::ex2(lp - d.mp) * d.izp;
+  const float qv = uno::ex2(lq - d.mq) * d.izq;
   return fmaxf(0.f, pv - qv);
 }
 
-// All threads of the CTA call this. Returns the drawn token, or -1 when every
-// weight is zero.
+// Sums of chunks c0 + w0, c0 + w0 + wstep, ... (< c1) of the draw rows of
+// sequence b, one warp per chunk, stored to the workspace. Returns this lane's
+// largest positive-weight index, or -1. When both rows are 16-byte aligned and
+// V and the chunk length are whole vectors, each lane loads 16-byte vectors,
+// all of the warp's chunks at once; otherwise it falls back to scalar loads.
 template <typename T>
-__device__ int draw_token(DrawShared& sh, int mode, const T* rp, const T* rq, int V, float mp,
-                          float izp, float mq, float izq, float u) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int chunk_len = (V + kMaxChunks - 1) / kMaxChunks;
-  chunk_len = chunk_len < 256 ? 256 : ((chunk_len + 31) / 32) * 32;
-  const int nchunks = (V + chunk_len - 1) / chunk_len;
-
-  if (tid == 0) sh.last_pos = -1;
-  __syncthreads();
-  // Phase A: every chunk's weight sum (one warp per chunk, fixed order inside).
-  int my_last = -1;
-  for (int c = warp; c < nchunks; c += kWarps) {
-    const int v0 = c * chunk_len;
-    const int v1 = min(v0 + chunk_len, V);
+__device__ int chunk_sums(const VerifyParams& P, int b, const DrawRows& d, const T* rp,
+                          const T* rq, int c0, int c1, int w0, int wstep) {
+  constexpr int kVec = Elem<T>::kVec;
+  constexpr int kMaxVecs = 4;  // vectors per lane held in flight per row
+  const int lane = threadIdx.x & 31;
+  int last = -1;
+  const int vpl = P.chunk_len / (32 * kVec);  // vectors per lane per chunk
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(rp) | reinterpret_cast<uintptr_t>(rq)) & 15) == 0 &&
+                      (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0 && vpl >= 1;
+  if (vec_ok) {
+    const uint4* vp = reinterpret_cast<const uint4*>(rp);
+    const uint4* vq = reinterpret_cast<const uint4*>(rq);
+    const int nvec_row = P.V / kVec;
+    for (int c = c0 + w0; c < c1; c += wstep) {
+      float s = 0.f;
+      for (int q0 = 0; q0 < vpl; q0 += kMaxVecs) {
+        uint4 a[kMaxVecs], bq[kMaxVecs];
+        int vi[kMaxVecs];
+#pragma unroll
+        for (int k = 0; k < kMaxVecs; ++k) {
+          vi[k] = c * (P.chunk_len / kVec) + (q0 + k) * 32 + lane;
+          const bool in = (q0 + k < vpl) && (vi[k] < nvec_row);
+          a[k] = in ? __ldg(vp + vi[k]) : make_uint4(0, 0, 0, 0);
+          bq[k] = (in && d.mode == 0) ? __ldg(vq + vi[k]) : make_uint4(0, 0, 0, 0);
+          if (!in) vi[k] = -1;
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxVecs; ++k) {
+          if (vi[k] < 0) continue;
+          float fp[kVec], fq[kVec];
+          Elem<T>::unpack(a[k], fp);
+          Elem<T>::unpack(bq[k], fq);
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) {
+            float w;
+            const float lp = fp[e] * kLog2e;
+            if (d.mode) {
+              w = uno::ex2(lp - d.mp) * d.izp;
+            } else {
+              const float lq = fq[e] * kLog2e;
+              w = (lp - lq < d.c - 1e-3f)
+                      ? 0.f
+                      : fmaxf(0.f, uno::ex2(lp - d.mp) * d.izp - uno::ex2(lq - d.mq) * d.izq);
+            }
+            s += w;
+            if (w > 0.f) last = max(last, vi[k] * kVec + e);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+      if (lane == 0) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = s;
+    }
+    return last;
+  }
+  for (int c = c0 + w0; c < c1; c += wstep) {
+    const int v0 = c * P.chunk_len;
+    const int v1 = min(v0 + P.chunk_len, P.V);
     float s = 0.f;
-    for (int v = v0 + lane; v < v1; v += 32) {
-      const float w = weight<T>(mode, rp, rq, v, mp, izp, mq, izq);
-      s += w;
-      if (w > 0.f) my_last = v;
+    for (int base = v0; base < v1; base += 32 * 8) {
+      float w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int v = base + k * 32 + lane;
+        w[k] = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        s += w[k];
+        if (w[k] > 0.f) last = max(last, base + k * 32 + lane);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (lane == 0) sh.chunk_sum[c] = s;
+    if (lane == 0) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = s;
   }
-  if (my_last >= 0) atomicMax(&sh.last_pos, my_last);
-  __syncthreads();
-  if (sh.last_pos < 0) return -1;  // all weights zero (uniform value for every thread)
-
-  // Phase B (warp 0): running sum of chunk sums in float64; find the chunk.
-  if (warp == 0) {
-    const int per = (nchunks + 31) / 32;
-    const int c0 = lane * per, c1 = min(c0 + per, nchunks);
-    double mine = 0.0;
-    for (int c = c0; c < c1; ++c) mine += static_cast<double>(sh.chunk_sum[c]);
-    double incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double up = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += up;
-    }
-    const double total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    const double t = static_cast<double>(u) * total;
-    double run = incl - mine;  // exclusive prefix of this lane's block
-    int found = INT_MAX;
-    for (int c = c0; c < c1; ++c) {
-      const double nxt = run + static_cast<double>(sh.chunk_sum[c]);
-      if (nxt > t) { found = c; break; }
-      run = nxt;
-    }
-    const unsigned hit = __ballot_sync(0xFFFFFFFFu, found != INT_MAX);
-    const int src = hit ? (__ffs(hit) - 1) : 31;
-    const int chunk = __shfl_sync(0xFFFFFFFFu, found, src);
-    if (lane == 0) {
-      sh.t = t;
-      sh.chunk = (chunk == INT_MAX) ? -1 : chunk;
-      sh.token = -1;
-    }
-    // Phase C: scan inside the chosen chunk.
-    const int ch = __shfl_sync(0xFFFFFFFFu, chunk, 0);
-    if (ch != INT_MAX) {
-      double carry = 0.0;
-      for (int c = 0; c < ch; ++c) carry += static_cast<double>(sh.chunk_sum[c]);
-      const int v0 = ch * chunk_len, v1 = min(v0 + chunk_len, V);
-      int tok = -1, last_pos_in_chunk = -1;
-      for (int base = v0; base < v1 && tok < 0; base += 32) {
-        const int v = base + lane;
-        const float w = (v < v1) ? weight<T>(mode, rp, rq, v, mp, izp, mq, izq) : 0.f;
-        float incl_w = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float up = __shfl_up_sync(0xFFFFFFFFu, incl_w, o);
-          if (lane >= o) incl_w += up;
-        }
-        const bool cross = (v < v1) && (w > 0.f) && (carry + static_cast<double>(incl_w) > t);
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, cross);
-        const unsigned pos = __ballot_sync(0xFFFFFFFFu, (v < v1) && (w > 0.f));
-        if (pos) last_pos_in_chunk = base + 31 - __clz(pos);
-        if (m) tok = base + __ffs(m) - 1;
-        carry += static_cast<double>(__shfl_sync(0xFFFFFFFFu, incl_w, 31));
-      }
-      if (lane == 0) sh.token = (tok >= 0) ? tok : last_pos_in_chunk;
-    }
-  }
-  __syncthreads();
-  const int tok = sh.token;
-  return tok >= 0 ? tok : sh.last_pos;
+  return last;
 }
 
-// ---- finalize (runs in the CTA that completes sequence b) --------------------
+// Per-thread block sums of the chunk sums and their exclusive running sum in
+// index order (float64): thread t owns chunks [c0, c1); sh.scan[t] receives the
+// sum of all chunks before c0 and sh.total the sum of all chunks.
+__device__ void prefix_chunks(const float* cs, int c0, int c1, DrawShared& sh) {
+  const int tid = threadIdx.x;
+  double mine = 0.0;
+  for (int c = c0; c < c1; ++c) mine += static_cast<double>(__ldcg(cs + c));
+  sh.scan[tid] = mine;
+  __syncthreads();
+  if (tid == 0) {
+    double run = 0.0;
+    for (int t = 0; t < kThreads; ++t) {
+      const double x = sh.scan[t];
+      sh.scan[t] = run;
+      run += x;
+    }
+    sh.total = run;
+    sh.chunk = INT_MAX;
+    sh.token = -1;
+  }
+  __syncthreads();
+}
 
-struct FinalShared {
-  float m[kMaxRows];
-  float z[kMaxRows];
-  int first_reject;
-  int invalid;
-  DrawShared draw;
-};
+// Final inverse-CDF step of sequence b (the whole CTA); returns the token.
+template <typename T>
+__device__ int finish_draw(const VerifyParams& P, int b, int n, DrawRows d, const T* rp,
+                           const T* rq, DrawShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
+  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, n).y);
+  const int per = (P.nchunks + kThreads - 1) / kThreads;
+  const int c0 = min(tid * per, P.nchunks), c1 = min(c0 + per, P.nchunks);
+  int last_pos = __ldcg(P.max_pos + b) - 1;
+  prefix_chunks(cs, c0, c1, sh);
+  if (sh.total <= 0.0 && d.mode == 0) {
+    // The residual mass is zero (possible only through rounding): draw from p_n.
+    d.mode = 1;
+    rq = rp;
+    if (tid == 0) sh.last_pos = -1;
+    __syncthreads();
+    const int l = chunk_sums<T>(P, b, d, rp, rp, 0, P.nchunks, warp, kWarps);
+    if (l >= 0) atomicMax(&sh.last_pos, l);
+    __threadfence();
+    __syncthreads();
+    last_pos = sh.last_pos;
+    prefix_chunks(cs, c0, c1, sh);
+  }
+  const double t = static_cast<double>(u) * sh.total;
+  {
+    double run = sh.scan[tid];
+    for (int c = c0; c < c1; ++c) {
+      const double nxt = run + static_cast<double>(__ldcg(cs + c));
+      if (nxt > t) {
+        atomicMin(&sh.chunk, c);
+        break;
+      }
+      run = nxt;
+    }
+  }
+  __syncthreads();
+  const int ch = sh.chunk;
+  if (warp == 0 && ch != INT_MAX) {
+    double carry = 0.0;
+    for (int c = lane; c < ch; c += 32) carry += static_cast<double>(__ldcg(cs + c));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) carry += __shfl_xor_sync(0xFFFFFFFFu, carry, o);
+    const int v0 = ch * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
+    int tok = -1, last_in_chunk = -1;
+    for (int base = v0; base < v1 && tok < 0; base += 32) {
+      const int v = base + lane;
+      const float w = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
+      float incl = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float up = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += up;
+      }
+      const bool cross = (w > 0.f) && (carry + static_cast<double>(incl) > t);
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, cross);
+      const unsigned pos = __ballot_sync(0xFFFFFFFFu, w > 0.f);
+      if (pos) last_in_chunk = base + 31 - __clz(pos);
+      if (hit) tok = base + __ffs(hit) - 1;
+      carry += static_cast<double>(__shfl_sync(0xFFFFFFFFu, incl, 31));
+    }
+    if (lane == 0) sh.token = (tok >= 0) ? tok : last_in_chunk;
+  }
+  __syncthreads();
+  return (sh.token >= 0) ? sh.token : last_pos;
+}
 
 template <typename T>
-__device__ void finalize_sequence(const VerifyParams& P, int b, FinalShared& sh) {
+__global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParams P) {
+  __shared__ DrawShared sh;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int b = blockIdx.x / P.SD, du = blockIdx.x % P.SD;
   const int K = P.K, R = 2 * K + 1, S = P.S, V = P.V;
-  const int tid = threadIdx.x;
+  const bool reporter = (du == 0);  // writes the per-position and per-row outputs
+
+  // 1. row statistics: merge the slab partials of every row in slab order
+  for (int j = tid; j < R; j += kThreads) {
+    const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
+    float m = -INFINITY, z = 0.f;
+    for (int s0 = 0; s0 < S; s0 += 8) {  // eight loads in flight, merged in slab order
+      Partial v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? pp[s0 + k] : Partial{-INFINITY, 0.f};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) merge(m, z, v[k].m, v[k].z);
+    }
+    sh.row_m[j] = m;
+    sh.row_z[j] = z;
+    if (reporter && P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
+  }
   if (tid == 0) {
     sh.first_reject = K;
     sh.invalid = 0;
-  }
-  // 1. merge slab partials of every row, slabs in index order, and clear them
-  //    so the workspace is zero-filled again when the call completes.
-  for (int j = tid; j < R; j += kThreads) {
-    Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
-    float m = -INFINITY, z = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(pp + s));
-      merge(m, z, v.x, v.y);
-      pp[s] = Partial{0.f, 0.f};
-    }
-    sh.m[j] = m;
-    sh.z[j] = z;
-    if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
+    sh.last_pos = -1;
   }
   __syncthreads();
 
-  // 2. accept tests, one thread per drafted position; first rejection by ballot.
+  // 2. accept tests, one thread per position; first rejection by ballot
   for (int i0 = 0; i0 < K; i0 += kThreads) {
     const int i = i0 + tid;
     bool rejected = false;
@@ -331,138 +531,73 @@ __device__ void finalize_sequence(const VerifyParams& P, int b, FinalShared& sh)
         size_t off;
         const T* rp = row_ptr<T>(P, b, i, &off);
         const T* rq = row_ptr<T>(P, b, K + 1 + i, &off);
-        const float pp = uno::ex2(fmaf(Elem<T>::at(rp, x), kLog2e, -sh.m[i])) / sh.z[i];
-        const float qq =
-            uno::ex2(fmaf(Elem<T>::at(rq, x), kLog2e, -sh.m[K + 1 + i])) / sh.z[K + 1 + i];
+        const float pp = uno::ex2(fmaf(Elem<T>::at(rp, x), kLog2e, -sh.row_m[i])) / sh.row_z[i];
+        const float qq = uno::ex2(fmaf(Elem<T>::at(rq, x), kLog2e, -sh.row_m[K + 1 + i])) /
+                         sh.row_z[K + 1 + i];
         const uint4 w = uno::verify_block_words(P.seed, P.step, b, i);
-        const float u = uno::uniform24(w.x);
-        rejected = !(u * qq < pp);
-        if (P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
-        if (P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
+        rejected = !(uno::uniform24(w.x) * qq < pp);
+        if (reporter && P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
+        if (reporter && P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
       }
     }
     const unsigned ballot = __ballot_sync(0xFFFFFFFFu, rejected);
-    if (ballot && (tid & 31) == 0) atomicMin(&sh.first_reject, i0 + (tid & ~31) + __ffs(ballot) - 1);
+    if (ballot && (tid & 31) == 0)
+      atomicMin(&sh.first_reject, i0 + (tid & ~31) + __ffs(ballot) - 1);
   }
   __syncthreads();
-
   const int n = sh.first_reject;
+  const bool invalid = sh.invalid != 0;
   int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
-  if (sh.invalid) {
-    for (int i = tid; i <= K; i += kThreads) out[i] = -1;
-    if (tid == 0) P.accepted_len[b] = -1;
-    return;
-  }
 
-  // 3. residual (n < K) or bonus (n == K) draw with u'_n.
+  // 3. this CTA's share of the chunk sums of the draw rows
+  DrawRows d{};
   size_t off;
   const T* rp = row_ptr<T>(P, b, n, &off);
-  const T* rq = (n < K) ? row_ptr<T>(P, b, K + 1 + n, &off) : rp;
-  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, n).y);
-  const float mp = sh.m[n], izp = 1.f / sh.z[n];
-  const float mq = (n < K) ? sh.m[K + 1 + n] : 0.f;
-  const float izq = (n < K) ? 1.f / sh.z[K + 1 + n] : 0.f;
-  int y = draw_token<T>(sh.draw, (n < K) ? 0 : 1, rp, rq, V, mp, izp, mq, izq, u);
-  if (y < 0) y = draw_token<T>(sh.draw, 1, rp, rp, V, mp, izp, 0.f, 0.f, u);  // empty residual
+  const T* rq = rp;
+  d.mode = (n < K) ? 0 : 1;
+  d.mp = sh.row_m[n];
+  d.izp = 1.f / sh.row_z[n];
+  if (n < K) {
+    rq = row_ptr<T>(P, b, K + 1 + n, &off);
+    d.mq = sh.row_m[K + 1 + n];
+    d.izq = 1.f / sh.row_z[K + 1 + n];
+    d.c = (sh.row_m[n] + log2f(sh.row_z[n])) - (sh.row_m[K + 1 + n] + log2f(sh.row_z[K + 1 + n]));
+  }
+  if (invalid) {
+    if (reporter) {
+      for (int i = tid; i <= K; i += kThreads) out[i] = -1;
+      if (tid == 0) P.accepted_len[b] = -1;
+    }
+  } else {
+    const int c0 = du * kChunksPerDrawCta;
+    const int c1 = min(c0 + kChunksPerDrawCta, P.nchunks);
+    const int l = chunk_sums<T>(P, b, d, rp, rq, c0, c1, warp, kWarps);
+    if (l >= 0) atomicMax(&sh.last_pos, l);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (sh.last_pos >= 0) atomicMax(P.max_pos + b, sh.last_pos + 1);
+    __threadfence();
+    sh.is_last = (atomicAdd(P.draw_count + b, 1) == P.SD - 1);
+  }
+  __syncthreads();
+  if (!sh.is_last || invalid) return;
 
-  // 4. outputs.
+  // 4. the CTA that completes the sequence picks the token and writes outputs
+  __threadfence();
+  const int y = finish_draw<T>(P, b, n, d, rp, rq, sh);
   const int32_t* x = P.draft + static_cast<size_t>(b) * K;
   for (int i = tid; i <= K; i += kThreads) out[i] = (i < n) ? x[i] : ((i == n) ? y : -1);
   if (tid == 0) P.accepted_len[b] = n;
 }
 
-// ---- the kernel ----------------------------------------------------------------
+// ---- host side -----------------------------------------------------------------------
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 4) verify_kernel(const VerifyParams P) {
-  constexpr int kVec = Elem<T>::kVec;
-  __shared__ FinalShared sh_final;
-  __shared__ float red_m[kWarps], red_z[kWarps];
-  __shared__ int is_last;
-
-  const int R = 2 * P.K + 1;
-  const int unit = blockIdx.x;
-  const int s = unit % P.S;
-  const int rj = unit / P.S;
-  const int j = rj % R;
-  const int b = rj / R;
-  const int tid = threadIdx.x;
-
-  size_t off;
-  const T* row = row_ptr<T>(P, b, j, &off);
-  const RowGeom g = row_geom<T>(off, P.V);
-  const int per = (g.nvec + P.S - 1) / P.S;
-  const int v_begin = min(s * per, g.nvec);
-  const int v_end = min(v_begin + per, g.nvec);
-
-  float m = -INFINITY, z = 0.f;
-  const uint4* vrow = reinterpret_cast<const uint4*>(row + g.head);
-  for (int base = v_begin; base < v_end; base += kThreads * kUnroll) {
-    uint4 raw[kUnroll];
-#pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int idx = base + k * kThreads + tid;
-      raw[k] = (idx < v_end) ? __ldg(vrow + idx)
-                             : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
-    }
-    float f[kUnroll * kVec];
-#pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int idx = base + k * kThreads + tid;
-      Elem<T>::unpack(raw[k], f + k * kVec);
-      if (idx >= v_end) {
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) f[k * kVec + e] = -INFINITY;
-      }
-    }
-    fold<kUnroll * kVec>(m, z, f);
-  }
-  // scalar head (first slab) and tail (last slab)
-  if (s == 0 && tid < g.head) {
-    const float v = Elem<T>::at(row, tid);
-    fold<1>(m, z, &v);
-  }
-  if (s == P.S - 1 && tid < g.tail) {
-    const float v = Elem<T>::at(row, static_cast<size_t>(g.head) + static_cast<size_t>(g.nvec) * kVec + tid);
-    fold<1>(m, z, &v);
-  }
-
-  warp_merge(m, z);
-  const int lane = tid & 31, warp = tid >> 5;
-  if (lane == 0) {
-    red_m[warp] = m;
-    red_z[warp] = z;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float bm = red_m[0], bz = red_z[0];
-    for (int w = 1; w < kWarps; ++w) merge(bm, bz, red_m[w], red_z[w]);
-    P.partials[static_cast<size_t>(rj) * P.S + s] = Partial{bm, bz};
-    __threadfence();
-    const int prev = atomicAdd(P.counters + b, 1);
-    is_last = (prev == R * P.S - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  finalize_sequence<T>(P, b, sh_final);
-  if (tid == 0) P.counters[b] = 0;  // leave the workspace zero-filled
-}
-
-// ---- host side -----------------------------------------------------------------
-
-int choose_slabs(int B, int K, int V, int dtype) {
-  const int vec = (dtype == UNO_BF16) ? 8 : 4;
-  const long long rows = static_cast<long long>(B) * (2 * K + 1);
-  const long long nvec = V / vec;
-  long long smax = nvec / kMinVecPerSlab;
-  if (smax < 1) smax = 1;
-  const long long target = 148LL * 32;  // about four waves of eight CTAs per SM
-  long long s = (target + rows - 1) / rows;
-  if (s > smax) s = smax;
-  if (s < 1) s = 1;
-  return static_cast<int>(s);
-}
+struct Geometry {
+  int S, nchunks, chunk_len, SD;
+  long long stream_ctas, draw_ctas;
+  size_t off_counts, off_partials, off_chunks, bytes;
+};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -471,13 +606,49 @@ bool verify_sizes_ok(int B, int K, int V, int dtype) {
          K <= kMaxK && V >= 1 && V <= (1 << 28);
 }
 
+// Slabs, chunks and the workspace layout: a function of (B, K, V, dtype) only.
+Geometry geometry(int B, int K, int V, int dtype) {
+  Geometry g{};
+  const size_t esize = (dtype == UNO_BF16) ? 2 : 4;
+  const long long rows = static_cast<long long>(B) * (2 * K + 1);
+  const size_t row_bytes = static_cast<size_t>(V) * esize;
+  long long s = static_cast<long long>((row_bytes + kSlabBytes - 1) / kSlabBytes);
+  const long long want = static_cast<long long>(kSizingSms) * kStreamCtasPerSm * 2;
+  if (rows > 0 && s * rows < want) s = (want + rows - 1) / rows;
+  long long smax = static_cast<long long>(row_bytes / kMinSlabBytes);
+  if (smax < 1) smax = 1;
+  if (s > smax) s = smax;
+  if (s < 1) s = 1;
+  g.S = static_cast<int>(s);
+  int cl = (V + kMaxChunks - 1) / kMaxChunks;
+  cl = ((cl + kChunkMin - 1) / kChunkMin) * kChunkMin;
+  if (cl < kChunkMin) cl = kChunkMin;
+  g.chunk_len = cl;
+  g.nchunks = (V + cl - 1) / cl;
+  g.SD = (g.nchunks + kChunksPerDrawCta - 1) / kChunksPerDrawCta;
+  g.stream_ctas = rows * g.S;
+  g.draw_ctas = static_cast<long long>(B) * g.SD;
+  g.off_counts = 0;
+  g.off_partials = align_up(2 * sizeof(int) * static_cast<size_t>(B), 256);
+  g.off_chunks =
+      align_up(g.off_partials + sizeof(Partial) * static_cast<size_t>(g.stream_ctas), 256);
+  g.bytes = align_up(g.off_chunks + sizeof(float) * static_cast<size_t>(B) * g.nchunks, 256);
+  return g;
+}
+
+template <typename T>
+int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
+  verify_stream_kernel<T><<<static_cast<unsigned>(g.stream_ctas), kThreads, 0, st>>>(P);
+  if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
+  verify_draw_kernel<T><<<static_cast<unsigned>(g.draw_ctas), kThreads, 0, st>>>(P);
+  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" size_t uno_verify_workspace_bytes(int B, int K, int V, int dtype) {
   if (!verify_sizes_ok(B, K, V, dtype)) return 0;
-  const int S = choose_slabs(B, K, V, dtype);
-  const size_t partial = static_cast<size_t>(B) * (2 * K + 1) * S * sizeof(Partial);
-  return align_up(partial, 16) + align_up(static_cast<size_t>(B) * sizeof(int), 16);
+  return geometry(B, K, V, dtype).bytes;
 }
 
 extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
@@ -498,11 +669,13 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
       !uno_host::aligned(p_at_draft, 4) || !uno_host::aligned(q_at_draft, 4) ||
       !uno_host::aligned(row_lse, 4))
     return UNO_ERR_ALIGN;
-  const size_t need = uno_verify_workspace_bytes(B, K, V, dtype);
-  if (workspace_bytes < need) return UNO_ERR_WORKSPACE;
+  const Geometry g = geometry(B, K, V, dtype);
+  if (workspace_bytes < g.bytes) return UNO_ERR_WORKSPACE;
+  if (g.stream_ctas > INT_MAX || g.draw_ctas > INT_MAX) return UNO_ERR_SIZE;
   const int dev_status = uno_host::check_device();
   if (dev_status != UNO_OK) return dev_status;
 
+  char* ws = static_cast<char*>(workspace);
   VerifyParams P;
   P.p_logits = p_logits;
   P.q_logits = q_logits;
@@ -510,7 +683,10 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.B = B;
   P.K = K;
   P.V = V;
-  P.S = choose_slabs(B, K, V, dtype);
+  P.S = g.S;
+  P.nchunks = g.nchunks;
+  P.chunk_len = g.chunk_len;
+  P.SD = g.SD;
   P.seed = seed;
   P.step = step;
   P.out_tokens = out_tokens;
@@ -518,16 +694,10 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.p_at_draft = p_at_draft;
   P.q_at_draft = q_at_draft;
   P.row_lse = row_lse;
-  const size_t partial_bytes =
-      align_up(static_cast<size_t>(B) * (2 * K + 1) * P.S * sizeof(Partial), 16);
-  P.partials = static_cast<Partial*>(workspace);
-  P.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes);
-
-  const long long grid = static_cast<long long>(B) * (2 * K + 1) * P.S;
+  P.draw_count = reinterpret_cast<int*>(ws + g.off_counts);
+  P.max_pos = P.draw_count + B;
+  P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
+  P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == UNO_BF16)
-    verify_kernel<uint16_t><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(P);
-  else
-    verify_kernel<float><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(P);
-  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
+  return (dtype == UNO_BF16) ? launch<uint16_t>(P, g, st) : launch<float>(P, g, st);
 }

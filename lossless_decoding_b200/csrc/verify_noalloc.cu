@@ -79,8 +79,8 @@ extern "C" int uno_verify_block_noalloc(const void* p_logits, const void* q_logi
   void* scratch = nullptr;
   const int st = scratch_for_current_device(&scratch);
   if (st != UNO_OK) return st;
-  // The array keeps whatever the previous call left; the verifier needs the
-  // part it uses to start at zero, so clear it on the caller's stream.
+  // The array keeps whatever the previous call left; clear the part this call
+  // uses on the caller's stream so every call starts from the same state.
   if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return UNO_ERR_CUDA;
   return uno_verify_block(p_logits, q_logits, draft_tokens, B, K, V, dtype, seed, step,

@@ -61,8 +61,9 @@ def test_parity_small(api, B, K, V, dtype, dist, sigma):
 
 def test_workspace_is_reusable_and_calls_are_independent(api):
     v = verify_inputs(8, 6, 3001, dtype="bf16", seed=5)
-    ws = torch.zeros(api.verify_workspace_bytes(8, 6, 3001, torch.bfloat16), dtype=torch.uint8,
-                     device=DEV)
+    # start from garbage: the kernels must not depend on the workspace contents
+    ws = torch.full((api.verify_workspace_bytes(8, 6, 3001, torch.bfloat16),), 0xA5,
+                    dtype=torch.uint8, device=DEV)
     outs = []
     for step in range(4):
         res = api.verify_block(v.p_logits.to(DEV), v.q_logits.to(DEV), v.draft_tokens.to(DEV),
@@ -70,7 +71,6 @@ def test_workspace_is_reusable_and_calls_are_independent(api):
         torch.cuda.synchronize()
         compare_verify(res, _oracle(v, 9, step))
         outs.append(res.out_tokens.cpu())
-    assert torch.count_nonzero(ws).item() == 0  # left zero-filled
     again = api.verify_block(v.p_logits.to(DEV), v.q_logits.to(DEV), v.draft_tokens.to(DEV),
                              seed=9, step=0, workspace=ws)
     torch.cuda.synchronize()
