@@ -8,23 +8,23 @@
 // from the verifier), with the standard speculative accept rule
 // u < p(x)/q(x) and residual max(0, p - q) that the pages cite.
 //
-// Two launches per call, with no waiting between CTAs:
+// Three launches per call; no CTA ever waits for another:
 //  1. verify_stream_kernel streams every logit row once. One CTA per slab
-//     (about 64 KB of one row) issues 16-byte loads, four per thread in flight
-//     plus the next four prefetched, folds them into a running
-//     (reference, sum of 2^(x - reference)) in the log2 domain and writes one
-//     partial per slab.
-//     Nothing else happens on this path, so it runs at the speed of HBM.
-//  2. verify_draw_kernel runs SD CTAs per sequence. Each CTA merges the slab
-//     partials of the sequence's 2K+1 rows in a fixed order, evaluates the
-//     accept tests with Philox uniforms and finds the first rejection by
-//     ballot -- every CTA of a sequence computes the same decision from the
-//     same data, so none waits for another -- then sums the residual weights
-//     max(0, p_n - q_n) (or the bonus row p_K) over its range of fixed-size
-//     vocabulary chunks. The CTA that completes a sequence (atomic counter)
-//     takes the float64 running sum of the chunk sums, finds the chunk where
-//     u' * total is crossed, scans it with warp prefix sums to pick the token
-//     and writes the outputs.
+//     (up to 256 KB of one row, a whole number of 16 KB rounds) issues 16-byte
+//     loads, four per thread in flight plus the next four prefetched, folds
+//     them into a running (reference, sum of 2^(x - reference)) in the log2
+//     domain and writes one partial per slab. Nothing else happens on this
+//     path.
+//  2. verify_decide_kernel, one CTA per sequence, merges the slab partials of
+//     the sequence's 2K+1 rows in slab order, evaluates the accept tests with
+//     Philox uniforms, finds the first rejection by ballot and records what the
+//     draw needs (which rows, their statistics).
+//  3. verify_draw_kernel runs SD CTAs per sequence; each sums the residual
+//     weights max(0, p_n - q_n) (or the bonus row p_K) over its range of
+//     fixed-size vocabulary chunks with 16-byte loads. The CTA that completes a
+//     sequence (atomic counter) takes the float64 running sum of the chunk
+//     sums, finds the chunk where u' * total is crossed, scans it with warp
+//     prefix sums to pick the token and writes the outputs.
 #include <atomic>
 #include <cfloat>
 #include <climits>
@@ -43,13 +43,14 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kStreamCtasPerSm = 4;
 constexpr int kRound = 4;                 // 16-byte vectors per thread per round
-constexpr int kSlabBytes = 65536;         // target bytes streamed by one CTA
+constexpr int kSlabBytes = 262144;        // target bytes streamed by one CTA
 constexpr int kMinSlabBytes = kThreads * 16;
 constexpr int kMaxK = 256;
 constexpr int kMaxRows = 2 * kMaxK + 1;
 constexpr int kChunkMin = 256;            // vocabulary entries per inverse-CDF chunk
 constexpr int kMaxChunks = 4096;          // chunks per row (the chunk length grows beyond)
-constexpr int kChunksPerDrawCta = 16;
+constexpr int kDrawCtasPerSm = 2;
+constexpr int kDrawCtasTarget = 148 * kDrawCtasPerSm;  // one wave of draw CTAs
 constexpr int kSizingSms = 148;           // fixed, so the workspace size is device-independent
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -57,6 +58,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 struct Partial {
   float m;  // reference in the log2 domain (see fold)
   float z;  // sum over the slab of 2^(l * log2(e) - m)
+};
+
+// What the draw needs to know about one sequence.
+struct __align__(16) Decision {
+  int n;        // first rejected position (K: all accepted)
+  int invalid;  // a draft id was out of range
+  int mode;     // 0: residual max(0, p_n - q_n); 1: the row p_n itself
+  float mp, izp, mq, izq;  // draw rows: reference (log2 domain) and 1 / sum
+  float c;                 // residual sign threshold (log2 domain)
 };
 
 struct VerifyParams {
@@ -76,8 +86,8 @@ struct VerifyParams {
   float* row_lse;
   Partial* partials;  // [B][2K+1][S]
   float* chunk_sums;  // [B][nchunks]
-  int* draw_count;    // [B], set to 0 by the streaming launch
-  int* max_pos;       // [B], 1 + largest positive-weight index; set to 0 likewise
+  int* draw_count;    // [B], set to 0 by the decision launch
+  Decision* decisions;  // [B]
 };
 
 // ---- element access -----------------------------------------------------------
@@ -221,47 +231,52 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const int rj = blockIdx.x / P.S;
   const int j = rj % R, b = rj / R;
 
-  if (s == 0 && j == 0 && tid == 0) {  // counters the draw launch relies on
-    P.draw_count[b] = 0;
-    P.max_pos[b] = 0;
-  }
-
   size_t off;
   const T* row = row_ptr<T>(P, b, j, &off);
   const RowGeom g = row_geom<T>(off, P.V);
-  const int per = (g.nvec + P.S - 1) / P.S;
+  constexpr int kStep = kRound * kThreads;  // vectors per round of the whole CTA
+  // Every slab but the last of a row holds a whole number of rounds.
+  const int per = ((g.nvec + P.S - 1) / P.S + kStep - 1) / kStep * kStep;
   const int v0 = min(s * per, g.nvec), v1 = min(v0 + per, g.nvec);
   const uint4* vrow = reinterpret_cast<const uint4*>(row + g.head);
 
   float m = -INFINITY, z = 0.f;
-  constexpr int kStep = kRound * kThreads;
-  const int full = (v1 - v0) / kStep;  // rounds in which every thread has kRound vectors
+  const int rounds = (v1 - v0 + kStep - 1) / kStep;  // the last one may be partial
   uint4 cur[kRound], nxt[kRound];
-  if (full > 0) {
 #pragma unroll
-    for (int k = 0; k < kRound; ++k) cur[k] = __ldg(vrow + v0 + k * kThreads + tid);
+  for (int k = 0; k < kRound; ++k) {
+    const int idx = v0 + k * kThreads + tid;
+    cur[k] = (idx < v1) ? __ldg(vrow + idx) : make_uint4(0, 0, 0, 0);
   }
-  for (int r = 0; r < full; ++r) {
-    const int nb = v0 + (r + 1) * kStep;
-    if (r + 1 < full) {
+  for (int r = 0; r < rounds; ++r) {
+    const int base = v0 + r * kStep;
+    if (r + 1 < rounds) {  // prefetch the next round (predicated: it may be partial)
 #pragma unroll
-      for (int k = 0; k < kRound; ++k) nxt[k] = __ldg(vrow + nb + k * kThreads + tid);
+      for (int k = 0; k < kRound; ++k) {
+        const int idx = base + kStep + k * kThreads + tid;
+        nxt[k] = (idx < v1) ? __ldg(vrow + idx) : make_uint4(0, 0, 0, 0);
+      }
     }
+    if (base + kStep <= v1) {  // a full round: no predication
 #pragma unroll
-    for (int k = 0; k < kRound; k += 2) {
-      float f[2 * kVec];
-      Elem<T>::unpack(cur[k], f);
-      Elem<T>::unpack(cur[k + 1], f + kVec);
-      fold<2 * kVec>(m, z, f);
+      for (int k = 0; k < kRound; k += 2) {
+        float f[2 * kVec];
+        Elem<T>::unpack(cur[k], f);
+        Elem<T>::unpack(cur[k + 1], f + kVec);
+        fold<2 * kVec>(m, z, f);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kRound; ++k) {
+        if (base + k * kThreads + tid < v1) {
+          float f[kVec];
+          Elem<T>::unpack(cur[k], f);
+          fold<kVec>(m, z, f);
+        }
+      }
     }
 #pragma unroll
     for (int k = 0; k < kRound; ++k) cur[k] = nxt[k];
-  }
-  // remainder: fewer than kRound vectors per thread
-  for (int idx = v0 + full * kStep + tid; idx < v1; idx += kThreads) {
-    float f[kVec];
-    Elem<T>::unpack(__ldg(vrow + idx), f);
-    fold<kVec>(m, z, f);
   }
   if (s == 0 && tid < g.head) {
     const float v = Elem<T>::at(row, tid);
@@ -288,18 +303,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 
 // ---- launch 2: decision and draw ----------------------------------------------------------
 
-struct DrawShared {
-  float row_m[kMaxRows], row_z[kMaxRows];
-  double scan[kThreads];
-  double total;
-  int first_reject, invalid, last_pos, is_last, chunk, token;
-};
-
-struct DrawRows {
-  int mode;  // 0: residual max(0, p_n - q_n); 1: the row p_n itself
-  float mp, izp, mq, izq;
-  float c;   // residual sign threshold (log2 domain)
-};
+using DrawRows = Decision;
 
 // Weight of token v. mode 0: max(0, p(v) - q(v)), skipping both exponentials
 // where the log-domain test shows p(v) < q(v) by a clear margin; mode 1: p(v).
@@ -323,55 +327,70 @@ template <typename T>
 __device__ int chunk_sums(const VerifyParams& P, int b, const DrawRows& d, const T* rp,
                           const T* rq, int c0, int c1, int w0, int wstep) {
   constexpr int kVec = Elem<T>::kVec;
-  constexpr int kMaxVecs = 4;  // vectors per lane held in flight per row
+  constexpr int kMaxVecs = 8;  // vectors per lane held in flight per row
   const int lane = threadIdx.x & 31;
   int last = -1;
   const int vpl = P.chunk_len / (32 * kVec);  // vectors per lane per chunk
   const bool vec_ok = ((reinterpret_cast<uintptr_t>(rp) | reinterpret_cast<uintptr_t>(rq)) & 15) == 0 &&
-                      (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0 && vpl >= 1;
+                      (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0 && vpl >= 1 &&
+                      vpl <= kMaxVecs;
   if (vec_ok) {
     const uint4* vp = reinterpret_cast<const uint4*>(rp);
     const uint4* vq = reinterpret_cast<const uint4*>(rq);
-    const int nvec_row = P.V / kVec;
-    for (int c = c0 + w0; c < c1; c += wstep) {
-      float s = 0.f;
-      for (int q0 = 0; q0 < vpl; q0 += kMaxVecs) {
-        uint4 a[kMaxVecs], bq[kMaxVecs];
-        int vi[kMaxVecs];
+    const int cvec = P.chunk_len / kVec;  // vectors per chunk
+    const int nvec_row = P.V / kVec;      // vectors per row (V is a multiple of kVec here)
+    // Each pass covers up to kMaxVecs (chunk, vector) pairs per lane: all loads
+    // of a pass are issued before any is used.
+    const int per_pass_chunks = max(1, kMaxVecs / vpl);
+    for (int cb = c0 + w0; cb < c1; cb += wstep * per_pass_chunks) {
+      uint4 a[kMaxVecs], bq[kMaxVecs];
 #pragma unroll
-        for (int k = 0; k < kMaxVecs; ++k) {
-          vi[k] = c * (P.chunk_len / kVec) + (q0 + k) * 32 + lane;
-          const bool in = (q0 + k < vpl) && (vi[k] < nvec_row);
-          a[k] = in ? __ldg(vp + vi[k]) : make_uint4(0, 0, 0, 0);
-          bq[k] = (in && d.mode == 0) ? __ldg(vq + vi[k]) : make_uint4(0, 0, 0, 0);
-          if (!in) vi[k] = -1;
-        }
+      for (int k = 0; k < kMaxVecs; ++k) {
+        const int c = cb + (k / vpl) * wstep;
+        const int q = k % vpl;
+        const int vi = c * cvec + q * 32 + lane;
+        const bool in = (k < per_pass_chunks * vpl) && (c < c1) && (q < vpl) && (vi < nvec_row);
+        a[k] = in ? __ldg(vp + vi) : make_uint4(0, 0, 0, 0);
+        bq[k] = (in && d.mode == 0) ? __ldg(vq + vi) : make_uint4(0, 0, 0, 0);
+      }
+      float s[kMaxVecs / 1];
 #pragma unroll
-        for (int k = 0; k < kMaxVecs; ++k) {
-          if (vi[k] < 0) continue;
-          float fp[kVec], fq[kVec];
-          Elem<T>::unpack(a[k], fp);
-          Elem<T>::unpack(bq[k], fq);
+      for (int k = 0; k < kMaxVecs; ++k) {
+        const int c = cb + (k / vpl) * wstep;
+        const int q = k % vpl;
+        s[k] = 0.f;
+        const int vi = c * cvec + q * 32 + lane;
+        if (!((k < per_pass_chunks * vpl) && (c < c1) && (q < vpl) && (vi < nvec_row))) continue;
+        float fp[kVec], fq[kVec];
+        Elem<T>::unpack(a[k], fp);
+        Elem<T>::unpack(bq[k], fq);
 #pragma unroll
-          for (int e = 0; e < kVec; ++e) {
-            float w;
-            const float lp = fp[e] * kLog2e;
-            if (d.mode) {
-              w = uno::ex2(lp - d.mp) * d.izp;
-            } else {
-              const float lq = fq[e] * kLog2e;
-              w = (lp - lq < d.c - 1e-3f)
-                      ? 0.f
-                      : fmaxf(0.f, uno::ex2(lp - d.mp) * d.izp - uno::ex2(lq - d.mq) * d.izq);
-            }
-            s += w;
-            if (w > 0.f) last = max(last, vi[k] * kVec + e);
+        for (int e = 0; e < kVec; ++e) {
+          float w;
+          const float lp = fp[e] * kLog2e;
+          if (d.mode) {
+            w = uno::ex2(lp - d.mp) * d.izp;
+          } else {
+            const float lq = fq[e] * kLog2e;
+            w = (lp - lq < d.c - 1e-3f)
+                    ? 0.f
+                    : fmaxf(0.f, uno::ex2(lp - d.mp) * d.izp - uno::ex2(lq - d.mq) * d.izq);
           }
+          s[k] += w;
+          if (w > 0.f) last = max(last, vi * kVec + e);
         }
       }
+      // one sum per chunk of this pass
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = s;
+      for (int k0 = 0; k0 < kMaxVecs; k0 += 1) {
+        if (k0 % vpl != 0 || k0 >= per_pass_chunks * vpl) continue;
+        float t = 0.f;
+        for (int q = 0; q < vpl && k0 + q < kMaxVecs; ++q) t += s[k0 + q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+        const int c = cb + (k0 / vpl) * wstep;
+        if (lane == 0 && c < c1) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = t;
+      }
     }
     return last;
   }
@@ -399,105 +418,21 @@ __device__ int chunk_sums(const VerifyParams& P, int b, const DrawRows& d, const
   return last;
 }
 
-// Per-thread block sums of the chunk sums and their exclusive running sum in
-// index order (float64): thread t owns chunks [c0, c1); sh.scan[t] receives the
-// sum of all chunks before c0 and sh.total the sum of all chunks.
-__device__ void prefix_chunks(const float* cs, int c0, int c1, DrawShared& sh) {
+// ---- launch 2: the decision of each sequence (one CTA per sequence) ---------------------
+
+struct DecideShared {
+  float row_m[kMaxRows], row_z[kMaxRows];
+  int first_reject, invalid;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyParams P) {
+  __shared__ DecideShared sh;
   const int tid = threadIdx.x;
-  double mine = 0.0;
-  for (int c = c0; c < c1; ++c) mine += static_cast<double>(__ldcg(cs + c));
-  sh.scan[tid] = mine;
-  __syncthreads();
-  if (tid == 0) {
-    double run = 0.0;
-    for (int t = 0; t < kThreads; ++t) {
-      const double x = sh.scan[t];
-      sh.scan[t] = run;
-      run += x;
-    }
-    sh.total = run;
-    sh.chunk = INT_MAX;
-    sh.token = -1;
-  }
-  __syncthreads();
-}
-
-// Final inverse-CDF step of sequence b (the whole CTA); returns the token.
-template <typename T>
-__device__ int finish_draw(const VerifyParams& P, int b, int n, DrawRows d, const T* rp,
-                           const T* rq, DrawShared& sh) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
-  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, n).y);
-  const int per = (P.nchunks + kThreads - 1) / kThreads;
-  const int c0 = min(tid * per, P.nchunks), c1 = min(c0 + per, P.nchunks);
-  int last_pos = __ldcg(P.max_pos + b) - 1;
-  prefix_chunks(cs, c0, c1, sh);
-  if (sh.total <= 0.0 && d.mode == 0) {
-    // The residual mass is zero (possible only through rounding): draw from p_n.
-    d.mode = 1;
-    rq = rp;
-    if (tid == 0) sh.last_pos = -1;
-    __syncthreads();
-    const int l = chunk_sums<T>(P, b, d, rp, rp, 0, P.nchunks, warp, kWarps);
-    if (l >= 0) atomicMax(&sh.last_pos, l);
-    __threadfence();
-    __syncthreads();
-    last_pos = sh.last_pos;
-    prefix_chunks(cs, c0, c1, sh);
-  }
-  const double t = static_cast<double>(u) * sh.total;
-  {
-    double run = sh.scan[tid];
-    for (int c = c0; c < c1; ++c) {
-      const double nxt = run + static_cast<double>(__ldcg(cs + c));
-      if (nxt > t) {
-        atomicMin(&sh.chunk, c);
-        break;
-      }
-      run = nxt;
-    }
-  }
-  __syncthreads();
-  const int ch = sh.chunk;
-  if (warp == 0 && ch != INT_MAX) {
-    double carry = 0.0;
-    for (int c = lane; c < ch; c += 32) carry += static_cast<double>(__ldcg(cs + c));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) carry += __shfl_xor_sync(0xFFFFFFFFu, carry, o);
-    const int v0 = ch * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
-    int tok = -1, last_in_chunk = -1;
-    for (int base = v0; base < v1 && tok < 0; base += 32) {
-      const int v = base + lane;
-      const float w = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
-      float incl = w;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float up = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += up;
-      }
-      const bool cross = (w > 0.f) && (carry + static_cast<double>(incl) > t);
-      const unsigned hit = __ballot_sync(0xFFFFFFFFu, cross);
-      const unsigned pos = __ballot_sync(0xFFFFFFFFu, w > 0.f);
-      if (pos) last_in_chunk = base + 31 - __clz(pos);
-      if (hit) tok = base + __ffs(hit) - 1;
-      carry += static_cast<double>(__shfl_sync(0xFFFFFFFFu, incl, 31));
-    }
-    if (lane == 0) sh.token = (tok >= 0) ? tok : last_in_chunk;
-  }
-  __syncthreads();
-  return (sh.token >= 0) ? sh.token : last_pos;
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParams P) {
-  __shared__ DrawShared sh;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int b = blockIdx.x / P.SD, du = blockIdx.x % P.SD;
+  const int b = blockIdx.x;
   const int K = P.K, R = 2 * K + 1, S = P.S, V = P.V;
-  const bool reporter = (du == 0);  // writes the per-position and per-row outputs
 
-  // 1. row statistics: merge the slab partials of every row in slab order
+  // row statistics: merge the slab partials of every row in slab order
   for (int j = tid; j < R; j += kThreads) {
     const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
     float m = -INFINITY, z = 0.f;
@@ -510,16 +445,16 @@ __global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParam
     }
     sh.row_m[j] = m;
     sh.row_z[j] = z;
-    if (reporter && P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
+    if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
   }
   if (tid == 0) {
     sh.first_reject = K;
     sh.invalid = 0;
-    sh.last_pos = -1;
+    P.draw_count[b] = 0;
   }
   __syncthreads();
 
-  // 2. accept tests, one thread per position; first rejection by ballot
+  // accept tests, one thread per position; first rejection by ballot
   for (int i0 = 0; i0 < K; i0 += kThreads) {
     const int i = i0 + tid;
     bool rejected = false;
@@ -536,8 +471,8 @@ __global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParam
                          sh.row_z[K + 1 + i];
         const uint4 w = uno::verify_block_words(P.seed, P.step, b, i);
         rejected = !(uno::uniform24(w.x) * qq < pp);
-        if (reporter && P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
-        if (reporter && P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
+        if (P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
+        if (P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
       }
     }
     const unsigned ballot = __ballot_sync(0xFFFFFFFFu, rejected);
@@ -546,46 +481,172 @@ __global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParam
   }
   __syncthreads();
   const int n = sh.first_reject;
-  const bool invalid = sh.invalid != 0;
-  int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
-
-  // 3. this CTA's share of the chunk sums of the draw rows
-  DrawRows d{};
-  size_t off;
-  const T* rp = row_ptr<T>(P, b, n, &off);
-  const T* rq = rp;
-  d.mode = (n < K) ? 0 : 1;
-  d.mp = sh.row_m[n];
-  d.izp = 1.f / sh.row_z[n];
-  if (n < K) {
-    rq = row_ptr<T>(P, b, K + 1 + n, &off);
-    d.mq = sh.row_m[K + 1 + n];
-    d.izq = 1.f / sh.row_z[K + 1 + n];
-    d.c = (sh.row_m[n] + log2f(sh.row_z[n])) - (sh.row_m[K + 1 + n] + log2f(sh.row_z[K + 1 + n]));
+  if (sh.invalid) {
+    int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
+    for (int i = tid; i <= K; i += kThreads) out[i] = -1;
   }
-  if (invalid) {
-    if (reporter) {
-      for (int i = tid; i <= K; i += kThreads) out[i] = -1;
-      if (tid == 0) P.accepted_len[b] = -1;
+  if (tid == 0) {
+    Decision d{};
+    d.n = n;
+    d.invalid = sh.invalid;
+    d.mode = (n < K) ? 0 : 1;
+    d.mp = sh.row_m[n];
+    d.izp = 1.f / sh.row_z[n];
+    if (n < K) {
+      d.mq = sh.row_m[K + 1 + n];
+      d.izq = 1.f / sh.row_z[K + 1 + n];
+      d.c = (sh.row_m[n] + log2f(sh.row_z[n])) -
+            (sh.row_m[K + 1 + n] + log2f(sh.row_z[K + 1 + n]));
     }
-  } else {
-    const int c0 = du * kChunksPerDrawCta;
-    const int c1 = min(c0 + kChunksPerDrawCta, P.nchunks);
-    const int l = chunk_sums<T>(P, b, d, rp, rq, c0, c1, warp, kWarps);
-    if (l >= 0) atomicMax(&sh.last_pos, l);
+    P.decisions[b] = d;
+    if (sh.invalid) P.accepted_len[b] = -1;
+  }
+}
+
+// ---- launch 3: the draw -------------------------------------------------------------------
+
+struct DrawShared {
+  double warp_tot[kWarps];
+  double total;
+  double carry;
+  int is_last, chunk, last_chunk, token_min, last_in_chunk;
+};
+
+// Exclusive running sum (float64, index order) of per-thread values across the
+// CTA; also leaves the grand total in sh.total.
+__device__ double block_exclusive_scan(double mine, DrawShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double up = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += up;
+  }
+  if (lane == 31) sh.warp_tot[warp] = incl;
+  __syncthreads();
+  double before = 0.0;
+  for (int w = 0; w < warp; ++w) before += sh.warp_tot[w];
+  if (threadIdx.x == kThreads - 1) sh.total = before + incl;
+  __syncthreads();
+  return before + incl - mine;
+}
+
+// Largest index with positive weight in chunk c (the whole CTA), or -1.
+template <typename T>
+__device__ int last_positive_in_chunk(const VerifyParams& P, const DrawRows& d, const T* rp,
+                                      const T* rq, int c, DrawShared& sh) {
+  if (threadIdx.x == 0) sh.last_in_chunk = -1;
+  __syncthreads();
+  const int v0 = c * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
+  for (int v = v0 + threadIdx.x; v < v1; v += kThreads)
+    if (weight<T>(d, rp, rq, v) > 0.f) atomicMax(&sh.last_in_chunk, v);
+  __syncthreads();
+  return sh.last_in_chunk;
+}
+
+// Final inverse-CDF step of sequence b (the whole CTA); returns the token.
+// Thread t holds the sums of chunks [t * per, (t + 1) * per) in registers.
+template <typename T>
+__device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp, const T* rq,
+                           DrawShared& sh) {
+  constexpr int kMaxPer = kMaxChunks / kThreads;
+  const int tid = threadIdx.x;
+  float* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
+  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, d.n).y);
+  const int per = (P.nchunks + kThreads - 1) / kThreads;
+  const int c0 = tid * per;
+  float mine_cs[kMaxPer];
+  double mine = 0.0, before = 0.0;
+  for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k)
+      mine_cs[k] = (k < per && c0 + k < P.nchunks) ? __ldcg(cs + c0 + k) : 0.f;
+    mine = 0.0;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) mine += static_cast<double>(mine_cs[k]);
+    before = block_exclusive_scan(mine, sh);
+    if (sh.total > 0.0 || d.mode == 1) break;
+    // The residual mass is zero (possible only through rounding): draw from p_n.
+    d.mode = 1;
+    rq = rp;
+    chunk_sums<T>(P, b, d, rp, rp, 0, P.nchunks, threadIdx.x >> 5, kWarps);
+    __threadfence();
+    __syncthreads();
+  }
+  if (tid == 0) {
+    sh.chunk = INT_MAX;
+    sh.last_chunk = -1;
+    sh.token_min = INT_MAX;
+    sh.last_in_chunk = -1;
   }
   __syncthreads();
+  const double t = static_cast<double>(u) * sh.total;
+  {
+    double run = before;
+    int found = -1, last_pos_chunk = -1;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+      if (k < per && c0 + k < P.nchunks) {
+        const double nxt = run + static_cast<double>(mine_cs[k]);
+        if (found < 0 && nxt > t) found = c0 + k;
+        if (mine_cs[k] > 0.f) last_pos_chunk = c0 + k;
+        if (found < 0) run = nxt;
+      }
+    }
+    if (found >= 0) atomicMin(&sh.chunk, found);
+    if (last_pos_chunk >= 0) atomicMax(&sh.last_chunk, last_pos_chunk);
+    __syncthreads();
+    if (found >= 0 && found == sh.chunk) sh.carry = run;  // running sum before that chunk
+  }
+  __syncthreads();
+  const int ch = sh.chunk;
+  if (ch == INT_MAX) {
+    // Rounding left no crossing: the largest index with positive weight.
+    return (sh.last_chunk >= 0) ? last_positive_in_chunk<T>(P, d, rp, rq, sh.last_chunk, sh) : -1;
+  }
+  double carry = sh.carry;
+  const int v0 = ch * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
+  for (int base = v0; base < v1; base += kThreads) {
+    const int v = base + tid;
+    const float w = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
+    const double bef = carry + block_exclusive_scan(static_cast<double>(w), sh);
+    if ((w > 0.f) && (bef + static_cast<double>(w) > t)) atomicMin(&sh.token_min, v);
+    if (w > 0.f) atomicMax(&sh.last_in_chunk, v);
+    carry += sh.total;
+    __syncthreads();
+    if (sh.token_min != INT_MAX) break;
+  }
+  return (sh.token_min != INT_MAX) ? sh.token_min : sh.last_in_chunk;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(const VerifyParams P) {
+  __shared__ DrawShared sh;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int b = blockIdx.x / P.SD, du = blockIdx.x % P.SD;
+  const int K = P.K;
+  const Decision d = P.decisions[b];
+  if (d.invalid) return;  // the decision launch wrote this sequence's outputs
+  size_t off;
+  const T* rp = row_ptr<T>(P, b, d.n, &off);
+  const T* rq = (d.mode == 0) ? row_ptr<T>(P, b, K + 1 + d.n, &off) : rp;
+  const int per_cta = (P.nchunks + P.SD - 1) / P.SD;
+  const int c0 = du * per_cta;
+  const int c1 = min(c0 + per_cta, P.nchunks);
+  chunk_sums<T>(P, b, d, rp, rq, c0, c1, warp, kWarps);
+  __syncthreads();
   if (tid == 0) {
-    if (sh.last_pos >= 0) atomicMax(P.max_pos + b, sh.last_pos + 1);
     __threadfence();
     sh.is_last = (atomicAdd(P.draw_count + b, 1) == P.SD - 1);
   }
   __syncthreads();
-  if (!sh.is_last || invalid) return;
+  if (!sh.is_last) return;
 
-  // 4. the CTA that completes the sequence picks the token and writes outputs
+  // the CTA that completes the sequence picks the token and writes outputs
   __threadfence();
-  const int y = finish_draw<T>(P, b, n, d, rp, rq, sh);
+  const int y = finish_draw<T>(P, b, d, rp, rq, sh);
+  const int n = d.n;
+  int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
   const int32_t* x = P.draft + static_cast<size_t>(b) * K;
   for (int i = tid; i <= K; i += kThreads) out[i] = (i < n) ? x[i] : ((i == n) ? y : -1);
   if (tid == 0) P.accepted_len[b] = n;
@@ -596,7 +657,7 @@ __global__ void __launch_bounds__(kThreads) verify_draw_kernel(const VerifyParam
 struct Geometry {
   int S, nchunks, chunk_len, SD;
   long long stream_ctas, draw_ctas;
-  size_t off_counts, off_partials, off_chunks, bytes;
+  size_t off_counts, off_decisions, off_partials, off_chunks, bytes;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -625,11 +686,17 @@ Geometry geometry(int B, int K, int V, int dtype) {
   if (cl < kChunkMin) cl = kChunkMin;
   g.chunk_len = cl;
   g.nchunks = (V + cl - 1) / cl;
-  g.SD = (g.nchunks + kChunksPerDrawCta - 1) / kChunksPerDrawCta;
+  // draw CTAs per sequence: about one wave in total, at least 8 chunks each
+  long long sd = (B > 0) ? (kDrawCtasTarget + B - 1) / B : 1;
+  const long long sd_max = (g.nchunks + 7) / 8;
+  if (sd > sd_max) sd = sd_max;
+  if (sd < 1) sd = 1;
+  g.SD = static_cast<int>(sd);
   g.stream_ctas = rows * g.S;
   g.draw_ctas = static_cast<long long>(B) * g.SD;
   g.off_counts = 0;
-  g.off_partials = align_up(2 * sizeof(int) * static_cast<size_t>(B), 256);
+  g.off_decisions = align_up(sizeof(int) * static_cast<size_t>(B), 256);
+  g.off_partials = align_up(g.off_decisions + sizeof(Decision) * static_cast<size_t>(B), 256);
   g.off_chunks =
       align_up(g.off_partials + sizeof(Partial) * static_cast<size_t>(g.stream_ctas), 256);
   g.bytes = align_up(g.off_chunks + sizeof(float) * static_cast<size_t>(B) * g.nchunks, 256);
@@ -639,6 +706,8 @@ Geometry geometry(int B, int K, int V, int dtype) {
 template <typename T>
 int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
   verify_stream_kernel<T><<<static_cast<unsigned>(g.stream_ctas), kThreads, 0, st>>>(P);
+  if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
+  verify_decide_kernel<T><<<static_cast<unsigned>(P.B), kThreads, 0, st>>>(P);
   if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
   verify_draw_kernel<T><<<static_cast<unsigned>(g.draw_ctas), kThreads, 0, st>>>(P);
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
@@ -695,7 +764,7 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.q_at_draft = q_at_draft;
   P.row_lse = row_lse;
   P.draw_count = reinterpret_cast<int*>(ws + g.off_counts);
-  P.max_pos = P.draw_count + B;
+  P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
   P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
   P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
