@@ -272,10 +272,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if constexpr (PARTIAL) {
           float* base = p.partial + static_cast<size_t>(split) * p.M * p.ncols;
           if constexpr (!SWAP) {
+            // 32 consecutive columns of one row: 16-byte stores (ncols % 4 == 0)
             if (arow < p.M) {
+              float* dst = base + static_cast<size_t>(arow) * p.ncols + brow;
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (brow + e < p.ncols) base[static_cast<size_t>(arow) * p.ncols + brow + e] = f0[e];
+              for (int g = 0; g < 8; ++g)
+                if (brow + g * 4 < p.ncols)
+                  *reinterpret_cast<float4*>(dst + g * 4) =
+                      make_float4(f0[g * 4], f0[g * 4 + 1], f0[g * 4 + 2], f0[g * 4 + 3]);
             }
           } else {
             if (arow < p.ncols) {
@@ -321,19 +325,296 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The dual GEMM, persistent. Each CTA takes tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... (the 128-row A tile index varies fastest, so
+// neighbouring CTAs share a B tile in L2). TMEM holds two BN-column fp32
+// accumulators, used by alternate tiles. Per tile the MMA thread accumulates
+// x W^T over all K-blocks into the tile's accumulator; the epilogue drains it
+// as y_ar and says so; the adapter product T Bm^T (two 64-wide K-blocks for
+// r = 128) is then accumulated into the same accumulator, which the epilogue
+// drains again as y_draft. The adapter K-blocks of tile i ride in the operand
+// ring after the first kInsert K-blocks of tile i + 1, so the tensor pipe works
+// on the next tile while the epilogue drains y_ar.
+// ---------------------------------------------------------------------------
+constexpr int kInsert = 6;
+
+template <typename T, int BN, bool SWAP>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                const GemmParams p, int rowsA, int rowsB) {
+  constexpr int STAGES = stages_for<BN>();
+  constexpr int kAbytes = kBM * kRowBytes;
+  constexpr int kStage = (kBM + BN) * kRowBytes;
+  constexpr bool kTf32 = sizeof(T) == 4;
+  constexpr int kElemsPerRow = kRowBytes / static_cast<int>(sizeof(T));
+  constexpr uint32_t kIdesc = sm100::instr_desc(kTf32, kBM, BN);
+  constexpr int kAcc = pow2_at_least(BN);  // columns of one accumulator buffer
+  constexpr uint32_t kTmemCols = 2 * kAcc;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && kTmemCols <= 512, "BN");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * kStage);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* acc_full = empty_bar + STAGES;   // [2] main product done
+  uint64_t* ar_read = acc_full + 2;          // [2] epilogue drained y_ar
+  uint64_t* draft_full = ar_read + 2;        // [2] adapter product done
+  uint64_t* acc_empty = draft_full + 2;      // [2] epilogue drained the buffer
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_a = (rowsA + kBM - 1) / kBM;
+  const int tiles_b = (rowsB + BN - 1) / BN;
+  const int ntiles = tiles_a * tiles_b;
+  const int nmine = (ntiles > static_cast<int>(blockIdx.x))
+                        ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                        : 0;
+  const int nkb = p.kb_total;
+  const bool adapter = p.nkb_adapt > 0;
+  const int nad = adapter ? p.nkb_adapt : 0;
+  const int ins = min(kInsert, nkb);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      sm100::mbar_init(&full_bar[s], 1);
+      sm100::mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(&acc_full[b], 1);
+      sm100::mbar_init(&ar_read[b], 4);
+      sm100::mbar_init(&draft_full[b], 1);
+      sm100::mbar_init(&acc_empty[b], 4);
+    }
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tmA);
+    sm100::tma_prefetch_desc(&tmB);
+    if (adapter) {
+      sm100::tma_prefetch_desc(&tmA2);
+      sm100::tma_prefetch_desc(&tmB2);
+    }
+  }
+  if (warp == 1) sm100::tmem_alloc(tmem_holder, kTmemCols);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // The operand stream of this CTA, in ring order: for local tile i, its main
+  // K-blocks 0..ins-1, then the adapter K-blocks of tile i-1, then its main
+  // K-blocks ins..nkb-1; after the last tile, that tile's adapter K-blocks.
+  // Item q of local tile i (0 <= q < nkb + nad, nad only for i >= 1) maps to:
+  //   q < ins            -> main block q of tile i
+  //   ins <= q < ins+nad -> adapter block q-ins of tile i-1
+  //   otherwise          -> main block q-nad of tile i
+  auto tile_coords = [&](int li, int& a0, int& b0) {
+    const int t = static_cast<int>(blockIdx.x) + li * static_cast<int>(gridDim.x);
+    a0 = (t % tiles_a) * kBM;
+    b0 = (t / tiles_a) * BN;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer ----
+      int it = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* ma, const CUtensorMap* mb, int kx, int a0, int b0) {
+        const int s = it % STAGES;
+        if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
+          set_fault(kFaultProducer, &abort_flag);
+          ok = false;
+          return;
+        }
+        if (abort_flag) {
+          ok = false;
+          return;
+        }
+        uint8_t* sa = smem + s * kStage;
+        sm100::mbar_arrive_expect_tx(&full_bar[s], kStage);
+        sm100::tma_load_2d(sa, ma, &full_bar[s], kx, a0);
+        sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, b0);
+        ++it;
+      };
+      for (int li = 0; li <= nmine && ok; ++li) {
+        int a0 = 0, b0 = 0, pa0 = 0, pb0 = 0;
+        if (li < nmine) tile_coords(li, a0, b0);
+        if (li > 0) tile_coords(li - 1, pa0, pb0);
+        const int nmain = (li < nmine) ? nkb : 0;
+        const int nadp = (li > 0) ? nad : 0;
+        const int items = nmain + nadp;
+        for (int q = 0; q < items && ok; ++q) {
+          const int qa = q - min(ins, nmain);
+          if (q < min(ins, nmain)) {
+            load(&tmA, &tmB, q * kElemsPerRow, a0, b0);
+          } else if (qa < nadp) {
+            load(&tmA2, &tmB2, qa * kElemsPerRow, pa0, pb0);
+          } else {
+            load(&tmA, &tmB, (q - nadp) * kElemsPerRow, a0, b0);
+          }
+        }
+      }
+      for (int k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+        if (!sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1))
+          set_fault(kFaultProducer, &abort_flag);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      int it = 0;
+      bool ok = true;
+      auto consume = [&](uint32_t d, bool accumulate_first) {
+        const int s = it % STAGES;
+        if (!sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
+          set_fault(kFaultMma, &abort_flag);
+          ok = false;
+          return;
+        }
+        sm100::tc_fence_after();
+        const uint32_t sa = sm100::smem_addr(smem + s * kStage);
+        const uint64_t da = sm100::smem_desc_k_sw128(sa);
+        const uint64_t db = sm100::smem_desc_k_sw128(sa + kAbytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, kIdesc, accumulate_first || (k > 0));
+        sm100::mma_commit(&empty_bar[s]);
+        ++it;
+      };
+      for (int li = 0; li <= nmine && ok; ++li) {
+        const int buf = li & 1, pbuf = (li - 1) & 1;
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * kAcc);
+        const uint32_t pd = tmem + static_cast<uint32_t>(pbuf * kAcc);
+        const int nmain = (li < nmine) ? nkb : 0;
+        const int nadp = (li > 0) ? nad : 0;
+        const int items = nmain + nadp;
+        if (nmain && li >= 2 &&
+            !sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {  // buffer drained
+          set_fault(kFaultMma, &abort_flag);
+          break;
+        }
+        sm100::tc_fence_after();
+        for (int q = 0; q < items && ok; ++q) {
+          const int qa = q - min(ins, nmain);
+          if (q < min(ins, nmain)) {
+            consume(d, q > 0);
+            if (q == nmain - 1) sm100::mma_commit(&acc_full[buf]);
+          } else if (qa < nadp) {
+            if (qa == 0) {
+              if (!sm100::mbar_wait(&ar_read[pbuf], ((li - 1) >> 1) & 1)) {
+                set_fault(kFaultMma, &abort_flag);
+                ok = false;
+                break;
+              }
+              sm100::tc_fence_after();
+            }
+            consume(pd, true);  // adds T Bm^T onto y_ar of the previous tile
+            if (qa == nadp - 1) sm100::mma_commit(&draft_full[pbuf]);
+          } else {
+            const int kb = q - nadp;
+            consume(d, kb > 0);
+            if (kb == nmain - 1) sm100::mma_commit(&acc_full[buf]);
+          }
+        }
+      }
+    }
+  } else {
+    // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    T* ya = static_cast<T*>(p.y_ar);
+    T* yd = static_cast<T*>(p.y_draft);
+    auto drain = [&](uint32_t acc, int a0, int b0, T* y) {
+      if (!y) return;  // output not requested: nothing to read
+      const uint32_t tq = acc + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int arow = a0 + r;
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        sm100::tmem_ld_32x32b_x32(tq + c, v);
+        sm100::tmem_ld_wait();
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        const int brow = b0 + c;
+        if constexpr (!SWAP) {
+          if (arow < p.M && brow < p.ncols)
+            store_row32<T>(y + static_cast<size_t>(arow) * p.ncols + brow, f, p.ncols - brow);
+        } else {
+          if (arow < p.ncols) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * p.ncols + arow, f[e]);
+          }
+        }
+      }
+    };
+    for (int li = 0; li < nmine; ++li) {
+      const int buf = li & 1;
+      const uint32_t acc = tmem + static_cast<uint32_t>(buf * kAcc);
+      int a0, b0;
+      tile_coords(li, a0, b0);
+      const bool got = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&acc_full[buf], (li >> 1) & 1));
+      if (!got || abort_flag) {
+        if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
+        break;
+      }
+      sm100::tc_fence_after();
+      drain(acc, a0, b0, ya);
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(adapter ? &ar_read[buf] : &acc_empty[buf]);
+      if (!adapter) continue;
+      const bool got2 = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&draft_full[buf], (li >> 1) & 1));
+      if (!got2 || abort_flag) {
+        if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
+        break;
+      }
+      sm100::tc_fence_after();
+      drain(acc, a0, b0, yd);
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // T = scale * sum_s partial[s]  (splits summed in index order), rounded to T.
+// Four consecutive elements per thread (count is a multiple of 4).
 template <typename T>
 __global__ void reduce_t_kernel(const float* __restrict__ partial, int splits, size_t count,
                                 float scale, T* __restrict__ out) {
-  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i >= count) return;
-  float s = 0.f;
-  for (int k = 0; k < splits; ++k) s += __ldg(partial + static_cast<size_t>(k) * count + i);
-  s *= scale;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < splits; ++k) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(partial + static_cast<size_t>(k) * count + i));
+    s.x += v.x;
+    s.y += v.y;
+    s.z += v.z;
+    s.w += v.w;
+  }
+  s.x *= scale;
+  s.y *= scale;
+  s.z *= scale;
+  s.w *= scale;
   if constexpr (sizeof(T) == 2) {
-    out[i] = static_cast<uint16_t>(pack_bf16x2(s, 0.f) & 0xFFFFu);
+    uint2 w;
+    w.x = pack_bf16x2(s.x, s.y);
+    w.y = pack_bf16x2(s.z, s.w);
+    *reinterpret_cast<uint2*>(out + i) = w;
   } else {
-    out[i] = s;
+    *reinterpret_cast<float4*>(out + i) = s;
   }
 }
 
@@ -391,6 +672,53 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
   }
   kern<<<grid, kGemmThreads, bytes, st>>>(a, b, a2, b2, p);
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
+}
+
+int sm_count_dual() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <typename T, int BN, bool SWAP>
+int launch_dual(int rowsA, int rowsB, const CUtensorMap& a, const CUtensorMap& b,
+                const CUtensorMap& a2, const CUtensorMap& b2, const GemmParams& p,
+                cudaStream_t st) {
+  constexpr int bytes = smem_bytes<BN, stages_for<BN>()>();
+  auto kern = dual_kernel<T, BN, SWAP>;
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return UNO_ERR_CUDA;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (!bit || !(attr_done.load(std::memory_order_relaxed) & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return UNO_ERR_CUDA;
+    attr_done.fetch_or(bit, std::memory_order_relaxed);
+  }
+  const long long tiles =
+      static_cast<long long>((rowsA + kBM - 1) / kBM) * ((rowsB + BN - 1) / BN);
+  long long grid = sm_count_dual();
+  if (grid > tiles) grid = tiles;
+  kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, p, rowsA, rowsB);
+  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
+}
+
+template <typename T, bool SWAP>
+int launch_dual_bn(int bn, int rowsA, int rowsB, const CUtensorMap& a, const CUtensorMap& b,
+                   const CUtensorMap& a2, const CUtensorMap& b2, const GemmParams& p,
+                   cudaStream_t st) {
+  switch (bn) {
+    case 32: return launch_dual<T, 32, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
+    case 64: return launch_dual<T, 64, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
+    case 128: return launch_dual<T, 128, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
+    default: return launch_dual<T, 256, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
+  }
 }
 
 // Dispatch over the B-tile height (32, 64, 128 or 256 rows).
@@ -485,7 +813,7 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
                       : launch_bn<T, false, true>(pl.t_bn, grid, ta, tb, ta, tb, gp, st);
     if (st_code != UNO_OK) return st_code;
     const size_t count = static_cast<size_t>(M) * r;
-    reduce_t_kernel<T><<<static_cast<unsigned>((count + 255) / 256), 256, 0, st>>>(
+    reduce_t_kernel<T><<<static_cast<unsigned>((count / 4 + 255) / 256), 256, 0, st>>>(
         partial, pl.t_splits, count, scale, Tbuf);
     if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
   }
@@ -505,17 +833,15 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
     if (adapter) ok = ok && make_map(&mBm, Bm, dtype, r, d_out, kBM) &&
                       make_map(&mT, Tbuf, dtype, r, M, bn);
     if (!ok) return UNO_ERR_CUDA;
-    const dim3 grid((d_out + kBM - 1) / kBM, 1, 1);
-    return launch_bn<T, true, false>(bn, grid, mW, mx, adapter ? mBm : mW, adapter ? mT : mx, gp,
-                                     st);
+    return launch_dual_bn<T, true>(bn, d_out, M, mW, mx, adapter ? mBm : mW, adapter ? mT : mx,
+                                   gp, st);
   }
   bool ok = make_map(&mx, x, dtype, d_in, M, xrows_box) && make_map(&mW, W, dtype, d_in, d_out, 256);
   if (adapter) ok = ok && make_map(&mT, Tbuf, dtype, r, M, kBM) &&
                     make_map(&mBm, Bm, dtype, r, d_out, 256);
   if (!ok) return UNO_ERR_CUDA;
-  const dim3 grid((M + kBM - 1) / kBM, (d_out + 255) / 256, 1);
-  return launch_gemm<T, 256, false, false>(grid, mx, mW, adapter ? mT : mx, adapter ? mBm : mW,
-                                           gp, st);
+  return launch_dual<T, 256, false>(M, d_out, mx, mW, adapter ? mT : mx, adapter ? mBm : mW, gp,
+                                    st);
 }
 
 }  // namespace
