@@ -10,19 +10,31 @@
 //   T       = (alpha / r) x A^T
 //   y_draft = y_ar + T Bm^T
 //
-// Two launches:
-//  1. T: a split-K tcgen05 GEMM writes float32 partial products of x A^T to
-//     the workspace; a small kernel sums the splits in index order, scales by
-//     alpha/r and rounds to the operand type.
-//  2. The dual GEMM streams W once. Per output tile, a TMA producer warp feeds
-//     a multi-stage shared-memory ring; one thread issues tcgen05.mma into a
-//     TMEM accumulator D0 = x W^T over all of d_in, then r/64 more K-blocks
-//     of T Bm^T into a second accumulator D1; four epilogue warps read both
-//     with tcgen05.ld and store y_ar = D0 and y_draft = D0 + D1.
-// For M <= 256 the operands swap roles (W rows fill the 128-row MMA side and
-// the few activation rows are the N side), so small-batch decode still runs
-// at full tile height while it is bound by the stream of W.
+// One persistent launch, one CTA per SM. Its tiles, in schedule order:
+//  * T tiles: T = scale * x A^T for one 128-row block (or, with swapped
+//    operands, one 128-column block of T), rounded to the operand type and
+//    stored to the workspace; a release store of the call's epoch to the
+//    tile's flag announces it.
+//  * main tiles: a 128 x BN tile of x W^T over all of d_in, accumulated in
+//    TMEM; the epilogue drains it as y_ar, then the adapter product T Bm^T is
+//    accumulated onto the same accumulator and drained as y_draft.
+// Warp roles: warp 0 issues TMA loads into a multi-stage shared-memory ring,
+// warp 1 owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain
+// TMEM with tcgen05.ld. Two accumulator buffers alternate between tiles, and
+// the adapter K-blocks of a tile ride in the ring a few K-blocks into the next
+// tile, so the tensor pipe keeps working while the epilogue drains.
+//
+// A main tile's producer reads T only after the T tile's flag holds the
+// call's epoch (acquire, then an async-proxy fence before the TMA load). T
+// tiles come first in the schedule, so the CTAs computing them started no
+// later than any CTA that waits for them; the wait is bounded and reports
+// through the fault flags.
+//
+// For M <= 256 the operands swap roles (W rows fill the 128-row MMA side, the
+// few activation rows are the N side), so small-batch decode still runs at full
+// tile height while it is bound by the stream of W.
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -40,24 +52,31 @@
 
 namespace {
 
-constexpr int kBM = 128;              // MMA M (rows of the A operand per tile)
-constexpr int kRowBytes = 128;        // bytes of K per tile row and stage (one swizzle row)
-constexpr int kGemmThreads = 192;     // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
-constexpr int kSmSplitTarget = 148;   // CTAs the T product aims to fill
+constexpr int kBM = 128;           // MMA M (rows of the A operand per tile)
+constexpr int kRowBytes = 128;     // bytes of K per tile row and stage (one swizzle row)
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int kInsert = 6;         // main K-blocks of the next tile before an adapter
+constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum : unsigned { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
 
 __device__ unsigned int g_fault_flags;
 
 struct GemmParams {
-  int kb_total;      // K-blocks of the main product over the whole K extent
-  int kb_per_split;  // K-blocks handled by one split (== kb_total without split)
-  int nkb_adapt;     // K-blocks of the adapter product (0: none)
-  int M;             // output rows
-  int ncols;         // output columns (d_out, or r for the T product)
-  void* y_ar;        // dual mode, may be null
-  void* y_draft;     // dual mode, may be null
-  float* partial;    // partial mode: [split][M][ncols]
+  int kb_total;       // K-blocks over d_in
+  int nkb_adapt;      // K-blocks over r (0: no adapter, no T tiles)
+  int M;              // output rows
+  int ncols;          // output columns (d_out)
+  int rowsA, rowsB;   // rows of the main A and B operands
+  int nT;             // T tiles
+  int r;              // adapter rank
+  uint32_t idesc_t;   // instruction descriptor of the T tiles
+  uint32_t epoch;     // value a T tile's flag takes once T is stored
+  float scale;        // alpha / r
+  void* y_ar;         // may be null
+  void* y_draft;      // may be null
+  void* t_buf;        // T [M][r]
+  uint32_t* t_flags;  // [nT]
 };
 
 __host__ __device__ constexpr int pow2_at_least(int x) {
@@ -87,7 +106,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// Store 32 consecutive columns of one output row (non-swapped tiles).
+// Store 32 consecutive columns of one output row (valid_cols of them exist).
 template <typename T>
 __device__ __forceinline__ void store_row32(T* dst, const float* v, int valid_cols) {
   if constexpr (sizeof(T) == 2) {
@@ -121,229 +140,42 @@ __device__ __forceinline__ void store_one(T* dst, float v) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// The tile GEMM. D[a, b] = sum_k A_op[a, k] * B_op[b, k] for a 128-row tile of
-// the A operand and a BN-row tile of the B operand, both K-major in global
-// memory and loaded by TMA with 128-byte swizzling.
-//   PARTIAL = false: dual mode (main product + optional adapter product).
-//   PARTIAL = true : float32 partial products of one K split.
-//   SWAP    = false: output row = A row, output column = B row.
-//   SWAP    = true : output row = B row, output column = A row.
-// ---------------------------------------------------------------------------
-template <typename T, int BN, bool SWAP, bool PARTIAL>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmA2,
-                const __grid_constant__ CUtensorMap tmB2, const GemmParams p) {
-  constexpr int STAGES = stages_for<BN>();
-  constexpr int kAbytes = kBM * kRowBytes;
-  constexpr int kStage = (kBM + BN) * kRowBytes;
-  constexpr bool kTf32 = sizeof(T) == 4;
-  constexpr int kElemsPerRow = kRowBytes / static_cast<int>(sizeof(T));
-  constexpr uint32_t kIdesc = sm100::instr_desc(kTf32, kBM, BN);
-  constexpr int kD1 = pow2_at_least(BN);                     // column of the adapter accumulator
-  constexpr uint32_t kTmemCols = PARTIAL ? pow2_at_least(BN) : 2 * pow2_at_least(BN);
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
-  static_assert(kTmemCols <= 512, "TMEM");
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * kStage);
-  uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* accum_bar = empty_bar + STAGES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum_bar + 1);
-  __shared__ volatile int abort_flag;
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int a_row0 = blockIdx.x * kBM;
-  const int b_row0 = blockIdx.y * BN;
-  const int split = blockIdx.z;
-  const int kb_begin = split * p.kb_per_split;
-  const int nkb = min(p.kb_per_split, p.kb_total - kb_begin);
-  const int nadapt = PARTIAL ? 0 : p.nkb_adapt;
-  const int total_it = nkb + nadapt;
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      sm100::mbar_init(&full_bar[s], 1);
-      sm100::mbar_init(&empty_bar[s], 1);
-    }
-    sm100::mbar_init(accum_bar, 1);
-    abort_flag = 0;
-    sm100::fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    sm100::tma_prefetch_desc(&tmA);
-    sm100::tma_prefetch_desc(&tmB);
-    if (nadapt) {
-      sm100::tma_prefetch_desc(&tmA2);
-      sm100::tma_prefetch_desc(&tmB2);
-    }
-  }
-  if (warp == 1) sm100::tmem_alloc(tmem_holder, kTmemCols);
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---- TMA producer ----
-      int issued = 0;
-      for (int it = 0; it < total_it; ++it) {
-        const int s = it % STAGES;
-        if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
-          set_fault(kFaultProducer, &abort_flag);
-          break;
-        }
-        if (abort_flag) break;
-        uint8_t* sa = smem + s * kStage;
-        uint8_t* sb = sa + kAbytes;
-        sm100::mbar_arrive_expect_tx(&full_bar[s], kStage);
-        if (it < nkb) {
-          const int kx = (kb_begin + it) * kElemsPerRow;
-          sm100::tma_load_2d(sa, &tmA, &full_bar[s], kx, a_row0);
-          sm100::tma_load_2d(sb, &tmB, &full_bar[s], kx, b_row0);
-        } else {
-          const int kx = (it - nkb) * kElemsPerRow;
-          sm100::tma_load_2d(sa, &tmA2, &full_bar[s], kx, a_row0);
-          sm100::tma_load_2d(sb, &tmB2, &full_bar[s], kx, b_row0);
-        }
-        issued = it + 1;
-      }
-      // Every issued load must land before the CTA may exit: wait for the
-      // latest phase of each stage that received one (at most STAGES).
-      for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it) {
-        if (!sm100::mbar_wait(&full_bar[it % STAGES], (it / STAGES) & 1))
-          set_fault(kFaultProducer, &abort_flag);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---- MMA issuer ----
-      for (int it = 0; it < total_it; ++it) {
-        const int s = it % STAGES;
-        if (!sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
-          set_fault(kFaultMma, &abort_flag);
-          break;
-        }
-        if (abort_flag) break;
-        sm100::tc_fence_after();
-        const uint32_t sa = sm100::smem_addr(smem + s * kStage);
-        const uint64_t da = sm100::smem_desc_k_sw128(sa);
-        const uint64_t db = sm100::smem_desc_k_sw128(sa + kAbytes);
-        const bool main = it < nkb;
-        const int kb_local = main ? it : it - nkb;
-        const uint32_t d = tmem + (main ? 0u : static_cast<uint32_t>(kD1));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          // 32 bytes of K per instruction: 16 bf16 or 8 tf32 elements.
-          sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, kIdesc, (kb_local > 0) || (k > 0));
-        }
-        sm100::mma_commit(&empty_bar[s]);
-      }
-      sm100::mma_commit(accum_bar);  // fires when every issued MMA has completed
-    }
-  } else {
-    // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
-    // tcgen05.ld is warp-collective: decide for the whole warp at once.
-    const bool ok = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(accum_bar, 0));
-    if (!ok && lane == 0) set_fault(kFaultEpilogue, &abort_flag);
-    sm100::tc_fence_after();
-    if (__all_sync(0xFFFFFFFFu, ok && !abort_flag)) {
-      const int quarter = warp & 3;
-      const int r = quarter * 32 + lane;
-      const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int arow = a_row0 + r;
-      const bool with_adapter = !PARTIAL && nadapt > 0;
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t v0[32], v1[32];
-        sm100::tmem_ld_32x32b_x32(tq + c, v0);
-        if (with_adapter) sm100::tmem_ld_32x32b_x32(tq + kD1 + c, v1);
-        sm100::tmem_ld_wait();
-        float f0[32], f1[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          f0[e] = __uint_as_float(v0[e]);
-          f1[e] = with_adapter ? f0[e] + __uint_as_float(v1[e]) : f0[e];
-        }
-        const int brow = b_row0 + c;  // first B row of this 32-column slice
-        if constexpr (PARTIAL) {
-          float* base = p.partial + static_cast<size_t>(split) * p.M * p.ncols;
-          if constexpr (!SWAP) {
-            // 32 consecutive columns of one row: 16-byte stores (ncols % 4 == 0)
-            if (arow < p.M) {
-              float* dst = base + static_cast<size_t>(arow) * p.ncols + brow;
-#pragma unroll
-              for (int g = 0; g < 8; ++g)
-                if (brow + g * 4 < p.ncols)
-                  *reinterpret_cast<float4*>(dst + g * 4) =
-                      make_float4(f0[g * 4], f0[g * 4 + 1], f0[g * 4 + 2], f0[g * 4 + 3]);
-            }
-          } else {
-            if (arow < p.ncols) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (brow + e < p.M) base[static_cast<size_t>(brow + e) * p.ncols + arow] = f0[e];
-            }
-          }
-        } else {
-          T* ya = static_cast<T*>(p.y_ar);
-          T* yd = static_cast<T*>(p.y_draft);
-          if constexpr (!SWAP) {
-            if (arow < p.M) {
-              const size_t off = static_cast<size_t>(arow) * p.ncols + brow;
-              const int valid = p.ncols - brow;
-              if (valid > 0) {
-                if (ya) store_row32<T>(ya + off, f0, valid);
-                if (yd) store_row32<T>(yd + off, f1, valid);
-              }
-            }
-          } else {
-            if (arow < p.ncols) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                if (brow + e < p.M) {
-                  const size_t off = static_cast<size_t>(brow + e) * p.ncols + arow;
-                  if (ya) store_one<T>(ya + off, f0[e]);
-                  if (yd) store_one<T>(yd + off, f1[e]);
-                }
-              }
-            }
-          }
-        }
-      }
-    }
-  }
-
-  sm100::tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, kTmemCols);
+// Bounded wait until *flag == epoch.
+__device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
+  if (ld_acquire_u32(flag) == epoch) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_u32(flag) == epoch) return true;
+    if (sm100::globaltimer_ns() - t0 > kWaitNs) return false;
   }
 }
 
 // ---------------------------------------------------------------------------
-// The dual GEMM, persistent. Each CTA takes tiles t = blockIdx.x,
-// blockIdx.x + gridDim.x, ... (the 128-row A tile index varies fastest, so
-// neighbouring CTAs share a B tile in L2). TMEM holds two BN-column fp32
-// accumulators, used by alternate tiles. Per tile the MMA thread accumulates
-// x W^T over all K-blocks into the tile's accumulator; the epilogue drains it
-// as y_ar and says so; the adapter product T Bm^T (two 64-wide K-blocks for
-// r = 128) is then accumulated into the same accumulator, which the epilogue
-// drains again as y_draft. The adapter K-blocks of tile i ride in the operand
-// ring after the first kInsert K-blocks of tile i + 1, so the tensor pipe works
-// on the next tile while the epilogue drains y_ar.
+// The kernel. tmA/tmB: main operands (non-swapped: x, W; swapped: W, x).
+// tmA2/tmB2: adapter operands (non-swapped: T, Bm; swapped: Bm, T). tmL: the
+// LoRA down weight A for the T tiles (non-swapped: the B side, box BN rows;
+// swapped: the A side, box 128 rows).
 // ---------------------------------------------------------------------------
-constexpr int kInsert = 6;
-
 template <typename T, int BN, bool SWAP>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                const GemmParams p, int rowsA, int rowsB) {
+                const __grid_constant__ CUtensorMap tmL, const GemmParams p) {
   constexpr int STAGES = stages_for<BN>();
   constexpr int kAbytes = kBM * kRowBytes;
   constexpr int kStage = (kBM + BN) * kRowBytes;
@@ -359,20 +191,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * kStage);
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* acc_full = empty_bar + STAGES;   // [2] main product done
-  uint64_t* ar_read = acc_full + 2;          // [2] epilogue drained y_ar
-  uint64_t* draft_full = ar_read + 2;        // [2] adapter product done
-  uint64_t* acc_empty = draft_full + 2;      // [2] epilogue drained the buffer
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_full = empty_bar + STAGES;  // [2] main product done
+  uint64_t* ar_read = acc_full + 2;         // [2] epilogue drained y_ar
+  uint64_t* draft_full = ar_read + 2;       // [2] adapter product done
+  uint64_t* acc_empty = draft_full + 2;     // [2] epilogue drained the buffer
+  uint64_t* t_stored = acc_empty + 2;       // [1] epilogue warps stored a T tile
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(t_stored + 1);
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_a = (rowsA + kBM - 1) / kBM;
-  const int tiles_b = (rowsB + BN - 1) / BN;
-  const int ntiles = tiles_a * tiles_b;
-  const int nmine = (ntiles > static_cast<int>(blockIdx.x))
-                        ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                        : 0;
+  const int tiles_a = (p.rowsA + kBM - 1) / kBM;
+  const int tiles_b = (p.rowsB + BN - 1) / BN;
+  const int ntiles = p.nT + tiles_a * tiles_b;
+  const int G = static_cast<int>(gridDim.x), C = static_cast<int>(blockIdx.x);
+  const int nmine = (ntiles > C) ? (ntiles - 1 - C) / G + 1 : 0;
+  // This CTA's T tiles are its first nt_mine tiles (their global indices are
+  // the lowest); main tile li has ordinal li - nt_mine among its main tiles,
+  // which indexes the ar_read / draft_full barriers and their phases.
+  const int nt_mine = (p.nT > C) ? (p.nT - 1 - C) / G + 1 : 0;
   const int nkb = p.kb_total;
   const bool adapter = p.nkb_adapt > 0;
   const int nad = adapter ? p.nkb_adapt : 0;
@@ -389,6 +225,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::mbar_init(&draft_full[b], 1);
       sm100::mbar_init(&acc_empty[b], 4);
     }
+    sm100::mbar_init(t_stored, 4);
     abort_flag = 0;
     sm100::fence_mbar_init();
   }
@@ -398,6 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (adapter) {
       sm100::tma_prefetch_desc(&tmA2);
       sm100::tma_prefetch_desc(&tmB2);
+      sm100::tma_prefetch_desc(&tmL);
     }
   }
   if (warp == 1) sm100::tmem_alloc(tmem_holder, kTmemCols);
@@ -406,17 +244,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  // The operand stream of this CTA, in ring order: for local tile i, its main
-  // K-blocks 0..ins-1, then the adapter K-blocks of tile i-1, then its main
-  // K-blocks ins..nkb-1; after the last tile, that tile's adapter K-blocks.
-  // Item q of local tile i (0 <= q < nkb + nad, nad only for i >= 1) maps to:
-  //   q < ins            -> main block q of tile i
-  //   ins <= q < ins+nad -> adapter block q-ins of tile i-1
-  //   otherwise          -> main block q-nad of tile i
-  auto tile_coords = [&](int li, int& a0, int& b0) {
-    const int t = static_cast<int>(blockIdx.x) + li * static_cast<int>(gridDim.x);
-    a0 = (t % tiles_a) * kBM;
-    b0 = (t / tiles_a) * BN;
+  // Local tile li of this CTA: global tile t = C + li * G. t < nT is T tile t
+  // (its A rows start at t * 128: rows of x, or with swapped operands rows of
+  // the LoRA A); otherwise main tile u = t - nT at (u % tiles_a, u / tiles_a).
+  struct Tile {
+    bool is_t;
+    int a0, b0;  // first A row, first B row
+    int tt;      // T tile index
+  };
+  auto tile_at = [&](int li) {
+    const int t = C + li * G;
+    Tile x;
+    x.is_t = t < p.nT;
+    x.tt = t;
+    if (x.is_t) {
+      x.a0 = t * kBM;
+      x.b0 = 0;
+    } else {
+      const int u = t - p.nT;
+      x.a0 = (u % tiles_a) * kBM;
+      x.b0 = (u / tiles_a) * BN;
+    }
+    return x;
+  };
+  // Ring items of local iteration li (li = 0..nmine): the first ins main
+  // K-blocks of tile li, the adapter K-blocks of tile li-1 (if it was a main
+  // tile), then the remaining main K-blocks of tile li.
+  auto counts = [&](int li, int& nmain, int& nadp) {
+    nmain = (li < nmine) ? nkb : 0;
+    nadp = (li > 0 && adapter && !tile_at(li - 1).is_t) ? nad : 0;
   };
 
   if (warp == 0) {
@@ -424,7 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ---- TMA producer ----
       int it = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* ma, const CUtensorMap* mb, int kx, int a0, int b0) {
+      auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx) {
         const int s = it % STAGES;
         if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
           set_fault(kFaultProducer, &abort_flag);
@@ -437,25 +293,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         uint8_t* sa = smem + s * kStage;
         sm100::mbar_arrive_expect_tx(&full_bar[s], kStage);
-        sm100::tma_load_2d(sa, ma, &full_bar[s], kx, a0);
-        sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, b0);
+        sm100::tma_load_2d(sa, ma, &full_bar[s], kx, ay);
+        sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
         ++it;
       };
+      auto load_main = [&](const Tile& x, int kb) {
+        const int kx = kb * kElemsPerRow;
+        if (x.is_t) {
+          if constexpr (SWAP) load(&tmL, x.a0, &tmB, 0, kx);
+          else load(&tmA, x.a0, &tmL, 0, kx);
+        } else {
+          load(&tmA, x.a0, &tmB, x.b0, kx);
+        }
+      };
       for (int li = 0; li <= nmine && ok; ++li) {
-        int a0 = 0, b0 = 0, pa0 = 0, pb0 = 0;
-        if (li < nmine) tile_coords(li, a0, b0);
-        if (li > 0) tile_coords(li - 1, pa0, pb0);
-        const int nmain = (li < nmine) ? nkb : 0;
-        const int nadp = (li > 0) ? nad : 0;
+        int nmain, nadp;
+        counts(li, nmain, nadp);
+        const Tile cur = tile_at(li);
+        const Tile prev = (li > 0) ? tile_at(li - 1) : cur;
         const int items = nmain + nadp;
         for (int q = 0; q < items && ok; ++q) {
           const int qa = q - min(ins, nmain);
           if (q < min(ins, nmain)) {
-            load(&tmA, &tmB, q * kElemsPerRow, a0, b0);
+            load_main(cur, q);
           } else if (qa < nadp) {
-            load(&tmA2, &tmB2, qa * kElemsPerRow, pa0, pb0);
+            if (qa == 0) {
+              // T must be stored before its TMA load: wait for the T tile(s)
+              bool ready = true;
+              if constexpr (SWAP) {
+                for (int t = 0; t < p.nT && ready; ++t)
+                  ready = wait_flag(p.t_flags + t, p.epoch);
+              } else {
+                ready = wait_flag(p.t_flags + prev.a0 / kBM, p.epoch);
+              }
+              if (!ready) {
+                set_fault(kFaultProducer, &abort_flag);
+                ok = false;
+                break;
+              }
+              fence_proxy_async_global();
+            }
+            load(&tmA2, prev.a0, &tmB2, prev.b0, qa * kElemsPerRow);
           } else {
-            load(&tmA, &tmB, (q - nadp) * kElemsPerRow, a0, b0);
+            load_main(cur, q - nadp);
           }
         }
       }
@@ -468,7 +348,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ---- MMA issuer ----
       int it = 0;
       bool ok = true;
-      auto consume = [&](uint32_t d, bool accumulate_first) {
+      auto consume = [&](uint32_t d, uint32_t idesc, bool accumulate_first) {
         const int s = it % STAGES;
         if (!sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
           set_fault(kFaultMma, &abort_flag);
@@ -481,19 +361,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint64_t db = sm100::smem_desc_k_sw128(sa + kAbytes);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, kIdesc, accumulate_first || (k > 0));
+          sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
         sm100::mma_commit(&empty_bar[s]);
         ++it;
       };
       for (int li = 0; li <= nmine && ok; ++li) {
+        int nmain, nadp;
+        counts(li, nmain, nadp);
         const int buf = li & 1, pbuf = (li - 1) & 1;
         const uint32_t d = tmem + static_cast<uint32_t>(buf * kAcc);
         const uint32_t pd = tmem + static_cast<uint32_t>(pbuf * kAcc);
-        const int nmain = (li < nmine) ? nkb : 0;
-        const int nadp = (li > 0) ? nad : 0;
+        const uint32_t idesc = (nmain && tile_at(li).is_t && !SWAP) ? p.idesc_t : kIdesc;
         const int items = nmain + nadp;
-        if (nmain && li >= 2 &&
-            !sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {  // buffer drained
+        if (nmain && li >= 2 && !sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
           set_fault(kFaultMma, &abort_flag);
           break;
         }
@@ -501,22 +381,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int q = 0; q < items && ok; ++q) {
           const int qa = q - min(ins, nmain);
           if (q < min(ins, nmain)) {
-            consume(d, q > 0);
+            consume(d, idesc, q > 0);
             if (q == nmain - 1) sm100::mma_commit(&acc_full[buf]);
           } else if (qa < nadp) {
+            const int mo = li - 1 - nt_mine;  // main ordinal of the previous tile
             if (qa == 0) {
-              if (!sm100::mbar_wait(&ar_read[pbuf], ((li - 1) >> 1) & 1)) {
+              if (!sm100::mbar_wait(&ar_read[mo & 1], (mo >> 1) & 1)) {
                 set_fault(kFaultMma, &abort_flag);
                 ok = false;
                 break;
               }
               sm100::tc_fence_after();
             }
-            consume(pd, true);  // adds T Bm^T onto y_ar of the previous tile
-            if (qa == nadp - 1) sm100::mma_commit(&draft_full[pbuf]);
+            consume(pd, kIdesc, true);  // adds T Bm^T onto y_ar of the previous tile
+            if (qa == nadp - 1) sm100::mma_commit(&draft_full[mo & 1]);
           } else {
             const int kb = q - nadp;
-            consume(d, kb > 0);
+            consume(d, idesc, kb > 0);
             if (kb == nmain - 1) sm100::mma_commit(&acc_full[buf]);
           }
         }
@@ -525,29 +406,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
+    const int rr = quarter * 32 + lane;
     T* ya = static_cast<T*>(p.y_ar);
     T* yd = static_cast<T*>(p.y_draft);
-    auto drain = [&](uint32_t acc, int a0, int b0, T* y) {
-      if (!y) return;  // output not requested: nothing to read
+    T* tb = static_cast<T*>(p.t_buf);
+    // Drain accumulator columns [0, ncol) into y (row-major, ld columns, nrows rows).
+    auto drain = [&](uint32_t acc, int a0, int b0, T* y, int ld, int nrows, int ncol,
+                     float mul) {
+      if (!y) return;
       const uint32_t tq = acc + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int arow = a0 + r;
-      for (int c = 0; c < BN; c += 32) {
+      const int arow = a0 + rr;
+      for (int c = 0; c < ncol; c += 32) {
         uint32_t v[32];
         sm100::tmem_ld_32x32b_x32(tq + c, v);
         sm100::tmem_ld_wait();
         float f[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * mul;
         const int brow = b0 + c;
         if constexpr (!SWAP) {
-          if (arow < p.M && brow < p.ncols)
-            store_row32<T>(y + static_cast<size_t>(arow) * p.ncols + brow, f, p.ncols - brow);
+          // row = A row, column = B row
+          if (arow < nrows && brow < ld)
+            store_row32<T>(y + static_cast<size_t>(arow) * ld + brow, f, ld - brow);
         } else {
-          if (arow < p.ncols) {
+          // row = B row, column = A row
+          if (arow < ld) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * p.ncols + arow, f[e]);
+              if (brow + e < nrows)
+                store_one<T>(y + static_cast<size_t>(brow + e) * ld + arow, f[e]);
           }
         }
       }
@@ -555,26 +442,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int li = 0; li < nmine; ++li) {
       const int buf = li & 1;
       const uint32_t acc = tmem + static_cast<uint32_t>(buf * kAcc);
-      int a0, b0;
-      tile_coords(li, a0, b0);
+      const Tile x = tile_at(li);
       const bool got = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&acc_full[buf], (li >> 1) & 1));
       if (!got || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
       }
       sm100::tc_fence_after();
-      drain(acc, a0, b0, ya);
+      if (x.is_t) {
+        // T = scale * x A^T: non-swapped, rows of x by r columns; swapped, r
+        // rows (rows of A) by the M columns of x.
+        if constexpr (!SWAP) drain(acc, x.a0, 0, tb, p.r, p.M, p.r, p.scale);
+        else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.scale);
+        sm100::tc_fence_before();
+        __threadfence();
+        __syncwarp();
+        // One thread publishes the tile once all four epilogue warps stored
+        // their rows. T tiles are this CTA's tiles 0..nt_mine-1, so li counts
+        // the completed phases of t_stored; warp 2 frees the accumulator only
+        // after its wait, so the other warps cannot get two T tiles ahead.
+        if (lane == 0) {
+          sm100::mbar_arrive(t_stored);
+          if (warp == 2) {
+            if (sm100::mbar_wait(t_stored, li & 1)) {
+              fence_proxy_async_global();
+              st_release_u32(p.t_flags + x.tt, p.epoch);
+            } else {
+              set_fault(kFaultEpilogue, &abort_flag);
+            }
+          }
+          sm100::mbar_arrive(&acc_empty[buf]);
+        }
+        __syncwarp();
+        continue;
+      }
+      drain(acc, x.a0, x.b0, ya, p.ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(adapter ? &ar_read[buf] : &acc_empty[buf]);
+      const int mo = li - nt_mine;
+      if (lane == 0) sm100::mbar_arrive(adapter ? &ar_read[mo & 1] : &acc_empty[buf]);
       if (!adapter) continue;
-      const bool got2 = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&draft_full[buf], (li >> 1) & 1));
+      const bool got2 =
+          __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&draft_full[mo & 1], (mo >> 1) & 1));
       if (!got2 || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
       }
       sm100::tc_fence_after();
-      drain(acc, a0, b0, yd);
+      drain(acc, x.a0, x.b0, yd, p.ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
@@ -586,35 +501,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// T = scale * sum_s partial[s]  (splits summed in index order), rounded to T.
-// Four consecutive elements per thread (count is a multiple of 4).
-template <typename T>
-__global__ void reduce_t_kernel(const float* __restrict__ partial, int splits, size_t count,
-                                float scale, T* __restrict__ out) {
-  const size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
-  if (i >= count) return;
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k = 0; k < splits; ++k) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(partial + static_cast<size_t>(k) * count + i));
-    s.x += v.x;
-    s.y += v.y;
-    s.z += v.z;
-    s.w += v.w;
-  }
-  s.x *= scale;
-  s.y *= scale;
-  s.z *= scale;
-  s.w *= scale;
-  if constexpr (sizeof(T) == 2) {
-    uint2 w;
-    w.x = pack_bf16x2(s.x, s.y);
-    w.y = pack_bf16x2(s.z, s.w);
-    *reinterpret_cast<uint2*>(out + i) = w;
-  } else {
-    *reinterpret_cast<float4*>(out + i) = s;
   }
 }
 
@@ -654,27 +540,7 @@ bool make_map(CUtensorMap* map, const void* ptr, int dtype, int k_elems, int row
   return r == CUDA_SUCCESS;
 }
 
-template <typename T, int BN, bool SWAP, bool PARTIAL>
-int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const GemmParams& p, cudaStream_t st) {
-  constexpr int bytes = smem_bytes<BN, stages_for<BN>()>();
-  auto kern = gemm_kernel<T, BN, SWAP, PARTIAL>;
-  // The shared-memory opt-in is per device; remember which devices have it.
-  static std::atomic<uint64_t> attr_done{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return UNO_ERR_CUDA;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (!bit || !(attr_done.load(std::memory_order_relaxed) & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
-      return UNO_ERR_CUDA;
-    attr_done.fetch_or(bit, std::memory_order_relaxed);
-  }
-  kern<<<grid, kGemmThreads, bytes, st>>>(a, b, a2, b2, p);
-  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
-}
-
-int sm_count_dual() {
+int sm_count() {
   static int cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -685,13 +551,29 @@ int sm_count_dual() {
   return n;
 }
 
+// A fresh value per call for the T-tile flags. Seeded from the clock so that
+// a workspace left over from another process is not mistaken for this call's.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{0};
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const auto now = std::chrono::high_resolution_clock::now().time_since_epoch().count();
+    counter.store(static_cast<uint32_t>(now) * 2654435761u);
+  });
+  uint32_t e;
+  do {
+    e = counter.fetch_add(1) + 1;
+  } while (e == 0);
+  return e;
+}
+
 template <typename T, int BN, bool SWAP>
-int launch_dual(int rowsA, int rowsB, const CUtensorMap& a, const CUtensorMap& b,
-                const CUtensorMap& a2, const CUtensorMap& b2, const GemmParams& p,
+int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                const CUtensorMap& b2, const CUtensorMap& l, const GemmParams& p,
                 cudaStream_t st) {
   constexpr int bytes = smem_bytes<BN, stages_for<BN>()>();
   auto kern = dual_kernel<T, BN, SWAP>;
-  static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<uint64_t> attr_done{0};  // devices with the shared-memory opt-in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return UNO_ERR_CUDA;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
@@ -701,50 +583,27 @@ int launch_dual(int rowsA, int rowsB, const CUtensorMap& a, const CUtensorMap& b
       return UNO_ERR_CUDA;
     attr_done.fetch_or(bit, std::memory_order_relaxed);
   }
-  const long long tiles =
-      static_cast<long long>((rowsA + kBM - 1) / kBM) * ((rowsB + BN - 1) / BN);
-  long long grid = sm_count_dual();
+  const long long tiles = p.nT + static_cast<long long>((p.rowsA + kBM - 1) / kBM) *
+                                     ((p.rowsB + BN - 1) / BN);
+  long long grid = sm_count();
   if (grid > tiles) grid = tiles;
-  kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, p, rowsA, rowsB);
+  kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, l, p);
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
 template <typename T, bool SWAP>
-int launch_dual_bn(int bn, int rowsA, int rowsB, const CUtensorMap& a, const CUtensorMap& b,
-                   const CUtensorMap& a2, const CUtensorMap& b2, const GemmParams& p,
+int launch_dual_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                   const CUtensorMap& b2, const CUtensorMap& l, const GemmParams& p,
                    cudaStream_t st) {
   switch (bn) {
-    case 32: return launch_dual<T, 32, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
-    case 64: return launch_dual<T, 64, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
-    case 128: return launch_dual<T, 128, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
-    default: return launch_dual<T, 256, SWAP>(rowsA, rowsB, a, b, a2, b2, p, st);
-  }
-}
-
-// Dispatch over the B-tile height (32, 64, 128 or 256 rows).
-template <typename T, bool SWAP, bool PARTIAL>
-int launch_bn(int bn, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
-              const CUtensorMap& a2, const CUtensorMap& b2, const GemmParams& p,
-              cudaStream_t st) {
-  switch (bn) {
-    case 32: return launch_gemm<T, 32, SWAP, PARTIAL>(grid, a, b, a2, b2, p, st);
-    case 64: return launch_gemm<T, 64, SWAP, PARTIAL>(grid, a, b, a2, b2, p, st);
-    case 128: return launch_gemm<T, 128, SWAP, PARTIAL>(grid, a, b, a2, b2, p, st);
-    default: return launch_gemm<T, 256, SWAP, PARTIAL>(grid, a, b, a2, b2, p, st);
+    case 32: return launch_dual<T, 32, SWAP>(a, b, a2, b2, l, p, st);
+    case 64: return launch_dual<T, 64, SWAP>(a, b, a2, b2, l, p, st);
+    case 128: return launch_dual<T, 128, SWAP>(a, b, a2, b2, l, p, st);
+    default: return launch_dual<T, 256, SWAP>(a, b, a2, b2, l, p, st);
   }
 }
 
 int bn_for(int rows) { return rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256; }
-
-struct Plan {
-  bool swap;
-  int esize;
-  int kb_main;   // K-blocks over d_in
-  int kb_adapt;  // K-blocks over r
-  // T product
-  int t_bn, t_grid_x, t_splits, t_per;
-  size_t t_bytes, partial_bytes;
-};
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -756,26 +615,21 @@ bool dual_sizes_ok(int M, int d_in, int d_out, int r, int dtype) {
          d_out <= (1 << 24);
 }
 
+struct Plan {
+  bool swap;
+  int esize, kb_main, kb_adapt, nT;
+  size_t t_bytes, flag_bytes;
+};
+
 Plan make_plan(int M, int d_in, int r, int dtype) {
   Plan pl{};
   pl.esize = (dtype == UNO_BF16) ? 2 : 4;
   pl.swap = M <= 256;
   pl.kb_main = (d_in * pl.esize + kRowBytes - 1) / kRowBytes;
   pl.kb_adapt = (r * pl.esize + kRowBytes - 1) / kRowBytes;
-  if (pl.swap) {  // A op = A (r rows), B op = x (M rows)
-    pl.t_bn = bn_for(M);
-    pl.t_grid_x = (r + kBM - 1) / kBM;
-  } else {        // A op = x (M rows), B op = A (r rows)
-    pl.t_bn = bn_for(r);
-    pl.t_grid_x = (M + kBM - 1) / kBM;
-  }
-  int splits = (kSmSplitTarget + pl.t_grid_x - 1) / pl.t_grid_x;
-  if (splits > pl.kb_main) splits = pl.kb_main;
-  if (splits < 1) splits = 1;
-  pl.t_per = (pl.kb_main + splits - 1) / splits;
-  pl.t_splits = (pl.kb_main + pl.t_per - 1) / pl.t_per;
+  pl.nT = pl.swap ? (r + kBM - 1) / kBM : (M + kBM - 1) / kBM;
   pl.t_bytes = align256(static_cast<size_t>(M) * r * pl.esize);
-  pl.partial_bytes = align256(static_cast<size_t>(pl.t_splits) * M * r * sizeof(float));
+  pl.flag_bytes = align256(static_cast<size_t>(pl.nT) * sizeof(uint32_t));
   return pl;
 }
 
@@ -786,62 +640,54 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
   const Plan pl = make_plan(M, d_in, r, dtype);
   const bool adapter = (y_draft != nullptr);
   T* Tbuf = static_cast<T*>(workspace);
-  float* partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.t_bytes);
-  CUtensorMap mx, mW, mBm, mT;
-  const int xrows_box = pl.swap ? bn_for(M) : kBM;
-  int st_code = UNO_OK;
-
-  // 1. T = scale * x A^T (only when the draft output is wanted).
-  if (adapter) {
-    CUtensorMap ta, tb;
-    bool ok;
-    if (pl.swap) {
-      ok = make_map(&ta, A, dtype, d_in, r, kBM) && make_map(&tb, x, dtype, d_in, M, pl.t_bn);
-    } else {
-      ok = make_map(&ta, x, dtype, d_in, M, kBM) && make_map(&tb, A, dtype, d_in, r, pl.t_bn);
-    }
-    if (!ok) return UNO_ERR_CUDA;
-    GemmParams gp{};
-    gp.kb_total = pl.kb_main;
-    gp.kb_per_split = pl.t_per;
-    gp.nkb_adapt = 0;
-    gp.M = M;
-    gp.ncols = r;
-    gp.partial = partial;
-    const dim3 grid(pl.t_grid_x, 1, pl.t_splits);
-    st_code = pl.swap ? launch_bn<T, true, true>(pl.t_bn, grid, ta, tb, ta, tb, gp, st)
-                      : launch_bn<T, false, true>(pl.t_bn, grid, ta, tb, ta, tb, gp, st);
-    if (st_code != UNO_OK) return st_code;
-    const size_t count = static_cast<size_t>(M) * r;
-    reduce_t_kernel<T><<<static_cast<unsigned>((count / 4 + 255) / 256), 256, 0, st>>>(
-        partial, pl.t_splits, count, scale, Tbuf);
-    if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
-  }
-
-  // 2. dual GEMM over W.
+  uint32_t* flags = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + pl.t_bytes);
   GemmParams gp{};
   gp.kb_total = pl.kb_main;
-  gp.kb_per_split = pl.kb_main;
   gp.nkb_adapt = adapter ? pl.kb_adapt : 0;
   gp.M = M;
   gp.ncols = d_out;
+  gp.nT = adapter ? pl.nT : 0;
+  gp.r = r;
+  gp.epoch = next_epoch();
+  if (adapter) {
+    // A captured launch replays with the epoch it was captured with, so under
+    // stream capture the flags are cleared by a node of their own first.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return UNO_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone &&
+        cudaMemsetAsync(flags, 0, pl.flag_bytes, st) != cudaSuccess)
+      return UNO_ERR_CUDA;
+  }
+  gp.scale = scale;
   gp.y_ar = y_ar;
   gp.y_draft = y_draft;
+  gp.t_buf = Tbuf;
+  gp.t_flags = flags;
+  const bool tf32 = (dtype == UNO_F32);
+  CUtensorMap mA, mB, mA2, mB2, mL;
   if (pl.swap) {
     const int bn = bn_for(M);
-    bool ok = make_map(&mW, W, dtype, d_in, d_out, kBM) && make_map(&mx, x, dtype, d_in, M, bn);
-    if (adapter) ok = ok && make_map(&mBm, Bm, dtype, r, d_out, kBM) &&
-                      make_map(&mT, Tbuf, dtype, r, M, bn);
+    gp.rowsA = d_out;
+    gp.rowsB = M;
+    gp.idesc_t = sm100::instr_desc(tf32, kBM, bn);
+    bool ok = make_map(&mA, W, dtype, d_in, d_out, kBM) && make_map(&mB, x, dtype, d_in, M, bn);
+    if (adapter)
+      ok = ok && make_map(&mA2, Bm, dtype, r, d_out, kBM) &&
+           make_map(&mB2, Tbuf, dtype, r, M, bn) && make_map(&mL, A, dtype, d_in, r, kBM);
     if (!ok) return UNO_ERR_CUDA;
-    return launch_dual_bn<T, true>(bn, d_out, M, mW, mx, adapter ? mBm : mW, adapter ? mT : mx,
-                                   gp, st);
+    if (!adapter) mA2 = mB2 = mL = mA;
+    return launch_dual_bn<T, true>(bn, mA, mB, mA2, mB2, mL, gp, st);
   }
-  bool ok = make_map(&mx, x, dtype, d_in, M, xrows_box) && make_map(&mW, W, dtype, d_in, d_out, 256);
-  if (adapter) ok = ok && make_map(&mT, Tbuf, dtype, r, M, kBM) &&
-                    make_map(&mBm, Bm, dtype, r, d_out, 256);
+  gp.rowsA = M;
+  gp.rowsB = d_out;
+  gp.idesc_t = sm100::instr_desc(tf32, kBM, (r + 15) / 16 * 16);
+  bool ok = make_map(&mA, x, dtype, d_in, M, kBM) && make_map(&mB, W, dtype, d_in, d_out, 256);
+  if (adapter)
+    ok = ok && make_map(&mA2, Tbuf, dtype, r, M, kBM) &&
+         make_map(&mB2, Bm, dtype, r, d_out, 256) && make_map(&mL, A, dtype, d_in, r, 256);
   if (!ok) return UNO_ERR_CUDA;
-  return launch_dual<T, 256, false>(M, d_out, mx, mW, adapter ? mT : mx, adapter ? mBm : mW, gp,
-                                    st);
+  if (!adapter) mA2 = mB2 = mL = mA;
+  return launch_dual<T, 256, false>(mA, mB, mA2, mB2, mL, gp, st);
 }
 
 }  // namespace
@@ -849,7 +695,7 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
 extern "C" size_t uno_dualpath_workspace_bytes(int M, int d_in, int d_out, int r, int dtype) {
   if (!dual_sizes_ok(M, d_in, d_out, r, dtype)) return 0;
   const Plan pl = make_plan(M, d_in, r, dtype);
-  return pl.t_bytes + pl.partial_bytes;
+  return pl.t_bytes + pl.flag_bytes;
 }
 
 extern "C" int uno_dualpath_linear(const void* x, const void* W, const void* A, const void* Bm,
