@@ -57,6 +57,29 @@ def _peaks():
     return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's value (all ranks must call it, in the same
+    order); the tensor lives on `device` (CUDA under NCCL, CPU under gloo)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seeds(rank: int) -> tuple[int, int]:
+    """(input seed, Philox key) of one replica. Replicas decode independent
+    batches, so each draws its synthetic inputs and its acceptance / resampling
+    uniforms from its own stream."""
+    return 17 + rank, 1234 + rank
+
+
+def whole_job_rate(rows_per_step: int, world: int, ms_step_max: float) -> float:
+    """Rows per second over all ranks: each rank decodes rows_per_step rows per
+    step, and the slowest rank's step time bounds the job."""
+    return world * rows_per_step / (ms_step_max / 1e3)
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -141,9 +164,10 @@ class BatchedDecode:
 
     name = "batched_decode_b64_k16"
 
-    def __init__(self, dev, seed):
+    def __init__(self, dev, seed, philox_seed=1234):
         from lossless_decoding_b200 import api
         from lossless_decoding_b200.inputs import dualpath_inputs, verify_inputs
+        self.philox_seed = philox_seed
         self.api = api
         self.B, self.K, self.V = B64, K16, QWEN3_8B_VOCAB
         self.M = self.B * self.K
@@ -185,7 +209,8 @@ class BatchedDecode:
                 ev[1][i].record()
         if ev is not None:
             ev[2].record()
-        api.verify_block(self.v.p_logits, self.v.q_logits, self.v.draft_tokens, seed=1234,
+        api.verify_block(self.v.p_logits, self.v.q_logits, self.v.draft_tokens,
+                         seed=self.philox_seed,
                          step=seed_step, out=self.out, workspace=self.vws)
         if ev is not None:
             ev[3].record()
@@ -242,9 +267,10 @@ class SingleSequence(BatchedDecode):
 
     name = "qwen3_8b_b1"
 
-    def __init__(self, dev, seed):
+    def __init__(self, dev, seed, philox_seed=1234):
         from lossless_decoding_b200 import api
         from lossless_decoding_b200.inputs import dualpath_inputs
+        self.philox_seed = philox_seed
         self.api = api
         self.B, self.K, self.V = 1, K16, QWEN3_8B_VOCAB
         self.M = self.K + 1
@@ -280,7 +306,7 @@ class SingleSequence(BatchedDecode):
             ev[2].record()
         p = y_ar.view(1, self.M, self.V)
         q = y_dr[: self.K].view(1, self.K, self.V)
-        api.verify_block(p, q, self.drafts, seed=1234, step=seed_step, out=self.out,
+        api.verify_block(p, q, self.drafts, seed=self.philox_seed, step=seed_step, out=self.out,
                          workspace=self.vws)
         if ev is not None:
             ev[3].record()
@@ -428,7 +454,8 @@ def run_ours(args):
                                              device_id=dev)
     from lossless_decoding_b200 import api
 
-    wl = WORKLOADS[args.workload](dev, seed=17 + rank)
+    input_seed, philox_seed = replica_seeds(rank)
+    wl = WORKLOADS[args.workload](dev, seed=input_seed, philox_seed=philox_seed)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
@@ -436,12 +463,8 @@ def run_ours(args):
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     for i in range(args.warmup):
         wl.step(i)
@@ -462,18 +485,23 @@ def run_ours(args):
     barrier()
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
-    ms_step = max_over_ranks(ms_total / args.steps)
+    ms_step = rank_max(ms_total / args.steps)
     gemm_ms = [wl.op_times(e)[0] for e in events]
     ver_ms = [wl.op_times(e)[1] for e in events]
     emitted = wl.emitted()
     faults = api.device_fault_flags(clear=True)
 
     rows_per_step = wl.B * wl.K
-    value = world * rows_per_step / (ms_step / 1e3)
+    value = whole_job_rate(rows_per_step, world, ms_step)
     peaks = _peaks()
     gemm_avg = sum(gemm_ms) / len(gemm_ms)
     ver_avg = sum(ver_ms) / len(ver_ms)
     gemm_tflops = wl.gemm_flops / (gemm_avg / 1e3) / 1e12
+    per_proj = {}
+    for j, (name, d, *_) in enumerate(wl.layers):
+        us = 1e3 * sum(e[0][j].elapsed_time(e[1][j]) for e in events) / len(events)
+        fl = _dual_flops(d.x.shape[0], d.x.shape[1], d.W.shape[0], RANK)
+        per_proj[name] = {"us": round(us, 2), "tflops": round(fl / (us / 1e6) / 1e12, 1)}
     ver_gbs = wl.verify_bytes / (ver_avg / 1e3) / 1e9
     dominant_gemm = gemm_avg >= ver_avg
     roof_gemm = {"kernel": "dual_kernel (T tiles, x W^T and T Bm^T in one persistent tcgen05 launch)",
@@ -501,8 +529,8 @@ def run_ours(args):
         wl.e2e_step(host, 100 + i)
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps)
-    e2e_value = world * rows_per_step / (e2e_ms / 1e3)
+    e2e_ms = rank_max(e0.elapsed_time(e1) / e_steps)
+    e2e_value = whole_job_rate(rows_per_step, world, e2e_ms)
 
     if rank == 0:
         line = {
@@ -512,7 +540,7 @@ def run_ours(args):
             "dtype": "bf16", "data": "synthetic (seeded random weights, activations, logits)",
             "config": wl.config(),
             "emitted_tokens_per_s": world * emitted / (ms_step / 1e3),
-            "gemm_tflops": gemm_tflops, "verify_gbs": ver_gbs,
+            "gemm_tflops": gemm_tflops, "verify_gbs": ver_gbs, "gemm_per_projection": per_proj,
             "roofline": roof_gemm if dominant_gemm else roof_ver,
             "roofline_verify" if dominant_gemm else "roofline_gemm":
                 roof_ver if dominant_gemm else roof_gemm,
