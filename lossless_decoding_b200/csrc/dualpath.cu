@@ -18,11 +18,15 @@
 //  * main tiles: a 128 x BN tile of x W^T over all of d_in, accumulated in
 //    TMEM; the epilogue drains it as y_ar, then the adapter product T Bm^T is
 //    accumulated onto the same accumulator and drained as y_draft.
-// Warp roles: warp 0 issues TMA loads into a multi-stage shared-memory ring,
-// warp 1 owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain
-// TMEM with tcgen05.ld. Two accumulator buffers alternate between tiles, and
-// the adapter K-blocks of a tile ride in the ring a few K-blocks into the next
-// tile, so the tensor pipe keeps working while the epilogue drains.
+// Warp roles: two producer warps issue TMA loads into a multi-stage
+// shared-memory ring (a thread with copies in flight stalls at its next
+// mbarrier operation until they land, so one producer would keep a single
+// stage in flight); two issuer threads alternate K-blocks of tcgen05.mma (a thread that
+// has committed stalls the same way until its MMAs finish); four epilogue
+// warps drain TMEM with tcgen05.ld. Two accumulator buffers alternate between
+// tiles, and the adapter K-blocks of a tile ride in the ring a few K-blocks
+// into the next tile, so the tensor pipe keeps working while the epilogue
+// drains.
 //
 // A main tile's producer reads T only after the T tile's flag holds the
 // call's epoch (acquire, then an async-proxy fence before the TMA load). T
@@ -54,8 +58,14 @@ namespace {
 
 constexpr int kBM = 128;           // MMA M (rows of the A operand per tile)
 constexpr int kRowBytes = 128;     // bytes of K per tile row and stage (one swizzle row)
-constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+// Warp roles: 0-3 epilogue (TMEM lane quarter = warp), 4-5 MMA issuers (4
+// owns TMEM), kFirstProducer.. TMA producers.
+constexpr int kMmaWarp0 = 4;
+constexpr int kFirstProducer = 6;
+constexpr int kProducers = 2;
+constexpr int kGemmThreads = (kFirstProducer + kProducers) * 32;
 constexpr int kInsert = 6;         // main K-blocks of the next tile before an adapter
+constexpr int kPrefetch = 8;       // K-blocks of L2 prefetch ahead of the weight loads
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum : unsigned { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
@@ -154,6 +164,30 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+__device__ __forceinline__ void st_release_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(sm100::smem_addr(p)), "r"(v)
+               : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];"
+               : "=r"(v)
+               : "r"(sm100::smem_addr(p))
+               : "memory");
+  return v;
+}
+
+// Bounded wait until the other MMA issuer has handed over ring item `it`.
+__device__ bool wait_order(const int* order, int it, volatile int* abort_flag) {
+  if (ld_acquire_shared(order) == it) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  for (uint32_t k = 1;; ++k) {
+    if (ld_acquire_shared(order) == it) return true;
+    if ((k & 255u) == 0 && (*abort_flag || sm100::globaltimer_ns() - t0 > kWaitNs)) return false;
+  }
+}
+
 // Bounded wait until *flag == epoch.
 __device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
   if (ld_acquire_u32(flag) == epoch) return true;
@@ -197,6 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_empty = draft_full + 2;     // [2] epilogue drained the buffer
   uint64_t* t_stored = acc_empty + 2;       // [1] epilogue warps stored a T tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(t_stored + 1);
+  int* order = reinterpret_cast<int*>(tmem_holder + 1);  // next ring item to issue
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,16 +255,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      sm100::mbar_init(&acc_full[b], 1);
+      sm100::mbar_init(&acc_full[b], 2);  // one commit per MMA issuer
       sm100::mbar_init(&ar_read[b], 4);
-      sm100::mbar_init(&draft_full[b], 1);
+      sm100::mbar_init(&draft_full[b], 2);
       sm100::mbar_init(&acc_empty[b], 4);
     }
     sm100::mbar_init(t_stored, 4);
+    *order = 0;
     abort_flag = 0;
     sm100::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kFirstProducer && lane == 0) {
     sm100::tma_prefetch_desc(&tmA);
     sm100::tma_prefetch_desc(&tmB);
     if (adapter) {
@@ -238,7 +274,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::tma_prefetch_desc(&tmL);
     }
   }
-  if (warp == 1) sm100::tmem_alloc(tmem_holder, kTmemCols);
+  if (warp == kMmaWarp0) sm100::tmem_alloc(tmem_holder, kTmemCols);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -267,19 +303,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     return x;
   };
-  // Ring items of local iteration li (li = 0..nmine): the first ins main
-  // K-blocks of tile li, the adapter K-blocks of tile li-1 (if it was a main
-  // tile), then the remaining main K-blocks of tile li.
-  auto counts = [&](int li, int& nmain, int& nadp) {
-    nmain = (li < nmine) ? nkb : 0;
-    nadp = (li > 0 && adapter && !tile_at(li - 1).is_t) ? nad : 0;
+  // Ring items of local tile li: the first ins main K-blocks of tile li,
+  // the adapter K-blocks of tile li-1 (if that was a main tile other than the
+  // last: its adapter accumulates in place onto its drained y_ar), the
+  // remaining main K-blocks, and for this CTA's last tile (a main tile) its
+  // own adapter K-blocks into the other accumulator buffer, so that one drain
+  // writes both outputs.
+  struct Counts {
+    int nmain, nprev, nself;
+  };
+  auto counts = [&](int li) {
+    Counts c;
+    c.nmain = nkb;
+    c.nprev = (li > 0 && adapter && !tile_at(li - 1).is_t) ? nad : 0;
+    c.nself = (li == nmine - 1 && adapter && !tile_at(li).is_t) ? nad : 0;
+    return c;
+  };
+  // Item q of tile li: kind (0 main, 1 previous tile's adapter, 2 own adapter)
+  // and its K-block index within that kind.
+  auto item_of = [&](const Counts& c, int q) -> int2 {
+    const int head = min(ins, c.nmain);
+    if (q < head) return make_int2(0, q);
+    if (q < head + c.nprev) return make_int2(1, q - head);
+    if (q < c.nmain + c.nprev) return make_int2(0, q - c.nprev);
+    return make_int2(2, q - c.nmain - c.nprev);
   };
 
-  if (warp == 0) {
+  if (warp >= kFirstProducer) {
     if (lane == 0) {
-      // ---- TMA producer ----
+      // ---- TMA producers ----
+      // Producer pr issues ring items it with it % kProducers == pr. A thread
+      // that has TMA copies in flight stalls at its next mbarrier operation
+      // until they land, so one producer would keep a single stage in
+      // flight; kProducers of them keep kProducers stages in flight.
+      const int pr = warp - kFirstProducer;
       int it = 0;
       bool ok = true;
+      int t_ready = -1;  // previous-tile row block whose T this producer saw published
       auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx) {
         const int s = it % STAGES;
         if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
@@ -295,10 +355,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         sm100::mbar_arrive_expect_tx(&full_bar[s], kStage);
         sm100::tma_load_2d(sa, ma, &full_bar[s], kx, ay);
         sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
-        ++it;
       };
       auto load_main = [&](const Tile& x, int kb) {
         const int kx = kb * kElemsPerRow;
+        // The CTAs of one weight tile (all row blocks of x) ask for the same
+        // K-block at about the same time; the first of them warms L2 for
+        // K-block kb + kPrefetch so that none of them waits on DRAM.
+        if constexpr (!SWAP) {
+          if (!x.is_t && x.a0 == 0 && kb + kPrefetch < nkb)
+            sm100::tma_prefetch_l2_2d(&tmB, kx + kPrefetch * kElemsPerRow, x.b0);
+        }
         if (x.is_t) {
           if constexpr (SWAP) load(&tmL, x.a0, &tmB, 0, kx);
           else load(&tmA, x.a0, &tmL, 0, kx);
@@ -306,53 +372,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           load(&tmA, x.a0, &tmB, x.b0, kx);
         }
       };
-      for (int li = 0; li <= nmine && ok; ++li) {
-        int nmain, nadp;
-        counts(li, nmain, nadp);
+      int last_mine = -1;  // this producer's last ring item
+      for (int li = 0; li < nmine && ok; ++li) {
+        const Counts c = counts(li);
         const Tile cur = tile_at(li);
         const Tile prev = (li > 0) ? tile_at(li - 1) : cur;
-        const int items = nmain + nadp;
-        for (int q = 0; q < items && ok; ++q) {
-          const int qa = q - min(ins, nmain);
-          if (q < min(ins, nmain)) {
-            load_main(cur, q);
-          } else if (qa < nadp) {
-            if (qa == 0) {
-              // T must be stored before its TMA load: wait for the T tile(s)
-              bool ready = true;
-              if constexpr (SWAP) {
-                for (int t = 0; t < p.nT && ready; ++t)
-                  ready = wait_flag(p.t_flags + t, p.epoch);
-              } else {
-                ready = wait_flag(p.t_flags + prev.a0 / kBM, p.epoch);
-              }
-              if (!ready) {
-                set_fault(kFaultProducer, &abort_flag);
-                ok = false;
-                break;
-              }
-              fence_proxy_async_global();
-            }
-            load(&tmA2, prev.a0, &tmB2, prev.b0, qa * kElemsPerRow);
-          } else {
-            load_main(cur, q - nadp);
+        const int items = c.nmain + c.nprev + c.nself;
+        for (int q = 0; q < items && ok; ++q, ++it) {
+          if (it % kProducers != pr) continue;
+          last_mine = it;
+          const int2 ik = item_of(c, q);
+          const int kind = ik.x, kb = ik.y;
+          if (kind == 0) {
+            load_main(cur, kb);
+            continue;
           }
+          const Tile& owner = (kind == 1) ? prev : cur;
+          if (t_ready != owner.a0) {
+            // T must be stored before its TMA load: wait for the T tile(s)
+            bool ready = true;
+            if constexpr (SWAP) {
+              for (int t = 0; t < p.nT && ready; ++t) ready = wait_flag(p.t_flags + t, p.epoch);
+            } else {
+              ready = wait_flag(p.t_flags + owner.a0 / kBM, p.epoch);
+            }
+            if (!ready) {
+              set_fault(kFaultProducer, &abort_flag);
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            t_ready = owner.a0;
+          }
+          load(&tmA2, owner.a0, &tmB2, owner.b0, kb * kElemsPerRow);
         }
       }
-      for (int k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
-        if (!sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1))
+      // No copy may still be landing when the CTA exits: wait for this
+      // producer's items among the last STAGES.
+      for (int k = (it > STAGES ? it - STAGES : 0); k < it && k <= last_mine; ++k)
+        if (k % kProducers == pr && !sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1))
           set_fault(kFaultProducer, &abort_flag);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
     if (lane == 0) {
-      // ---- MMA issuer ----
+      // ---- MMA issuers ----
+      // Two threads (warps 4 and 5) issue alternate ring items: item it is
+      // issued by issuer it & 1, in ring order, handed over through `order`
+      // (a tcgen05 fence on each side of the hand-over orders the MMAs). A
+      // thread that has committed stalls at its next wait until its own
+      // MMAs finish; with two issuers the other thread's item keeps the
+      // tensor pipe busy meanwhile. Per-tile barriers (acc_full, draft_full)
+      // take one commit from each issuer, each tracking its own MMAs.
+      const int e = warp - kMmaWarp0;
       int it = 0;
       bool ok = true;
-      auto consume = [&](uint32_t d, uint32_t idesc, bool accumulate_first) {
+      auto fail = [&]() {
+        set_fault(kFaultMma, &abort_flag);
+        ok = false;
+      };
+      auto issue = [&](uint32_t d, uint32_t idesc, bool accumulate_first) {
         const int s = it % STAGES;
-        if (!sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
-          set_fault(kFaultMma, &abort_flag);
-          ok = false;
+        if (!wait_order(order, it, &abort_flag) ||
+            !sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
+          fail();
           return;
         }
         sm100::tc_fence_after();
@@ -362,50 +444,66 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
+        sm100::tc_fence_before();
+        st_release_shared(order, it + 1);
         sm100::mma_commit(&empty_bar[s]);
-        ++it;
       };
-      for (int li = 0; li <= nmine && ok; ++li) {
-        int nmain, nadp;
-        counts(li, nmain, nadp);
-        const int buf = li & 1, pbuf = (li - 1) & 1;
+      for (int li = 0; li < nmine && ok; ++li) {
+        const Counts c = counts(li);
+        const int buf = li & 1, pbuf = buf ^ 1;
         const uint32_t d = tmem + static_cast<uint32_t>(buf * kAcc);
         const uint32_t pd = tmem + static_cast<uint32_t>(pbuf * kAcc);
-        const uint32_t idesc = (nmain && tile_at(li).is_t && !SWAP) ? p.idesc_t : kIdesc;
-        const int items = nmain + nadp;
-        if (nmain && li >= 2 && !sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
-          set_fault(kFaultMma, &abort_flag);
-          break;
-        }
-        sm100::tc_fence_after();
-        for (int q = 0; q < items && ok; ++q) {
-          const int qa = q - min(ins, nmain);
-          if (q < min(ins, nmain)) {
-            consume(d, idesc, q > 0);
-            if (q == nmain - 1) sm100::mma_commit(&acc_full[buf]);
-          } else if (qa < nadp) {
-            const int mo = li - 1 - nt_mine;  // main ordinal of the previous tile
-            if (qa == 0) {
-              if (!sm100::mbar_wait(&ar_read[mo & 1], (mo >> 1) & 1)) {
-                set_fault(kFaultMma, &abort_flag);
-                ok = false;
-                break;
+        const uint32_t idesc = (tile_at(li).is_t && !SWAP) ? p.idesc_t : kIdesc;
+        const int items = c.nmain + c.nprev + c.nself;
+        const int mo = li - 1 - nt_mine;  // main ordinal of the previous tile
+        for (int q = 0; q < items && ok; ++q, ++it) {
+          const bool mine = (it & 1) == e;
+          const int2 ik = item_of(c, q);
+          const int kind = ik.x, kb = ik.y;
+          if (kind == 1) {
+            if (mine) {
+              if (kb == 0) {
+                if (!sm100::mbar_wait(&ar_read[mo & 1], (mo >> 1) & 1)) {
+                  fail();
+                  break;
+                }
+                sm100::tc_fence_after();
               }
-              sm100::tc_fence_after();
+              issue(pd, kIdesc, true);  // adds T Bm^T onto y_ar of the previous tile
             }
-            consume(pd, kIdesc, true);  // adds T Bm^T onto y_ar of the previous tile
-            if (qa == nadp - 1) sm100::mma_commit(&draft_full[mo & 1]);
+            if (ok && kb == c.nprev - 1) sm100::mma_commit(&draft_full[mo & 1]);
+          } else if (kind == 2) {
+            if (mine) {
+              if (kb == 0 && li >= 1) {
+                // the other buffer is free once tile li-1 has been drained
+                if (!sm100::mbar_wait(&acc_empty[pbuf], ((li - 1) >> 1) & 1)) {
+                  fail();
+                  break;
+                }
+                sm100::tc_fence_after();
+              }
+              issue(pd, kIdesc, kb > 0);  // T Bm^T of this tile, on its own
+            }
+            if (ok && kb == c.nself - 1) sm100::mma_commit(&acc_full[buf]);
           } else {
-            const int kb = q - nadp;
-            consume(d, idesc, kb > 0);
-            if (kb == nmain - 1) sm100::mma_commit(&acc_full[buf]);
+            if (mine) {
+              if (kb == 0 && li >= 2) {
+                if (!sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
+                  fail();
+                  break;
+                }
+                sm100::tc_fence_after();
+              }
+              issue(d, idesc, kb > 0);
+            }
+            if (ok && kb == c.nmain - 1 && c.nself == 0) sm100::mma_commit(&acc_full[buf]);
           }
         }
       }
     }
   } else {
-    // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
-    const int quarter = warp & 3;
+    // ---- epilogue: warps 0..3, TMEM lane quarter = warp ----
+    const int quarter = warp;
     const int rr = quarter * 32 + lane;
     T* ya = static_cast<T*>(p.y_ar);
     T* yd = static_cast<T*>(p.y_draft);
@@ -439,6 +537,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     };
+    // Drain y_ar = acc and y_draft = acc + adp (both BN columns wide).
+    auto drain2 = [&](uint32_t acc, uint32_t adp, int a0, int b0) {
+      const uint32_t lq = static_cast<uint32_t>(quarter * 32) << 16;
+      const int arow = a0 + rr;
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32], w[32];
+        sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
+        sm100::tmem_ld_32x32b_x32(adp + lq + c, w);
+        sm100::tmem_ld_wait();
+        float f[32];
+        const int brow = b0 + c;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          T* y = pass ? yd : ya;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            f[e] = pass ? f[e] + __uint_as_float(w[e]) : __uint_as_float(v[e]);
+          if (!y) continue;
+          if constexpr (!SWAP) {
+            if (arow < p.M && brow < p.ncols)
+              store_row32<T>(y + static_cast<size_t>(arow) * p.ncols + brow, f, p.ncols - brow);
+          } else {
+            if (arow < p.ncols) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * p.ncols + arow, f[e]);
+            }
+          }
+        }
+      }
+    };
     for (int li = 0; li < nmine; ++li) {
       const int buf = li & 1;
       const uint32_t acc = tmem + static_cast<uint32_t>(buf * kAcc);
@@ -459,11 +588,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         // One thread publishes the tile once all four epilogue warps stored
         // their rows. T tiles are this CTA's tiles 0..nt_mine-1, so li counts
-        // the completed phases of t_stored; warp 2 frees the accumulator only
+        // the completed phases of t_stored; warp 0 frees the accumulator only
         // after its wait, so the other warps cannot get two T tiles ahead.
         if (lane == 0) {
           sm100::mbar_arrive(t_stored);
-          if (warp == 2) {
+          if (warp == 0) {
             if (sm100::mbar_wait(t_stored, li & 1)) {
               fence_proxy_async_global();
               st_release_u32(p.t_flags + x.tt, p.epoch);
@@ -475,6 +604,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
         continue;
+      }
+      if (adapter && li == nmine - 1) {
+        // last tile: y_ar in this buffer, T Bm^T in the other; one pass
+        drain2(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc), x.a0, x.b0);
+        break;
       }
       drain(acc, x.a0, x.b0, ya, p.ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
@@ -498,7 +632,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp0) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, kTmemCols);
   }
