@@ -81,6 +81,7 @@ struct GemmParams {
   int nT;             // T tiles
   int r;              // adapter rank
   uint32_t idesc_t;   // instruction descriptor of the T tiles
+  int t_brows;        // rows of the B box of a T-tile item (per CTA)
   uint32_t epoch;     // value a T tile's flag takes once T is stored
   float scale;        // alpha / r
   void* y_ar;         // may be null
@@ -95,14 +96,21 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-template <int BN>
-__host__ __device__ constexpr int stages_for() {
-  return BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+// Bytes of one ring stage per CTA: a 128-row box of the A side and the B
+// rows this CTA holds (all BN, or half of them with the CTA pair).
+template <int BN, bool PAIR>
+__host__ __device__ constexpr int stage_bytes() {
+  return (kBM + (PAIR ? BN / 2 : BN)) * kRowBytes;
 }
 
-template <int BN, int STAGES>
+template <int BN, bool PAIR>
+__host__ __device__ constexpr int stages_for() {
+  return PAIR ? 6 : (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8));
+}
+
+template <int BN, bool PAIR>
 __host__ __device__ constexpr int smem_bytes() {
-  return STAGES * (kBM + BN) * kRowBytes + 1024 /*align*/ + 256 /*barriers*/;
+  return stages_for<BN, PAIR>() * stage_bytes<BN, PAIR>() + 1024 /*align*/ + 256 /*barriers*/;
 }
 
 __device__ __forceinline__ void set_fault(unsigned bit, volatile int* abort_flag) {
@@ -164,6 +172,10 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void st_release_shared(int* p, int v) {
   asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(sm100::smem_addr(p)), "r"(v)
                : "memory");
@@ -188,6 +200,86 @@ __device__ bool wait_order(const int* order, int it, volatile int* abort_flag) {
   }
 }
 
+// ---- two-SM (CTA pair) forms ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(sm100::smem_addr(p)), "r"(rank));
+  return r;
+}
+
+// Every thread of both CTAs arrives (threads need not be converged).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void arrive_at(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr)
+               : "memory");
+}
+
+// Bounded wait with cluster-scope acquire (barriers that a peer CTA or the
+// pair's tensor core arrives on).
+__device__ bool wait_cl(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = sm100::globaltimer_ns();
+  for (uint32_t k = 0;; ++k) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(sm100::smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((k & 255u) == 255u && sm100::globaltimer_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+// TMA load whose completion is counted on the mbarrier of the pair's leader.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(sm100::smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+template <bool kTf32>
+__device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         bool accumulate) {
+  if constexpr (kTf32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+        : "memory");
+  }
+}
+
+// Arrive on `bar` (same offset) in both CTAs of the pair once the issuing
+// thread's MMAs have completed.
+__device__ __forceinline__ void commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(sm100::smem_addr(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
 // Bounded wait until *flag == epoch.
 __device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
   if (ld_acquire_u32(flag) == epoch) return true;
@@ -205,17 +297,22 @@ __device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
 // LoRA down weight A for the T tiles (non-swapped: the B side, box BN rows;
 // swapped: the A side, box 128 rows).
 // ---------------------------------------------------------------------------
-template <typename T, int BN, bool SWAP>
+template <typename T, int BN, bool SWAP, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                const __grid_constant__ CUtensorMap tmL, const GemmParams p) {
-  constexpr int STAGES = stages_for<BN>();
+                const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmYa,
+                const __grid_constant__ CUtensorMap tmYd, const GemmParams p) {
+  static_assert(!(PAIR && SWAP), "the CTA pair serves the unswapped layout");
+  constexpr int STAGES = stages_for<BN, PAIR>();
   constexpr int kAbytes = kBM * kRowBytes;
-  constexpr int kStage = (kBM + BN) * kRowBytes;
+  constexpr int kBrows = PAIR ? BN / 2 : BN;   // rows of W (B side) per CTA and K-block
+  constexpr int kStage = stage_bytes<BN, PAIR>();
+  constexpr int kRows = PAIR ? 2 * kBM : kBM;  // output rows of a tile (both CTAs)
   constexpr bool kTf32 = sizeof(T) == 4;
   constexpr int kElemsPerRow = kRowBytes / static_cast<int>(sizeof(T));
-  constexpr uint32_t kIdesc = sm100::instr_desc(kTf32, kBM, BN);
+  constexpr uint32_t kIdesc = sm100::instr_desc(kTf32, kRows, BN);
+  constexpr int kEpiArrivals = PAIR ? 8 : 4;  // epilogue warps of the pair / the CTA
   constexpr int kAcc = pow2_at_least(BN);  // columns of one accumulator buffer
   constexpr uint32_t kTmemCols = 2 * kAcc;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && kTmemCols <= 512, "BN");
@@ -235,10 +332,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_a = (p.rowsA + kBM - 1) / kBM;
+  // With the CTA pair, rank 0 (the leader) issues the MMAs for both SMs; each
+  // CTA loads and drains its own 128 rows of the 256-row tile.
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int my_rows = static_cast<int>(rank) * kBM;     // this CTA's row offset in a tile
+  const int my_brows = static_cast<int>(rank) * kBrows;  // and in the B operand
+  const int tiles_a = (p.rowsA + kRows - 1) / kRows;
   const int tiles_b = (p.rowsB + BN - 1) / BN;
   const int ntiles = p.nT + tiles_a * tiles_b;
-  const int G = static_cast<int>(gridDim.x), C = static_cast<int>(blockIdx.x);
+  const int G = static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
+  const int C = static_cast<int>(blockIdx.x) / (PAIR ? 2 : 1);
   const int nmine = (ntiles > C) ? (ntiles - 1 - C) / G + 1 : 0;
   // This CTA's T tiles are its first nt_mine tiles (their global indices are
   // the lowest); main tile li has ordinal li - nt_mine among its main tiles,
@@ -256,11 +360,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       sm100::mbar_init(&acc_full[b], 2);  // one commit per MMA issuer
-      sm100::mbar_init(&ar_read[b], 4);
+      sm100::mbar_init(&ar_read[b], kEpiArrivals);
       sm100::mbar_init(&draft_full[b], 2);
-      sm100::mbar_init(&acc_empty[b], 4);
+      sm100::mbar_init(&acc_empty[b], kEpiArrivals);
     }
-    sm100::mbar_init(t_stored, 4);
+    sm100::mbar_init(t_stored, kEpiArrivals);
     *order = 0;
     abort_flag = 0;
     sm100::fence_mbar_init();
@@ -274,9 +378,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::tma_prefetch_desc(&tmL);
     }
   }
-  if (warp == kMmaWarp0) sm100::tmem_alloc(tmem_holder, kTmemCols);
+  if (warp == kMmaWarp0) {
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       sm100::smem_addr(tmem_holder)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      sm100::tmem_alloc(tmem_holder, kTmemCols);
+    }
+  }
   sm100::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // barriers of both CTAs initialised
+  else __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
@@ -294,11 +409,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     x.is_t = t < p.nT;
     x.tt = t;
     if (x.is_t) {
-      x.a0 = t * kBM;
+      x.a0 = t * kRows;
       x.b0 = 0;
     } else {
       const int u = t - p.nT;
-      x.a0 = (u % tiles_a) * kBM;
+      x.a0 = (u % tiles_a) * kRows;
       x.b0 = (u / tiles_a) * BN;
     }
     return x;
@@ -340,7 +455,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       int t_ready = -1;  // previous-tile row block whose T this producer saw published
-      auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx) {
+      // b_rows: rows of the B box (both CTAs of a pair load the same shape;
+      // the leader expects the bytes of both).
+      auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx,
+                      int b_rows) {
         const int s = it % STAGES;
         if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
           set_fault(kFaultProducer, &abort_flag);
@@ -352,9 +470,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           return;
         }
         uint8_t* sa = smem + s * kStage;
-        sm100::mbar_arrive_expect_tx(&full_bar[s], kStage);
-        sm100::tma_load_2d(sa, ma, &full_bar[s], kx, ay);
-        sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
+        const uint32_t bytes = static_cast<uint32_t>(kAbytes + b_rows * kRowBytes);
+        if constexpr (PAIR) {
+          if (leader) sm100::mbar_arrive_expect_tx(&full_bar[s], 2 * bytes);
+          const uint32_t bar = cluster_addr(&full_bar[s], 0);
+          tma_load_2d_pair(sa, ma, bar, kx, ay);
+          tma_load_2d_pair(sa + kAbytes, mb, bar, kx, by);
+        } else {
+          sm100::mbar_arrive_expect_tx(&full_bar[s], bytes);
+          sm100::tma_load_2d(sa, ma, &full_bar[s], kx, ay);
+          sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
+        }
       };
       auto load_main = [&](const Tile& x, int kb) {
         const int kx = kb * kElemsPerRow;
@@ -363,13 +489,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // K-block kb + kPrefetch so that none of them waits on DRAM.
         if constexpr (!SWAP) {
           if (!x.is_t && x.a0 == 0 && kb + kPrefetch < nkb)
-            sm100::tma_prefetch_l2_2d(&tmB, kx + kPrefetch * kElemsPerRow, x.b0);
+            sm100::tma_prefetch_l2_2d(&tmB, kx + kPrefetch * kElemsPerRow, x.b0 + my_brows);
         }
         if (x.is_t) {
-          if constexpr (SWAP) load(&tmL, x.a0, &tmB, 0, kx);
-          else load(&tmA, x.a0, &tmL, 0, kx);
+          if constexpr (SWAP) load(&tmL, x.a0, &tmB, 0, kx, kBrows);
+          else load(&tmA, x.a0 + my_rows, &tmL, static_cast<int>(rank) * p.t_brows, kx, p.t_brows);
         } else {
-          load(&tmA, x.a0, &tmB, x.b0, kx);
+          load(&tmA, x.a0 + my_rows, &tmB, x.b0 + my_brows, kx, kBrows);
         }
       };
       int last_mine = -1;  // this producer's last ring item
@@ -387,14 +513,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             load_main(cur, kb);
             continue;
           }
-          const Tile& owner = (kind == 1) ? prev : cur;
+          const Tile owner = (kind == 1) ? prev : cur;
           if (t_ready != owner.a0) {
             // T must be stored before its TMA load: wait for the T tile(s)
             bool ready = true;
             if constexpr (SWAP) {
               for (int t = 0; t < p.nT && ready; ++t) ready = wait_flag(p.t_flags + t, p.epoch);
             } else {
-              ready = wait_flag(p.t_flags + owner.a0 / kBM, p.epoch);
+              ready = wait_flag(p.t_flags + owner.a0 / kRows, p.epoch);
             }
             if (!ready) {
               set_fault(kFaultProducer, &abort_flag);
@@ -404,17 +530,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_global();
             t_ready = owner.a0;
           }
-          load(&tmA2, owner.a0, &tmB2, owner.b0, kb * kElemsPerRow);
+          load(&tmA2, owner.a0 + my_rows, &tmB2, owner.b0 + my_brows, kb * kElemsPerRow, kBrows);
         }
       }
       // No copy may still be landing when the CTA exits: wait for this
-      // producer's items among the last STAGES.
-      for (int k = (it > STAGES ? it - STAGES : 0); k < it && k <= last_mine; ++k)
+      // producer's items among the last STAGES (the leader's full barriers
+      // count the copies of both CTAs; the pair then meets at a cluster barrier).
+      for (int k = (it > STAGES ? it - STAGES : 0); leader && k < it && k <= last_mine; ++k)
         if (k % kProducers == pr && !sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1))
           set_fault(kFaultProducer, &abort_flag);
     }
   } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ---- MMA issuers ----
       // Two threads (warps 4 and 5) issue alternate ring items: item it is
       // issued by issuer it & 1, in ring order, handed over through `order`
@@ -430,6 +557,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         set_fault(kFaultMma, &abort_flag);
         ok = false;
       };
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (PAIR) commit_pair(bar);
+        else sm100::mma_commit(bar);
+      };
       auto issue = [&](uint32_t d, uint32_t idesc, bool accumulate_first) {
         const int s = it % STAGES;
         if (!wait_order(order, it, &abort_flag) ||
@@ -442,11 +573,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint64_t da = sm100::smem_desc_k_sw128(sa);
         const uint64_t db = sm100::smem_desc_k_sw128(sa + kAbytes);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
+        for (int k = 0; k < 4; ++k) {
+          if constexpr (PAIR)
+            mma_pair<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
+          else
+            sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
+        }
         sm100::tc_fence_before();
         st_release_shared(order, it + 1);
-        sm100::mma_commit(&empty_bar[s]);
+        commit(&empty_bar[s]);
       };
       for (int li = 0; li < nmine && ok; ++li) {
         const Counts c = counts(li);
@@ -463,7 +598,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (kind == 1) {
             if (mine) {
               if (kb == 0) {
-                if (!sm100::mbar_wait(&ar_read[mo & 1], (mo >> 1) & 1)) {
+                if (!wait_cl(&ar_read[mo & 1], (mo >> 1) & 1)) {
                   fail();
                   break;
                 }
@@ -471,12 +606,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
               issue(pd, kIdesc, true);  // adds T Bm^T onto y_ar of the previous tile
             }
-            if (ok && kb == c.nprev - 1) sm100::mma_commit(&draft_full[mo & 1]);
+            if (ok && kb == c.nprev - 1) commit(&draft_full[mo & 1]);
           } else if (kind == 2) {
             if (mine) {
               if (kb == 0 && li >= 1) {
                 // the other buffer is free once tile li-1 has been drained
-                if (!sm100::mbar_wait(&acc_empty[pbuf], ((li - 1) >> 1) & 1)) {
+                if (!wait_cl(&acc_empty[pbuf], ((li - 1) >> 1) & 1)) {
                   fail();
                   break;
                 }
@@ -484,11 +619,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
               issue(pd, kIdesc, kb > 0);  // T Bm^T of this tile, on its own
             }
-            if (ok && kb == c.nself - 1) sm100::mma_commit(&acc_full[buf]);
+            if (ok && kb == c.nself - 1) commit(&acc_full[buf]);
           } else {
             if (mine) {
               if (kb == 0 && li >= 2) {
-                if (!sm100::mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
+                if (!wait_cl(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
                   fail();
                   break;
                 }
@@ -496,7 +631,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
               issue(d, idesc, kb > 0);
             }
-            if (ok && kb == c.nmain - 1 && c.nself == 0) sm100::mma_commit(&acc_full[buf]);
+            if (ok && kb == c.nmain - 1 && c.nself == 0) commit(&acc_full[buf]);
           }
         }
       }
@@ -504,6 +639,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---- epilogue: warps 0..3, TMEM lane quarter = warp ----
     const int quarter = warp;
+    // Epilogue barriers live in the leader; a pair's second CTA arrives remotely.
+    auto arrive_leader = [&](uint64_t* bar) {
+      if constexpr (PAIR) arrive_at(cluster_addr(bar, 0));
+      else sm100::mbar_arrive(bar);
+    };
     const int rr = quarter * 32 + lane;
     T* ya = static_cast<T*>(p.y_ar);
     T* yd = static_cast<T*>(p.y_draft);
@@ -538,6 +678,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     };
     // Drain y_ar = acc and y_draft = acc + adp (both BN columns wide).
+    // Last tile with bf16 outputs and the pair layout: the ring is idle by
+    // now, so each warp stages its 32 rows of y_ar and y_draft in shared
+    // memory (128-byte swizzled boxes of 32 rows x 64 columns, 16 KB per
+    // output) and writes them with TMA stores: full 128-byte rows instead of
+    // 64-byte pieces 8 KB apart.
+    auto drain2_tma = [&](uint32_t acc, uint32_t adp, int a0, int b0) {
+      const uint32_t lq = static_cast<uint32_t>(quarter * 32) << 16;
+      uint8_t* stage_ar = smem + quarter * 32768;
+      uint8_t* stage_dr = stage_ar + 16384;
+      const uint32_t sw = static_cast<uint32_t>(lane & 7);
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32], w[32];
+        sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
+        sm100::tmem_ld_32x32b_x32(adp + lq + c, w);
+        sm100::tmem_ld_wait();
+        // columns c..c+31 = 4 chunks of 16 bytes in box c/64, chunks (c%64)/8..+3
+        const int box = c >> 6;
+        const uint32_t chunk0 = static_cast<uint32_t>((c & 63) >> 3);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float* fv = reinterpret_cast<const float*>(v) + 8 * g;
+          uint4 a, d;
+          a.x = pack_bf16x2(fv[0], fv[1]);
+          a.y = pack_bf16x2(fv[2], fv[3]);
+          a.z = pack_bf16x2(fv[4], fv[5]);
+          a.w = pack_bf16x2(fv[6], fv[7]);
+          float t[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = fv[e] + __uint_as_float(w[8 * g + e]);
+          d.x = pack_bf16x2(t[0], t[1]);
+          d.y = pack_bf16x2(t[2], t[3]);
+          d.z = pack_bf16x2(t[4], t[5]);
+          d.w = pack_bf16x2(t[6], t[7]);
+          const uint32_t off = static_cast<uint32_t>(box * 4096 + lane * 128) +
+                               (((chunk0 + g) ^ sw) << 4);
+          *reinterpret_cast<uint4*>(stage_ar + off) = a;
+          *reinterpret_cast<uint4*>(stage_dr + off) = d;
+        }
+      }
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        const int row = a0;  // first of this warp's 32 rows
+        for (int box = 0; box < BN / 64; ++box) {
+          if (ya) sm100::tma_store_2d(&tmYa, stage_ar + box * 4096, b0 + 64 * box, row);
+          sm100::tma_store_2d(&tmYd, stage_dr + box * 4096, b0 + 64 * box, row);
+        }
+        sm100::bulk_commit_group();
+        sm100::bulk_wait_group_0();
+      }
+      __syncwarp();
+    };
     auto drain2 = [&](uint32_t acc, uint32_t adp, int a0, int b0) {
       const uint32_t lq = static_cast<uint32_t>(quarter * 32) << 16;
       const int arow = a0 + rr;
@@ -572,7 +764,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int buf = li & 1;
       const uint32_t acc = tmem + static_cast<uint32_t>(buf * kAcc);
       const Tile x = tile_at(li);
-      const bool got = __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&acc_full[buf], (li >> 1) & 1));
+      const bool got = __all_sync(0xFFFFFFFFu, wait_cl(&acc_full[buf], (li >> 1) & 1));
       if (!got || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
@@ -581,7 +773,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (x.is_t) {
         // T = scale * x A^T: non-swapped, rows of x by r columns; swapped, r
         // rows (rows of A) by the M columns of x.
-        if constexpr (!SWAP) drain(acc, x.a0, 0, tb, p.r, p.M, p.r, p.scale);
+        if constexpr (!SWAP) drain(acc, x.a0 + my_rows, 0, tb, p.r, p.M, p.r, p.scale);
         else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.scale);
         sm100::tc_fence_before();
         __threadfence();
@@ -591,50 +783,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // the completed phases of t_stored; warp 0 frees the accumulator only
         // after its wait, so the other warps cannot get two T tiles ahead.
         if (lane == 0) {
-          sm100::mbar_arrive(t_stored);
-          if (warp == 0) {
-            if (sm100::mbar_wait(t_stored, li & 1)) {
+          arrive_leader(t_stored);
+          if (warp == 0 && leader) {
+            if (wait_cl(t_stored, li & 1)) {
               fence_proxy_async_global();
               st_release_u32(p.t_flags + x.tt, p.epoch);
             } else {
               set_fault(kFaultEpilogue, &abort_flag);
             }
           }
-          sm100::mbar_arrive(&acc_empty[buf]);
+          arrive_leader(&acc_empty[buf]);
         }
         __syncwarp();
         continue;
       }
       if (adapter && li == nmine - 1) {
         // last tile: y_ar in this buffer, T Bm^T in the other; one pass
-        drain2(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc), x.a0, x.b0);
+        if constexpr (PAIR && sizeof(T) == 2)
+          drain2_tma(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc),
+                     x.a0 + my_rows + quarter * 32, x.b0);
+        else
+          drain2(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc), x.a0 + my_rows, x.b0);
         break;
       }
-      drain(acc, x.a0, x.b0, ya, p.ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, ya, p.ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
       const int mo = li - nt_mine;
-      if (lane == 0) sm100::mbar_arrive(adapter ? &ar_read[mo & 1] : &acc_empty[buf]);
+      if (lane == 0) arrive_leader(adapter ? &ar_read[mo & 1] : &acc_empty[buf]);
       if (!adapter) continue;
-      const bool got2 =
-          __all_sync(0xFFFFFFFFu, sm100::mbar_wait(&draft_full[mo & 1], (mo >> 1) & 1));
+      const bool got2 = __all_sync(0xFFFFFFFFu, wait_cl(&draft_full[mo & 1], (mo >> 1) & 1));
       if (!got2 || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
       }
       sm100::tc_fence_after();
-      drain(acc, x.a0, x.b0, yd, p.ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, yd, p.ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) arrive_leader(&acc_empty[buf]);
     }
   }
 
   sm100::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // neither CTA leaves while its peer may touch it
+  else __syncthreads();
   if (warp == kMmaWarp0) {
     sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, kTmemCols);
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    else
+      sm100::tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -674,6 +875,20 @@ bool make_map(CUtensorMap* map, const void* ptr, int dtype, int k_elems, int row
   return r == CUDA_SUCCESS;
 }
 
+// Row-major bf16 [rows][cols] output: boxes of 64 columns (128 bytes) x 32
+// rows, 128-byte swizzle; the TMA store skips whatever lies out of bounds.
+bool make_store_map(CUtensorMap* map, void* ptr, int cols, int rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int cached[64];
   int dev = 0;
@@ -701,12 +916,40 @@ uint32_t next_epoch() {
   return e;
 }
 
-template <typename T, int BN, bool SWAP>
+// Clusters of two that can be resident at once (cached per device).
+template <typename K>
+int max_pairs(K kern, int bytes) {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
+  if (cached[dev]) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sm_count() & ~1));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(bytes);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  cached[dev] = n;
+  return n;
+}
+
+template <typename T, int BN, bool SWAP, bool PAIR>
 int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const CUtensorMap& l, const GemmParams& p,
-                cudaStream_t st) {
-  constexpr int bytes = smem_bytes<BN, stages_for<BN>()>();
-  auto kern = dual_kernel<T, BN, SWAP>;
+                const CUtensorMap& b2, const CUtensorMap& l, const CUtensorMap& ya,
+                const CUtensorMap& yd, const GemmParams& p, cudaStream_t st) {
+  constexpr int bytes = smem_bytes<BN, PAIR>();
+  constexpr int kRows = PAIR ? 2 * kBM : kBM;
+  auto kern = dual_kernel<T, BN, SWAP, PAIR>;
   static std::atomic<uint64_t> attr_done{0};  // devices with the shared-memory opt-in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return UNO_ERR_CUDA;
@@ -717,11 +960,30 @@ int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
       return UNO_ERR_CUDA;
     attr_done.fetch_or(bit, std::memory_order_relaxed);
   }
-  const long long tiles = p.nT + static_cast<long long>((p.rowsA + kBM - 1) / kBM) *
+  const long long tiles = p.nT + static_cast<long long>((p.rowsA + kRows - 1) / kRows) *
                                      ((p.rowsB + BN - 1) / BN);
-  long long grid = sm_count();
-  if (grid > tiles) grid = tiles;
-  kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, l, p);
+  if constexpr (PAIR) {
+    long long pairs = max_pairs(kern, bytes);
+    if (pairs > tiles) pairs = tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a, b, a2, b2, l, ya, yd, p) != cudaSuccess)
+      return UNO_ERR_CUDA;
+  } else {
+    long long grid = sm_count();
+    if (grid > tiles) grid = tiles;
+    kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, l, ya, yd, p);
+  }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
@@ -729,11 +991,12 @@ template <typename T, bool SWAP>
 int launch_dual_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                    const CUtensorMap& b2, const CUtensorMap& l, const GemmParams& p,
                    cudaStream_t st) {
+  // the swapped layout stores from registers; its output maps are unused
   switch (bn) {
-    case 32: return launch_dual<T, 32, SWAP>(a, b, a2, b2, l, p, st);
-    case 64: return launch_dual<T, 64, SWAP>(a, b, a2, b2, l, p, st);
-    case 128: return launch_dual<T, 128, SWAP>(a, b, a2, b2, l, p, st);
-    default: return launch_dual<T, 256, SWAP>(a, b, a2, b2, l, p, st);
+    case 32: return launch_dual<T, 32, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
+    case 64: return launch_dual<T, 64, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
+    case 128: return launch_dual<T, 128, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
+    default: return launch_dual<T, 256, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
   }
 }
 
@@ -761,7 +1024,8 @@ Plan make_plan(int M, int d_in, int r, int dtype) {
   pl.swap = M <= 256;
   pl.kb_main = (d_in * pl.esize + kRowBytes - 1) / kRowBytes;
   pl.kb_adapt = (r * pl.esize + kRowBytes - 1) / kRowBytes;
-  pl.nT = pl.swap ? (r + kBM - 1) / kBM : (M + kBM - 1) / kBM;
+  // with M > 256 a CTA pair computes 256-row tiles, so one T tile per 256 rows
+  pl.nT = pl.swap ? (r + kBM - 1) / kBM : (M + 2 * kBM - 1) / (2 * kBM);
   pl.t_bytes = align256(static_cast<size_t>(M) * r * pl.esize);
   pl.flag_bytes = align256(static_cast<size_t>(pl.nT) * sizeof(uint32_t));
   return pl;
@@ -804,6 +1068,7 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
     gp.rowsA = d_out;
     gp.rowsB = M;
     gp.idesc_t = sm100::instr_desc(tf32, kBM, bn);
+    gp.t_brows = bn;
     bool ok = make_map(&mA, W, dtype, d_in, d_out, kBM) && make_map(&mB, x, dtype, d_in, M, bn);
     if (adapter)
       ok = ok && make_map(&mA2, Bm, dtype, r, d_out, kBM) &&
@@ -812,16 +1077,26 @@ int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, fl
     if (!adapter) mA2 = mB2 = mL = mA;
     return launch_dual_bn<T, true>(bn, mA, mB, mA2, mB2, mL, gp, st);
   }
+  // Unswapped: a CTA pair per 256 x 256 tile (each CTA: 128 rows of x, 128
+  // rows of W); the T tiles' N is r rounded up to 16, half of it per CTA.
+  const int n_t = (r + 15) / 16 * 16;
   gp.rowsA = M;
   gp.rowsB = d_out;
-  gp.idesc_t = sm100::instr_desc(tf32, kBM, (r + 15) / 16 * 16);
-  bool ok = make_map(&mA, x, dtype, d_in, M, kBM) && make_map(&mB, W, dtype, d_in, d_out, 256);
+  gp.idesc_t = sm100::instr_desc(tf32, 2 * kBM, n_t);
+  gp.t_brows = n_t / 2;
+  bool ok = make_map(&mA, x, dtype, d_in, M, kBM) && make_map(&mB, W, dtype, d_in, d_out, kBM);
   if (adapter)
     ok = ok && make_map(&mA2, Tbuf, dtype, r, M, kBM) &&
-         make_map(&mB2, Bm, dtype, r, d_out, 256) && make_map(&mL, A, dtype, d_in, r, 256);
+         make_map(&mB2, Bm, dtype, r, d_out, kBM) && make_map(&mL, A, dtype, d_in, r, n_t / 2);
+  // output maps for the TMA-store epilogue (bf16): boxes of 32 rows x 64 columns
+  CUtensorMap mYa = mA, mYd = mA;
+  if (adapter && dtype == UNO_BF16) {
+    ok = ok && make_store_map(&mYd, y_draft, d_out, M);
+    if (y_ar) ok = ok && make_store_map(&mYa, y_ar, d_out, M);
+  }
   if (!ok) return UNO_ERR_CUDA;
   if (!adapter) mA2 = mB2 = mL = mA;
-  return launch_dual<T, 256, false>(mA, mB, mA2, mB2, mL, gp, st);
+  return launch_dual<T, 256, false, true>(mA, mB, mA2, mB2, mL, mYa, mYd, gp, st);
 }
 
 }  // namespace
