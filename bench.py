@@ -183,8 +183,19 @@ def _dual_flops(M, d_in, d_out, r):
     return 2.0 * M * d_in * d_out + 2.0 * M * r * (d_in + d_out)
 
 
+def layer_flops(M, layer):
+    """Algorithmic FLOPs of one dual-path launch (all its projections)."""
+    _, x, ds, *_ = layer
+    return sum(_dual_flops(M, x.shape[1], d.W.shape[0], RANK) for d in ds)
+
+
+# Projections that read the same activations run as one grouped launch.
+PROJECTION_GROUPS = (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gate_up", ("gate", "up")),
+                     ("down", ("down",)))
+
+
 class BatchedDecode:
-    """64 sequences x 16 drafts: 7 dual-path projections + verify."""
+    """64 sequences x 16 drafts: 7 dual-path projections (4 launches) + verify."""
 
     name = "batched_decode_b64_k16"
 
@@ -195,16 +206,22 @@ class BatchedDecode:
         self.api = api
         self.B, self.K, self.V = B64, K16, QWEN3_8B_VOCAB
         self.M = self.B * self.K
-        self.layers = []
+        projs = {}
         for i, (name, d_in, d_out) in enumerate(QWEN3_8B_PROJECTIONS):
-            d = dualpath_inputs(M=self.M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA,
-                                seed=seed * 100 + i, device=dev)
-            y_ar = torch.empty((self.M, d_out), dtype=torch.bfloat16, device=dev)
-            y_dr = torch.empty_like(y_ar)
-            ws = torch.empty(api.dualpath_workspace_bytes(self.M, d_in, d_out, RANK,
-                                                          torch.bfloat16),
-                             dtype=torch.uint8, device=dev)
-            self.layers.append((name, d, y_ar, y_dr, ws))
+            projs[name] = dualpath_inputs(M=self.M, d_in=d_in, d_out=d_out, r=RANK, alpha=ALPHA,
+                                          seed=seed * 100 + i, device=dev)
+        # layers: one grouped launch each, (name, x, [inputs], [y_ar], [y_draft], workspace)
+        self.layers = []
+        for lname, members in PROJECTION_GROUPS:
+            ds = [projs[m] for m in members]
+            x = ds[0].x  # the members of a group read the same activations
+            y_ars = [torch.empty((self.M, d.W.shape[0]), dtype=torch.bfloat16, device=dev)
+                     for d in ds]
+            y_drs = [torch.empty_like(y) for y in y_ars]
+            need = sum(api.dualpath_workspace_bytes(self.M, d.x.shape[1], d.W.shape[0], RANK,
+                                                    torch.bfloat16) for d in ds)
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            self.layers.append((lname, x, ds, y_ars, y_drs, ws))
         self.v = verify_inputs(self.B, self.K, self.V, dtype="bf16", dist="normal", p_std=2.0,
                                sigma=1.0, seed=seed, device=dev)
         self.vws = torch.zeros(api.verify_workspace_bytes(self.B, self.K, self.V,
@@ -213,22 +230,23 @@ class BatchedDecode:
         self.out = api.VerifyResult(
             torch.empty((self.B, self.K + 1), dtype=torch.int32, device=dev),
             torch.empty((self.B,), dtype=torch.int32, device=dev), None, None, None)
-        self.gemm_flops = sum(_dual_flops(self.M, d.x.shape[1], d.W.shape[0], RANK)
-                              for _, d, *_ in self.layers)
+        self.gemm_flops = sum(layer_flops(self.M, layer) for layer in self.layers)
         self.verify_bytes = (self.B * (2 * self.K + 1) * self.V * 2 + self.B * self.K * 4
                              + self.B * (self.K + 2) * 4)
         self.launches_per_step = len(self.layers) + 3  # one dual-path launch each, verify: 3
         # bytes a step reads at least once (all distinct, so L2 cannot carry them)
-        self.step_bytes = sum(d.x.numel() * 2 + d.W.numel() * 2 + d.A.numel() * 2
-                              + d.Bm.numel() * 2 for _, d, *_ in self.layers) + self.verify_bytes
+        self.step_bytes = sum(x.numel() * 2 + sum(d.W.numel() * 2 + d.A.numel() * 2
+                                                  + d.Bm.numel() * 2 for d in ds)
+                              for _, x, ds, *_ in self.layers) + self.verify_bytes
 
     def step(self, seed_step, ev=None):
         api = self.api
-        for i, (_, d, y_ar, y_dr, ws) in enumerate(self.layers):
+        for i, (_, x, ds, y_ars, y_drs, ws) in enumerate(self.layers):
             if ev is not None:
                 ev[0][i].record()
-            api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale, y_ar=y_ar, y_draft=y_dr,
-                                workspace=ws)
+            api.dualpath_linear_grouped(x, [d.W for d in ds], [d.A for d in ds],
+                                        [d.Bm for d in ds], [d.scale for d in ds],
+                                        y_ars=y_ars, y_drafts=y_drs, workspace=ws)
             if ev is not None:
                 ev[1][i].record()
         if ev is not None:
@@ -251,13 +269,13 @@ class BatchedDecode:
     # host-resident inputs for the end-to-end measurement
     def host_inputs(self):
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-        xs = [pin(d.x) for _, d, *_ in self.layers]
+        xs = [pin(x) for _, x, *_ in self.layers]
         return xs, pin(self.v.p_logits), pin(self.v.q_logits), pin(self.v.draft_tokens)
 
     def e2e_step(self, host, step):
         xs, hp, hq, hx = host
-        for (_, d, *_), hxv in zip(self.layers, xs):
-            d.x.copy_(hxv, non_blocking=True)
+        for (_, x, *_), hxv in zip(self.layers, xs):
+            x.copy_(hxv, non_blocking=True)
         self.v.p_logits.copy_(hp, non_blocking=True)
         self.v.q_logits.copy_(hq, non_blocking=True)
         self.v.draft_tokens.copy_(hx, non_blocking=True)
@@ -279,8 +297,9 @@ class BatchedDecode:
 
     def config(self):
         return {"workload": self.name, "B": self.B, "K": self.K, "V": self.V,
-                "rows_M": self.M, "projections": [f"{n}:{d.x.shape[1]}->{d.W.shape[0]}"
-                                                  for n, d, *_ in self.layers],
+                "rows_M": self.M,
+                "launches": [f"{n}:{x.shape[1]}->" + "+".join(str(d.W.shape[0]) for d in ds)
+                             for n, x, ds, *_ in self.layers],
                 "lora_rank": RANK, "lora_alpha": ALPHA, "logits": "bf16",
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e9:.2f} GB distinct per step",
                 "global_batch": self.B, "parallelism": "replicas (one batch per GPU)"}
@@ -305,7 +324,7 @@ class SingleSequence(BatchedDecode):
         ws = torch.empty(api.dualpath_workspace_bytes(self.M, QWEN3_8B_HIDDEN, self.V, RANK,
                                                       torch.bfloat16), dtype=torch.uint8,
                          device=dev)
-        self.layers = [("lm_head", d, y_ar, y_dr, ws)]
+        self.layers = [("lm_head", d.x, [d], [y_ar], [y_dr], ws)]
         g = torch.Generator(device=dev).manual_seed(seed)
         self.drafts = torch.randint(0, self.V, (1, self.K), generator=g, device=dev,
                                     dtype=torch.int32)
@@ -321,7 +340,7 @@ class SingleSequence(BatchedDecode):
 
     def step(self, seed_step, ev=None):
         api = self.api
-        _, d, y_ar, y_dr, ws = self.layers[0]
+        _, _, (d,), (y_ar,), (y_dr,), ws = self.layers[0]
         if ev is not None:
             ev[0][0].record()
         api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale, y_ar=y_ar, y_draft=y_dr, workspace=ws)
@@ -336,12 +355,12 @@ class SingleSequence(BatchedDecode):
             ev[3].record()
 
     def host_inputs(self):
-        _, d, *_ = self.layers[0]
-        return [d.x.cpu().pin_memory()], self.drafts.cpu().pin_memory()
+        _, x, *_ = self.layers[0]
+        return [x.cpu().pin_memory()], self.drafts.cpu().pin_memory()
 
     def e2e_step(self, host, step):
         xs, hx = host
-        self.layers[0][1].x.copy_(xs[0], non_blocking=True)
+        self.layers[0][1].copy_(xs[0], non_blocking=True)
         self.drafts.copy_(hx, non_blocking=True)
         self.step(step)
         self.h_tok.copy_(self.out.out_tokens, non_blocking=True)
@@ -356,7 +375,7 @@ class SingleSequence(BatchedDecode):
 
     def config(self):
         c = super().config()
-        c.update({"projections": [f"lm_head:{QWEN3_8B_HIDDEN}->{self.V}"], "rows_M": self.M,
+        c.update({"launches": [f"lm_head:{QWEN3_8B_HIDDEN}->{self.V}"], "rows_M": self.M,
                   "l2": "W of the LM head (1.24 GB) is larger than L2"})
         return c
 
@@ -522,9 +541,10 @@ def run_ours(args):
     ver_avg = sum(ver_ms) / len(ver_ms)
     gemm_tflops = wl.gemm_flops / (gemm_avg / 1e3) / 1e12
     per_proj = {}
-    for j, (name, d, *_) in enumerate(wl.layers):
+    for j, layer in enumerate(wl.layers):
+        name = layer[0]
         us = 1e3 * sum(e[0][j].elapsed_time(e[1][j]) for e in events) / len(events)
-        fl = _dual_flops(d.x.shape[0], d.x.shape[1], d.W.shape[0], RANK)
+        fl = layer_flops(wl.M, layer)
         per_proj[name] = {"us": round(us, 2), "tflops": round(fl / (us / 1e6) / 1e12, 1)}
     ver_gbs = wl.verify_bytes / (ver_avg / 1e3) / 1e9
     dominant_gemm = gemm_avg >= ver_avg
@@ -567,7 +587,7 @@ def run_ours(args):
             "dtype": "bf16", "data": "synthetic (seeded random weights, activations, logits)",
             "config": wl.config(),
             "emitted_tokens_per_s": world * emitted / (ms_step / 1e3),
-            "gemm_tflops": gemm_tflops, "verify_gbs": ver_gbs, "gemm_per_projection": per_proj,
+            "gemm_tflops": gemm_tflops, "verify_gbs": ver_gbs, "gemm_per_launch": per_proj,
             "roofline": roof_gemm if dominant_gemm else roof_ver,
             "roofline_verify" if dominant_gemm else "roofline_gemm":
                 roof_ver if dominant_gemm else roof_gemm,

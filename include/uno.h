@@ -171,6 +171,33 @@ int uno_dualpath_linear(const void* x, const void* W, const void* A, const void*
                         int r, int dtype, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/*
+ * Grouped dual-pathway linear: n (1..4) projections of the same activations x
+ * in one launch, e.g. the q, k and v projections of a layer, or gate and up.
+ * The summary page's "Methodology / Architecture" adds the LoRA to every
+ * attention and MLP projection; projections that read the same x share one
+ * launch, so small ones (k, v) fill the GPU together with a large one.
+ *
+ * Projection g has its own W[g] [d_out[g], d_in], A[g] [r, d_in],
+ * Bm[g] [d_out[g], r], scale[g], y_ar[g] and y_draft[g] [M, d_out[g]]; M,
+ * d_in, r and dtype are shared, with the limits of uno_dualpath_linear.
+ * Either every y_draft[g] is NULL (no adapter anywhere) or none is; y_ar[g]
+ * may be NULL per projection. The results equal n separate
+ * uno_dualpath_linear calls bit for bit.
+ * workspace  at least uno_dualpath_grouped_workspace_bytes(...) bytes, 16-byte
+ *            aligned, contents irrelevant on entry (n single-call workspaces
+ *            back to back).
+ * The pointer arrays are host arrays, read during the call only.
+ * Returns UNO_OK or a negative uno_status (UNO_ERR_SIZE for n outside 1..4).
+ */
+size_t uno_dualpath_grouped_workspace_bytes(int n, int M, int d_in, const int* d_out, int r,
+                                            int dtype);
+int uno_dualpath_linear_grouped(int n, const void* x, const void* const* W,
+                                const void* const* A, const void* const* Bm,
+                                const float* scale, void* const* y_ar, void* const* y_draft,
+                                int M, int d_in, const int* d_out, int r, int dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Device fault flags
  *

@@ -207,6 +207,65 @@ def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch
     return y_ar, y_draft
 
 
+def dualpath_linear_grouped(x: torch.Tensor, Ws, As, Bms, scales, *, want_ar: bool = True,
+                            want_draft: bool = True, y_ars=None, y_drafts=None,
+                            workspace: Optional[torch.Tensor] = None):
+    """Several dual-path projections of the same x in one launch.
+
+    Ws[g] [d_out_g, d_in], As[g] [r, d_in], Bms[g] [d_out_g, r], scales[g];
+    1 to 4 projections, one dtype. `want_ar` is one flag or one per
+    projection. Returns (y_ars, y_drafts), lists with one entry per projection
+    (entries None when not wanted).
+    """
+    n = len(Ws)
+    if not (1 <= n <= 4) or len(As) != n or len(Bms) != n or len(scales) != n:
+        raise ValueError("need 1 to 4 projections with one W, A, Bm and scale each")
+    if x.dim() != 2:
+        raise ValueError("expected 2-D x")
+    M, d_in = x.shape
+    r = As[0].shape[0]
+    d_outs = []
+    for W, A, Bm in zip(Ws, As, Bms):
+        if W.dim() != 2 or A.dim() != 2 or Bm.dim() != 2:
+            raise ValueError("expected 2-D W, A, Bm")
+        d_out = W.shape[0]
+        if W.shape[1] != d_in or tuple(A.shape) != (r, d_in) or tuple(Bm.shape) != (d_out, r):
+            raise ValueError("shape mismatch: x [M,d_in], W [d_out,d_in], A [r,d_in], Bm [d_out,r]")
+        if not (x.dtype == W.dtype == A.dtype == Bm.dtype):
+            raise TypeError("x, W, A and Bm must share a dtype")
+        d_outs.append(d_out)
+    dt = _dtype_code(x)
+    dev = _check_cuda(x, *Ws, *As, *Bms)
+    y_ars = list(y_ars) if y_ars is not None else [None] * n
+    y_drafts = list(y_drafts) if y_drafts is not None else [None] * n
+    # want_ar may be one flag or one per projection; y_draft is all or none
+    wants_ar = list(want_ar) if isinstance(want_ar, (list, tuple)) else [bool(want_ar)] * n
+    if len(wants_ar) != n:
+        raise ValueError("want_ar: one flag, or one per projection")
+    for g in range(n):
+        if wants_ar[g] and y_ars[g] is None:
+            y_ars[g] = torch.empty((M, d_outs[g]), dtype=x.dtype, device=dev)
+        if want_draft and y_drafts[g] is None:
+            y_drafts[g] = torch.empty((M, d_outs[g]), dtype=x.dtype, device=dev)
+        if not wants_ar[g]:
+            y_ars[g] = None
+        if not want_draft:
+            y_drafts[g] = None
+    _check_cuda(*y_ars, *y_drafts)
+    c_dout = (ctypes.c_int * n)(*d_outs)
+    need = int(lib.uno_dualpath_grouped_workspace_bytes(n, M, d_in, c_dout, r, dt))
+    ws = workspace if workspace is not None else _ws.get(dev, "dualpath", need)
+    vpa = ctypes.c_void_p * n
+    st = lib.uno_dualpath_linear_grouped(
+        n, _ptr(x), vpa(*[_ptr(t) for t in Ws]), vpa(*[_ptr(t) for t in As]),
+        vpa(*[_ptr(t) for t in Bms]), (ctypes.c_float * n)(*[float(s) for s in scales]),
+        vpa(*[_ptr(t) for t in y_ars]), vpa(*[_ptr(t) for t in y_drafts]), M, d_in, c_dout, r,
+        dt, _ptr(ws), ws.numel(), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_dualpath_linear_grouped")
+    return y_ars, y_drafts
+
+
 def device_fault_flags(clear: bool = True) -> int:
     """Fault bits set by a kernel wait that gave up (0 = none). Synchronises."""
     flags = ctypes.c_uint(0)

@@ -72,22 +72,44 @@ enum : unsigned { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
 
 __device__ unsigned int g_fault_flags;
 
+constexpr int kMaxGroups = 4;  // projections of one launch (they share x)
+
+// One projection of a (grouped) launch.
+struct GroupArgs {
+  int ncols;          // its d_out
+  int tiles_a;        // tiles along the A operand's rows
+  int tiles;          // its main tiles
+  int tile0;          // index of its first main tile among all main tiles
+  float scale;        // alpha / r
+  void* y_ar;         // may be null
+  void* y_draft;      // may be null (then for every projection)
+  void* t_buf;        // T [M][r]
+  uint32_t* t_flags;  // [nT]
+};
+
 struct GemmParams {
   int kb_total;       // K-blocks over d_in
   int nkb_adapt;      // K-blocks over r (0: no adapter, no T tiles)
   int M;              // output rows
-  int ncols;          // output columns (d_out)
-  int rowsA, rowsB;   // rows of the main A and B operands
-  int nT;             // T tiles
+  int nT;             // T tiles per projection
+  int ngroups;        // projections in this launch
   int r;              // adapter rank
   uint32_t idesc_t;   // instruction descriptor of the T tiles
   int t_brows;        // rows of the B box of a T-tile item (per CTA)
   uint32_t epoch;     // value a T tile's flag takes once T is stored
-  float scale;        // alpha / r
-  void* y_ar;         // may be null
-  void* y_draft;      // may be null
-  void* t_buf;        // T [M][r]
-  uint32_t* t_flags;  // [nT]
+  int main_tiles;     // main tiles over all projections
+  GroupArgs g[kMaxGroups];
+};
+
+// Tensor maps of a launch: x is shared; the rest is per projection.
+struct DualMaps {
+  CUtensorMap x;               // activations [M][d_in]
+  CUtensorMap w[kMaxGroups];   // W [d_out][d_in]
+  CUtensorMap bm[kMaxGroups];  // Bm [d_out][r]
+  CUtensorMap t[kMaxGroups];   // T [M][r] (workspace)
+  CUtensorMap l[kMaxGroups];   // LoRA A [r][d_in]
+  CUtensorMap ya[kMaxGroups];  // y_ar store map (TMA-store epilogue)
+  CUtensorMap yd[kMaxGroups];  // y_draft store map
 };
 
 __host__ __device__ constexpr int pow2_at_least(int x) {
@@ -292,17 +314,15 @@ __device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
 }
 
 // ---------------------------------------------------------------------------
-// The kernel. tmA/tmB: main operands (non-swapped: x, W; swapped: W, x).
-// tmA2/tmB2: adapter operands (non-swapped: T, Bm; swapped: Bm, T). tmL: the
-// LoRA down weight A for the T tiles (non-swapped: the B side, box BN rows;
-// swapped: the A side, box 128 rows).
+// The kernel. Main operands: x and W (unswapped: x is the A side; swapped: W
+// is). Adapter operands: T and Bm (unswapped: T on the A side; swapped: Bm).
+// T tiles: x and the LoRA down weight A (unswapped: A on the B side, swapped:
+// on the A side). Every projection of a grouped launch has its own W, Bm, T,
+// A and outputs; x is shared.
 // ---------------------------------------------------------------------------
 template <typename T, int BN, bool SWAP, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmYa,
-                const __grid_constant__ CUtensorMap tmYd, const GemmParams p) {
+    dual_kernel(const __grid_constant__ DualMaps m, const __grid_constant__ GemmParams p) {
   static_assert(!(PAIR && SWAP), "the CTA pair serves the unswapped layout");
   constexpr int STAGES = stages_for<BN, PAIR>();
   constexpr int kAbytes = kBM * kRowBytes;
@@ -338,16 +358,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int my_rows = static_cast<int>(rank) * kBM;     // this CTA's row offset in a tile
   const int my_brows = static_cast<int>(rank) * kBrows;  // and in the B operand
-  const int tiles_a = (p.rowsA + kRows - 1) / kRows;
-  const int tiles_b = (p.rowsB + BN - 1) / BN;
-  const int ntiles = p.nT + tiles_a * tiles_b;
+  const int nt_all = p.nT * p.ngroups;  // T tiles of all projections come first
+  const int ntiles = nt_all + p.main_tiles;
   const int G = static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
   const int C = static_cast<int>(blockIdx.x) / (PAIR ? 2 : 1);
   const int nmine = (ntiles > C) ? (ntiles - 1 - C) / G + 1 : 0;
   // This CTA's T tiles are its first nt_mine tiles (their global indices are
   // the lowest); main tile li has ordinal li - nt_mine among its main tiles,
   // which indexes the ar_read / draft_full barriers and their phases.
-  const int nt_mine = (p.nT > C) ? (p.nT - 1 - C) / G + 1 : 0;
+  const int nt_mine = (nt_all > C) ? (nt_all - 1 - C) / G + 1 : 0;
   const int nkb = p.kb_total;
   const bool adapter = p.nkb_adapt > 0;
   const int nad = adapter ? p.nkb_adapt : 0;
@@ -370,12 +389,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     sm100::fence_mbar_init();
   }
   if (warp == kFirstProducer && lane == 0) {
-    sm100::tma_prefetch_desc(&tmA);
-    sm100::tma_prefetch_desc(&tmB);
-    if (adapter) {
-      sm100::tma_prefetch_desc(&tmA2);
-      sm100::tma_prefetch_desc(&tmB2);
-      sm100::tma_prefetch_desc(&tmL);
+    sm100::tma_prefetch_desc(&m.x);
+    for (int g = 0; g < p.ngroups; ++g) {
+      sm100::tma_prefetch_desc(&m.w[g]);
+      if (adapter) {
+        sm100::tma_prefetch_desc(&m.bm[g]);
+        sm100::tma_prefetch_desc(&m.t[g]);
+        sm100::tma_prefetch_desc(&m.l[g]);
+      }
     }
   }
   if (warp == kMmaWarp0) {
@@ -395,26 +416,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  // Local tile li of this CTA: global tile t = C + li * G. t < nT is T tile t
-  // (its A rows start at t * 128: rows of x, or with swapped operands rows of
-  // the LoRA A); otherwise main tile u = t - nT at (u % tiles_a, u / tiles_a).
+  // Local tile li of this CTA: global tile t = C + li * G. The T tiles of
+  // all projections come first, projection-major: t < nT * ngroups is T tile
+  // t % nT of projection t / nT (its A rows start at that index * kRows:
+  // rows of x, or with swapped operands rows of the LoRA A). Then main tile
+  // u = t - nT * ngroups, projection-major, at (v % tiles_a, v / tiles_a)
+  // with v its index within the projection.
   struct Tile {
     bool is_t;
+    int g;       // projection
     int a0, b0;  // first A row, first B row
-    int tt;      // T tile index
+    int tt;      // T tile index within the projection
   };
   auto tile_at = [&](int li) {
     const int t = C + li * G;
     Tile x;
-    x.is_t = t < p.nT;
-    x.tt = t;
+    x.is_t = t < nt_all;
     if (x.is_t) {
-      x.a0 = t * kRows;
+      x.g = t / p.nT;
+      x.tt = t - x.g * p.nT;
+      x.a0 = x.tt * kRows;
       x.b0 = 0;
     } else {
-      const int u = t - p.nT;
-      x.a0 = (u % tiles_a) * kRows;
-      x.b0 = (u / tiles_a) * BN;
+      const int u = t - nt_all;
+      int g = 0;
+      while (g + 1 < p.ngroups && u >= p.g[g + 1].tile0) ++g;
+      const int v = u - p.g[g].tile0;
+      x.g = g;
+      x.tt = 0;
+      x.a0 = (v % p.g[g].tiles_a) * kRows;
+      x.b0 = (v / p.g[g].tiles_a) * BN;
     }
     return x;
   };
@@ -454,7 +485,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int pr = warp - kFirstProducer;
       int it = 0;
       bool ok = true;
-      int t_ready = -1;  // previous-tile row block whose T this producer saw published
+      int t_ready = -1;  // (projection, row block) whose T this producer saw published
       // b_rows: rows of the B box (both CTAs of a pair load the same shape;
       // the leader expects the bytes of both).
       auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx,
@@ -489,13 +520,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // K-block kb + kPrefetch so that none of them waits on DRAM.
         if constexpr (!SWAP) {
           if (!x.is_t && x.a0 == 0 && kb + kPrefetch < nkb)
-            sm100::tma_prefetch_l2_2d(&tmB, kx + kPrefetch * kElemsPerRow, x.b0 + my_brows);
+            sm100::tma_prefetch_l2_2d(&m.w[x.g], kx + kPrefetch * kElemsPerRow, x.b0 + my_brows);
         }
         if (x.is_t) {
-          if constexpr (SWAP) load(&tmL, x.a0, &tmB, 0, kx, kBrows);
-          else load(&tmA, x.a0 + my_rows, &tmL, static_cast<int>(rank) * p.t_brows, kx, p.t_brows);
+          if constexpr (SWAP) load(&m.l[x.g], x.a0, &m.x, 0, kx, kBrows);
+          else load(&m.x, x.a0 + my_rows, &m.l[x.g], static_cast<int>(rank) * p.t_brows, kx, p.t_brows);
         } else {
-          load(&tmA, x.a0 + my_rows, &tmB, x.b0 + my_brows, kx, kBrows);
+          if constexpr (SWAP) load(&m.w[x.g], x.a0, &m.x, x.b0, kx, kBrows);
+          else load(&m.x, x.a0 + my_rows, &m.w[x.g], x.b0 + my_brows, kx, kBrows);
         }
       };
       int last_mine = -1;  // this producer's last ring item
@@ -514,13 +546,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             continue;
           }
           const Tile owner = (kind == 1) ? prev : cur;
-          if (t_ready != owner.a0) {
+          const int key = (owner.g << 26) | owner.a0;
+          if (t_ready != key) {
             // T must be stored before its TMA load: wait for the T tile(s)
             bool ready = true;
+            const uint32_t* fl = p.g[owner.g].t_flags;
             if constexpr (SWAP) {
-              for (int t = 0; t < p.nT && ready; ++t) ready = wait_flag(p.t_flags + t, p.epoch);
+              for (int t = 0; t < p.nT && ready; ++t) ready = wait_flag(fl + t, p.epoch);
             } else {
-              ready = wait_flag(p.t_flags + owner.a0 / kRows, p.epoch);
+              ready = wait_flag(fl + owner.a0 / kRows, p.epoch);
             }
             if (!ready) {
               set_fault(kFaultProducer, &abort_flag);
@@ -528,9 +562,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             fence_proxy_async_global();
-            t_ready = owner.a0;
+            t_ready = key;
           }
-          load(&tmA2, owner.a0 + my_rows, &tmB2, owner.b0 + my_brows, kb * kElemsPerRow, kBrows);
+          if constexpr (SWAP)
+            load(&m.bm[owner.g], owner.a0, &m.t[owner.g], owner.b0, kb * kElemsPerRow, kBrows);
+          else
+            load(&m.t[owner.g], owner.a0 + my_rows, &m.bm[owner.g], owner.b0 + my_brows,
+                 kb * kElemsPerRow, kBrows);
         }
       }
       // No copy may still be landing when the CTA exits: wait for this
@@ -645,9 +683,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       else sm100::mbar_arrive(bar);
     };
     const int rr = quarter * 32 + lane;
-    T* ya = static_cast<T*>(p.y_ar);
-    T* yd = static_cast<T*>(p.y_draft);
-    T* tb = static_cast<T*>(p.t_buf);
+    // outputs of the projection of the tile being drained
+    T* ya = nullptr;
+    T* yd = nullptr;
+    T* tb = nullptr;
+    int ncols = 0, gi = 0;
     // Drain accumulator columns [0, ncol) into y (row-major, ld columns, nrows rows).
     auto drain = [&](uint32_t acc, int a0, int b0, T* y, int ld, int nrows, int ncol,
                      float mul) {
@@ -722,8 +762,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) {
         const int row = a0;  // first of this warp's 32 rows
         for (int box = 0; box < BN / 64; ++box) {
-          if (ya) sm100::tma_store_2d(&tmYa, stage_ar + box * 4096, b0 + 64 * box, row);
-          sm100::tma_store_2d(&tmYd, stage_dr + box * 4096, b0 + 64 * box, row);
+          if (ya) sm100::tma_store_2d(&m.ya[gi], stage_ar + box * 4096, b0 + 64 * box, row);
+          sm100::tma_store_2d(&m.yd[gi], stage_dr + box * 4096, b0 + 64 * box, row);
         }
         sm100::bulk_commit_group();
         sm100::bulk_wait_group_0();
@@ -748,13 +788,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             f[e] = pass ? f[e] + __uint_as_float(w[e]) : __uint_as_float(v[e]);
           if (!y) continue;
           if constexpr (!SWAP) {
-            if (arow < p.M && brow < p.ncols)
-              store_row32<T>(y + static_cast<size_t>(arow) * p.ncols + brow, f, p.ncols - brow);
+            if (arow < p.M && brow < ncols)
+              store_row32<T>(y + static_cast<size_t>(arow) * ncols + brow, f, ncols - brow);
           } else {
-            if (arow < p.ncols) {
+            if (arow < ncols) {
 #pragma unroll
               for (int e = 0; e < 32; ++e)
-                if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * p.ncols + arow, f[e]);
+                if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * ncols + arow, f[e]);
             }
           }
         }
@@ -770,11 +810,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       sm100::tc_fence_after();
+      gi = x.g;
+      ya = static_cast<T*>(p.g[gi].y_ar);
+      yd = static_cast<T*>(p.g[gi].y_draft);
+      tb = static_cast<T*>(p.g[gi].t_buf);
+      ncols = p.g[gi].ncols;
       if (x.is_t) {
         // T = scale * x A^T: non-swapped, rows of x by r columns; swapped, r
         // rows (rows of A) by the M columns of x.
-        if constexpr (!SWAP) drain(acc, x.a0 + my_rows, 0, tb, p.r, p.M, p.r, p.scale);
-        else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.scale);
+        if constexpr (!SWAP) drain(acc, x.a0 + my_rows, 0, tb, p.r, p.M, p.r, p.g[gi].scale);
+        else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.g[gi].scale);
         sm100::tc_fence_before();
         __threadfence();
         __syncwarp();
@@ -787,7 +832,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (warp == 0 && leader) {
             if (wait_cl(t_stored, li & 1)) {
               fence_proxy_async_global();
-              st_release_u32(p.t_flags + x.tt, p.epoch);
+              st_release_u32(p.g[gi].t_flags + x.tt, p.epoch);
             } else {
               set_fault(kFaultEpilogue, &abort_flag);
             }
@@ -806,7 +851,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           drain2(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc), x.a0 + my_rows, x.b0);
         break;
       }
-      drain(acc, x.a0 + my_rows, x.b0, ya, p.ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, ya, ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
       const int mo = li - nt_mine;
@@ -818,7 +863,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       sm100::tc_fence_after();
-      drain(acc, x.a0 + my_rows, x.b0, yd, p.ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, yd, ncols, p.M, BN, 1.f);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(&acc_empty[buf]);
@@ -944,11 +989,8 @@ int max_pairs(K kern, int bytes) {
 }
 
 template <typename T, int BN, bool SWAP, bool PAIR>
-int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const CUtensorMap& l, const CUtensorMap& ya,
-                const CUtensorMap& yd, const GemmParams& p, cudaStream_t st) {
+int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
   constexpr int bytes = smem_bytes<BN, PAIR>();
-  constexpr int kRows = PAIR ? 2 * kBM : kBM;
   auto kern = dual_kernel<T, BN, SWAP, PAIR>;
   static std::atomic<uint64_t> attr_done{0};  // devices with the shared-memory opt-in
   int dev = 0;
@@ -960,8 +1002,7 @@ int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
       return UNO_ERR_CUDA;
     attr_done.fetch_or(bit, std::memory_order_relaxed);
   }
-  const long long tiles = p.nT + static_cast<long long>((p.rowsA + kRows - 1) / kRows) *
-                                     ((p.rowsB + BN - 1) / BN);
+  const long long tiles = static_cast<long long>(p.nT) * p.ngroups + p.main_tiles;
   if constexpr (PAIR) {
     long long pairs = max_pairs(kern, bytes);
     if (pairs > tiles) pairs = tiles;
@@ -977,26 +1018,22 @@ int launch_dual(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a, b, a2, b2, l, ya, yd, p) != cudaSuccess)
-      return UNO_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, maps, p) != cudaSuccess) return UNO_ERR_CUDA;
   } else {
     long long grid = sm_count();
     if (grid > tiles) grid = tiles;
-    kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(a, b, a2, b2, l, ya, yd, p);
+    kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(maps, p);
   }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
-template <typename T, bool SWAP>
-int launch_dual_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                   const CUtensorMap& b2, const CUtensorMap& l, const GemmParams& p,
-                   cudaStream_t st) {
-  // the swapped layout stores from registers; its output maps are unused
+template <typename T>
+int launch_swapped(int bn, const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
   switch (bn) {
-    case 32: return launch_dual<T, 32, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
-    case 64: return launch_dual<T, 64, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
-    case 128: return launch_dual<T, 128, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
-    default: return launch_dual<T, 256, SWAP, false>(a, b, a2, b2, l, a, a, p, st);
+    case 32: return launch_dual<T, 32, true, false>(maps, p, st);
+    case 64: return launch_dual<T, 64, true, false>(maps, p, st);
+    case 128: return launch_dual<T, 128, true, false>(maps, p, st);
+    default: return launch_dual<T, 256, true, false>(maps, p, st);
   }
 }
 
@@ -1012,6 +1049,7 @@ bool dual_sizes_ok(int M, int d_in, int d_out, int r, int dtype) {
          d_out <= (1 << 24);
 }
 
+// Per-projection workspace: T [M][r] in the operand type, then its T-tile flags.
 struct Plan {
   bool swap;
   int esize, kb_main, kb_adapt, nT;
@@ -1032,71 +1070,129 @@ Plan make_plan(int M, int d_in, int r, int dtype) {
 }
 
 template <typename T>
-int run_dualpath(const void* x, const void* W, const void* A, const void* Bm, float scale,
-                 void* y_ar, void* y_draft, int M, int d_in, int d_out, int r, int dtype,
+int run_dualpath(int n, const void* x, const void* const* W, const void* const* A,
+                 const void* const* Bm, const float* scale, void* const* y_ar,
+                 void* const* y_draft, int M, int d_in, const int* d_out, int r, int dtype,
                  void* workspace, cudaStream_t st) {
   const Plan pl = make_plan(M, d_in, r, dtype);
-  const bool adapter = (y_draft != nullptr);
-  T* Tbuf = static_cast<T*>(workspace);
-  uint32_t* flags = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + pl.t_bytes);
+  const bool adapter = (y_draft[0] != nullptr);
+  const bool tf32 = (dtype == UNO_F32);
   GemmParams gp{};
   gp.kb_total = pl.kb_main;
   gp.nkb_adapt = adapter ? pl.kb_adapt : 0;
   gp.M = M;
-  gp.ncols = d_out;
   gp.nT = adapter ? pl.nT : 0;
+  gp.ngroups = n;
   gp.r = r;
   gp.epoch = next_epoch();
+  DualMaps maps;
+  const int bn = pl.swap ? bn_for(M) : 256;
+  const int n_t = (r + 15) / 16 * 16;  // N of the unswapped T tiles
+  bool ok = pl.swap ? make_map(&maps.x, x, dtype, d_in, M, bn) : make_map(&maps.x, x, dtype, d_in, M, kBM);
+  char* ws = static_cast<char*>(workspace);
+  int tile0 = 0;
+  for (int g = 0; g < n && ok; ++g) {
+    GroupArgs& a = gp.g[g];
+    a.ncols = d_out[g];
+    a.scale = scale[g];
+    a.y_ar = y_ar[g];
+    a.y_draft = y_draft[g];
+    a.t_buf = ws;
+    a.t_flags = reinterpret_cast<uint32_t*>(ws + pl.t_bytes);
+    ws += pl.t_bytes + pl.flag_bytes;
+    if (pl.swap) {
+      a.tiles_a = (d_out[g] + kBM - 1) / kBM;
+      a.tiles = a.tiles_a * ((M + bn - 1) / bn);
+      ok = make_map(&maps.w[g], W[g], dtype, d_in, d_out[g], kBM);
+      if (adapter)
+        ok = ok && make_map(&maps.bm[g], Bm[g], dtype, r, d_out[g], kBM) &&
+             make_map(&maps.t[g], a.t_buf, dtype, r, M, bn) &&
+             make_map(&maps.l[g], A[g], dtype, d_in, r, kBM);
+    } else {
+      // a CTA pair per 256 x 256 tile (each CTA: 128 rows of x, 128 rows of W);
+      // the T tiles' N is r rounded up to 16, half of it per CTA
+      a.tiles_a = (M + 2 * kBM - 1) / (2 * kBM);
+      a.tiles = a.tiles_a * ((d_out[g] + 255) / 256);
+      ok = make_map(&maps.w[g], W[g], dtype, d_in, d_out[g], kBM);
+      if (adapter)
+        ok = ok && make_map(&maps.bm[g], Bm[g], dtype, r, d_out[g], kBM) &&
+             make_map(&maps.t[g], a.t_buf, dtype, r, M, kBM) &&
+             make_map(&maps.l[g], A[g], dtype, d_in, r, n_t / 2);
+      // output maps of the TMA-store epilogue (bf16): 32 rows x 64 columns
+      if (ok && adapter && dtype == UNO_BF16) {
+        ok = make_store_map(&maps.yd[g], y_draft[g], d_out[g], M);
+        if (ok && y_ar[g]) ok = make_store_map(&maps.ya[g], y_ar[g], d_out[g], M);
+      }
+    }
+    a.tile0 = tile0;
+    tile0 += a.tiles;
+  }
+  if (!ok) return UNO_ERR_CUDA;
+  gp.main_tiles = tile0;
   if (adapter) {
     // A captured launch replays with the epoch it was captured with, so under
     // stream capture the flags are cleared by a node of their own first.
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return UNO_ERR_CUDA;
     if (cap != cudaStreamCaptureStatusNone &&
-        cudaMemsetAsync(flags, 0, pl.flag_bytes, st) != cudaSuccess)
+        cudaMemsetAsync(workspace, 0, n * (pl.t_bytes + pl.flag_bytes), st) != cudaSuccess)
       return UNO_ERR_CUDA;
   }
-  gp.scale = scale;
-  gp.y_ar = y_ar;
-  gp.y_draft = y_draft;
-  gp.t_buf = Tbuf;
-  gp.t_flags = flags;
-  const bool tf32 = (dtype == UNO_F32);
-  CUtensorMap mA, mB, mA2, mB2, mL;
   if (pl.swap) {
-    const int bn = bn_for(M);
-    gp.rowsA = d_out;
-    gp.rowsB = M;
     gp.idesc_t = sm100::instr_desc(tf32, kBM, bn);
     gp.t_brows = bn;
-    bool ok = make_map(&mA, W, dtype, d_in, d_out, kBM) && make_map(&mB, x, dtype, d_in, M, bn);
-    if (adapter)
-      ok = ok && make_map(&mA2, Bm, dtype, r, d_out, kBM) &&
-           make_map(&mB2, Tbuf, dtype, r, M, bn) && make_map(&mL, A, dtype, d_in, r, kBM);
-    if (!ok) return UNO_ERR_CUDA;
-    if (!adapter) mA2 = mB2 = mL = mA;
-    return launch_dual_bn<T, true>(bn, mA, mB, mA2, mB2, mL, gp, st);
+    return launch_swapped<T>(bn, maps, gp, st);
   }
-  // Unswapped: a CTA pair per 256 x 256 tile (each CTA: 128 rows of x, 128
-  // rows of W); the T tiles' N is r rounded up to 16, half of it per CTA.
-  const int n_t = (r + 15) / 16 * 16;
-  gp.rowsA = M;
-  gp.rowsB = d_out;
   gp.idesc_t = sm100::instr_desc(tf32, 2 * kBM, n_t);
   gp.t_brows = n_t / 2;
-  bool ok = make_map(&mA, x, dtype, d_in, M, kBM) && make_map(&mB, W, dtype, d_in, d_out, kBM);
-  if (adapter)
-    ok = ok && make_map(&mA2, Tbuf, dtype, r, M, kBM) &&
-         make_map(&mB2, Bm, dtype, r, d_out, kBM) && make_map(&mL, A, dtype, d_in, r, n_t / 2);
-  // output maps for the TMA-store epilogue (bf16): boxes of 32 rows x 64 columns
-  CUtensorMap mYa = mA, mYd = mA;
-  if (adapter && dtype == UNO_BF16) {
-    ok = ok && make_store_map(&mYd, y_draft, d_out, M);
-    if (y_ar) ok = ok && make_store_map(&mYa, y_ar, d_out, M);
+  return launch_dual<T, 256, false, true>(maps, gp, st);
+}
+
+// Argument checks shared by the single and the grouped entry points.
+int check_dual_args(int n, const void* x, const void* const* W, const void* const* A,
+                    const void* const* Bm, void* const* y_ar, void* const* y_draft, int M,
+                    int d_in, const int* d_out, int r, int dtype, const void* workspace,
+                    size_t workspace_bytes) {
+  if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
+  if (n < 1 || n > kMaxGroups) return UNO_ERR_SIZE;
+  if (!W || !y_ar || !y_draft || !d_out) return UNO_ERR_NULL;
+  for (int g = 0; g < n; ++g)
+    if (!dual_sizes_ok(M, d_in, d_out[g], r, dtype)) return UNO_ERR_SIZE;
+  if (M == 0) return UNO_OK;
+  if (!x) return UNO_ERR_NULL;
+  const bool adapter = y_draft[0] != nullptr;
+  for (int g = 0; g < n; ++g) {
+    if (!W[g] || (!y_ar[g] && !y_draft[g])) return UNO_ERR_NULL;
+    if ((y_draft[g] != nullptr) != adapter) return UNO_ERR_NULL;  // all or none
+    if (adapter && (!A || !Bm || !A[g] || !Bm[g])) return UNO_ERR_NULL;
+    for (const void* ptr : {static_cast<const void*>(W[g]), static_cast<const void*>(y_ar[g]),
+                            static_cast<const void*>(y_draft[g]),
+                            adapter ? A[g] : nullptr, adapter ? Bm[g] : nullptr})
+      if (!uno_host::aligned(ptr, 16)) return UNO_ERR_ALIGN;
   }
-  if (!ok) return UNO_ERR_CUDA;
-  if (!adapter) mA2 = mB2 = mL = mA;
-  return launch_dual<T, 256, false, true>(mA, mB, mA2, mB2, mL, mYa, mYd, gp, st);
+  if (!workspace) return UNO_ERR_WORKSPACE;
+  if (!uno_host::aligned(x, 16) || !uno_host::aligned(workspace, 16)) return UNO_ERR_ALIGN;
+  const Plan pl = make_plan(M, d_in, r, dtype);
+  if (workspace_bytes < static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes))
+    return UNO_ERR_WORKSPACE;
+  return 1;  // proceed
+}
+
+int dispatch(int n, const void* x, const void* const* W, const void* const* A,
+             const void* const* Bm, const float* scale, void* const* y_ar, void* const* y_draft,
+             int M, int d_in, const int* d_out, int r, int dtype, void* workspace,
+             size_t workspace_bytes, void* stream) {
+  const int chk = check_dual_args(n, x, W, A, Bm, y_ar, y_draft, M, d_in, d_out, r, dtype,
+                                  workspace, workspace_bytes);
+  if (chk != 1) return chk;
+  const int dev = uno_host::check_device();
+  if (dev != UNO_OK) return dev;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == UNO_BF16)
+    return run_dualpath<uint16_t>(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r,
+                                  dtype, workspace, st);
+  return run_dualpath<float>(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype,
+                             workspace, st);
 }
 
 }  // namespace
@@ -1107,29 +1203,32 @@ extern "C" size_t uno_dualpath_workspace_bytes(int M, int d_in, int d_out, int r
   return pl.t_bytes + pl.flag_bytes;
 }
 
+extern "C" size_t uno_dualpath_grouped_workspace_bytes(int n, int M, int d_in, const int* d_out,
+                                                       int r, int dtype) {
+  if (n < 1 || n > kMaxGroups || !d_out) return 0;
+  for (int g = 0; g < n; ++g)
+    if (!dual_sizes_ok(M, d_in, d_out[g], r, dtype)) return 0;
+  const Plan pl = make_plan(M, d_in, r, dtype);
+  return static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes);
+}
+
 extern "C" int uno_dualpath_linear(const void* x, const void* W, const void* A, const void* Bm,
                                    float scale, void* y_ar, void* y_draft, int M, int d_in,
                                    int d_out, int r, int dtype, void* workspace,
                                    size_t workspace_bytes, void* stream) {
-  if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
-  if (!dual_sizes_ok(M, d_in, d_out, r, dtype)) return UNO_ERR_SIZE;
-  if (M == 0) return UNO_OK;
-  if (!x || !W || (!y_ar && !y_draft)) return UNO_ERR_NULL;
-  if (y_draft && (!A || !Bm)) return UNO_ERR_NULL;
-  if (!workspace) return UNO_ERR_WORKSPACE;
-  for (const void* ptr : {x, W, A, Bm, static_cast<const void*>(y_ar),
-                          static_cast<const void*>(y_draft), static_cast<const void*>(workspace)})
-    if (!uno_host::aligned(ptr, 16)) return UNO_ERR_ALIGN;
-  if (workspace_bytes < uno_dualpath_workspace_bytes(M, d_in, d_out, r, dtype))
-    return UNO_ERR_WORKSPACE;
-  const int dev = uno_host::check_device();
-  if (dev != UNO_OK) return dev;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == UNO_BF16)
-    return run_dualpath<uint16_t>(x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype,
-                                  workspace, st);
-  return run_dualpath<float>(x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype,
-                             workspace, st);
+  return dispatch(1, x, &W, &A, &Bm, &scale, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
+                  workspace, workspace_bytes, stream);
+}
+
+extern "C" int uno_dualpath_linear_grouped(int n, const void* x, const void* const* W,
+                                           const void* const* A, const void* const* Bm,
+                                           const float* scale, void* const* y_ar,
+                                           void* const* y_draft, int M, int d_in,
+                                           const int* d_out, int r, int dtype, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!scale) return UNO_ERR_NULL;
+  return dispatch(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype, workspace,
+                  workspace_bytes, stream);
 }
 
 extern "C" int uno_device_fault_flags(int clear, unsigned int* flags) {

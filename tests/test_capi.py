@@ -103,6 +103,31 @@ def test_argument_errors_need_no_gpu(lib):
                        16, None)] == "UNO_ERR_WORKSPACE"
     assert dual(None, None, None, None, 2.0, None, None, 0, 4096, 4096, 128, 0, None, 0,
                 None) == 0
+    # grouped dual path
+    grouped = lib.uno_dualpath_linear_grouped
+    vp3 = ctypes.c_void_p * 3
+    outs = (ctypes.c_int * 3)(4096, 1024, 1024)
+    ptrs = vp3(fake, fake, fake)
+    sc = (ctypes.c_float * 3)(2.0, 2.0, 2.0)
+    assert STATUS[grouped(0, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+                          fake, 1 << 30, None)] == "UNO_ERR_SIZE"
+    assert STATUS[grouped(5, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+                          fake, 1 << 30, None)] == "UNO_ERR_SIZE"
+    mixed = vp3(fake, None, fake)  # y_draft for some projections only
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, mixed, 16, 4096, outs, 128, 0,
+                          fake, 1 << 30, None)] == "UNO_ERR_NULL"
+    bad = (ctypes.c_int * 3)(4096, 1020, 1024)  # d_out % 8
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, bad, 128, 0,
+                          fake, 1 << 30, None)] == "UNO_ERR_SIZE"
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
+                          fake, 1 << 30, None)] == "UNO_ERR_NULL"
+    need1 = lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 128, 0)
+    assert lib.uno_dualpath_grouped_workspace_bytes(3, 16, 4096, outs, 128, 0) == 3 * need1
+    assert lib.uno_dualpath_grouped_workspace_bytes(5, 16, 4096, outs, 128, 0) == 0
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+                          fake, 3 * need1 - 1, None)] == "UNO_ERR_WORKSPACE"
+    assert grouped(3, None, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 0, 4096, outs, 128, 0, None, 0,
+                   None) == 0
 
 
 def test_binding_refuses_cpu_tensors(lib):
