@@ -415,6 +415,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   else __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // Set-up above overlaps the previous kernel on the stream; global memory
+  // (x, T, outputs, flags) is touched only after it has completed.
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
 
   // Local tile li of this CTA: global tile t = C + li * G. The T tiles of
   // all projections come first, projection-major: t < nT * ngroups is T tile
@@ -1011,18 +1015,30 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
     cfg.blockDim = dim3(kGemmThreads);
     cfg.dynamicSmemBytes = bytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, maps, p) != cudaSuccess) return UNO_ERR_CUDA;
   } else {
     long long grid = sm_count();
     if (grid > tiles) grid = tiles;
-    kern<<<static_cast<unsigned>(grid), kGemmThreads, bytes, st>>>(maps, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, maps, p) != cudaSuccess) return UNO_ERR_CUDA;
   }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }

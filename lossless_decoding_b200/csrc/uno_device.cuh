@@ -40,6 +40,19 @@ __device__ __forceinline__ uint4 verify_block_words(uint64_t seed, uint64_t step
                        make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)));
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialisation may start while the previous kernel on the stream is still
+// running; it calls grid_dependency_wait() before it touches global memory the
+// previous kernel may write or read, which returns once that kernel has
+// completed and its writes are visible. launch_dependents() lets the next
+// kernel start (its CTAs only get SMs as this kernel's CTAs leave).
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // 2^x on the SFU (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -225,6 +225,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     verify_stream_kernel(const VerifyParams P) {
   constexpr int kVec = Elem<T>::kVec;
   __shared__ float red_m[kWarps], red_z[kWarps];
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = 2 * P.K + 1;
   const int s = blockIdx.x % P.S;
@@ -428,6 +430,8 @@ struct DecideShared {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyParams P) {
   __shared__ DecideShared sh;
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
   const int tid = threadIdx.x;
   const int b = blockIdx.x;
   const int K = P.K, R = 2 * K + 1, S = P.S, V = P.V;
@@ -622,6 +626,8 @@ __device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp
 template <typename T>
 __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(const VerifyParams P) {
   __shared__ DrawShared sh;
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
   const int tid = threadIdx.x, warp = tid >> 5;
   const int b = blockIdx.x / P.SD, du = blockIdx.x % P.SD;
   const int K = P.K;
@@ -686,8 +692,9 @@ Geometry geometry(int B, int K, int V, int dtype) {
   if (cl < kChunkMin) cl = kChunkMin;
   g.chunk_len = cl;
   g.nchunks = (V + cl - 1) / cl;
-  // draw CTAs per sequence: about one wave in total, at least 8 chunks each
-  long long sd = (B > 0) ? (kDrawCtasTarget + B - 1) / B : 1;
+  // draw CTAs per sequence: at most one wave in total (a second, partial wave
+  // would double the time of the sequences it holds), at least 8 chunks each
+  long long sd = (B > 0) ? kDrawCtasTarget / B : 1;
   const long long sd_max = (g.nchunks + 7) / 8;
   if (sd > sd_max) sd = sd_max;
   if (sd < 1) sd = 1;
@@ -703,13 +710,28 @@ Geometry geometry(int B, int K, int V, int dtype) {
   return g;
 }
 
+// Launch with programmatic stream serialisation: the kernel's CTAs may start
+// while the previous kernel on the stream finishes (each waits for it before
+// touching global memory).
+template <typename Kern>
+int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
 template <typename T>
 int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
-  verify_stream_kernel<T><<<static_cast<unsigned>(g.stream_ctas), kThreads, 0, st>>>(P);
-  if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
-  verify_decide_kernel<T><<<static_cast<unsigned>(P.B), kThreads, 0, st>>>(P);
-  if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
-  verify_draw_kernel<T><<<static_cast<unsigned>(g.draw_ctas), kThreads, 0, st>>>(P);
+  if (launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  if (launch_pdl(verify_decide_kernel<T>, P.B, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  if (launch_pdl(verify_draw_kernel<T>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
