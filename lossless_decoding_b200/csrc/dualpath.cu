@@ -37,6 +37,7 @@
 // For M <= 256 the operands swap roles (W rows fill the 128-row MMA side, the
 // few activation rows are the N side), so small-batch decode still runs at full
 // tile height while it is bound by the stream of W.
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <cstdint>
@@ -98,6 +99,16 @@ struct GemmParams {
   int t_brows;        // rows of the B box of a T-tile item (per CTA)
   uint32_t epoch;     // value a T tile's flag takes once T is stored
   int main_tiles;     // main tiles over all projections
+  // The last, partial round of main tiles may be split along K so that it
+  // fills the GPU: units [split_start, split_start + n_split * split_k) are
+  // piece (j % split_k) of main tile (split_start - nT * ngroups + j / split_k).
+  // Piece 0 adds the fp32 partials of the other pieces (part_buf slots,
+  // published through part_flags) before its epilogue.
+  int split_start;    // first split unit (== total units when nothing is split)
+  int split_k;        // pieces per split tile (1: no split)
+  float* part_buf;    // [n_split][split_k - 1][CTAs per tile][128][BN] fp32
+  uint32_t* part_flags;  // [n_split][split_k - 1]
+  size_t part_capacity;  // bytes available at part_buf (host side: decides the split)
   GroupArgs g[kMaxGroups];
 };
 
@@ -359,7 +370,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int my_rows = static_cast<int>(rank) * kBM;     // this CTA's row offset in a tile
   const int my_brows = static_cast<int>(rank) * kBrows;  // and in the B operand
   const int nt_all = p.nT * p.ngroups;  // T tiles of all projections come first
-  const int ntiles = nt_all + p.main_tiles;
+  const int n_split = p.main_tiles - (p.split_start - nt_all);  // tiles of the split round
+  const int ntiles = p.split_start + n_split * p.split_k;
   const int G = static_cast<int>(gridDim.x) / (PAIR ? 2 : 1);
   const int C = static_cast<int>(blockIdx.x) / (PAIR ? 2 : 1);
   const int nmine = (ntiles > C) ? (ntiles - 1 - C) / G + 1 : 0;
@@ -431,18 +443,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int g;       // projection
     int a0, b0;  // first A row, first B row
     int tt;      // T tile index within the projection
+    int kb0, kb1;  // K-blocks of this unit (a piece of a split tile covers a part)
+    int piece;   // piece of a split tile (0: the one that finishes the tile)
+    int sidx;    // index of the split tile (-1: not split)
   };
   auto tile_at = [&](int li) {
     const int t = C + li * G;
     Tile x;
     x.is_t = t < nt_all;
+    x.kb0 = 0;
+    x.kb1 = nkb;
+    x.piece = 0;
+    x.sidx = -1;
     if (x.is_t) {
       x.g = t / p.nT;
       x.tt = t - x.g * p.nT;
       x.a0 = x.tt * kRows;
       x.b0 = 0;
     } else {
-      const int u = t - nt_all;
+      int u = t - nt_all;
+      if (t >= p.split_start) {
+        const int j = t - p.split_start;
+        x.sidx = j / p.split_k;
+        x.piece = j - x.sidx * p.split_k;
+        x.kb0 = x.piece * nkb / p.split_k;  // balanced: no piece is empty (nkb >= split_k)
+        x.kb1 = (x.piece + 1) * nkb / p.split_k;
+        u = p.split_start - nt_all + x.sidx;
+      }
       int g = 0;
       while (g + 1 < p.ngroups && u >= p.g[g + 1].tile0) ++g;
       const int v = u - p.g[g].tile0;
@@ -464,9 +491,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
   auto counts = [&](int li) {
     Counts c;
-    c.nmain = nkb;
+    const Tile x = tile_at(li);
+    c.nmain = x.kb1 - x.kb0;
     c.nprev = (li > 0 && adapter && !tile_at(li - 1).is_t) ? nad : 0;
-    c.nself = (li == nmine - 1 && adapter && !tile_at(li).is_t) ? nad : 0;
+    c.nself = (li == nmine - 1 && adapter && !x.is_t && x.piece == 0) ? nad : 0;
     return c;
   };
   // Item q of tile li: kind (0 main, 1 previous tile's adapter, 2 own adapter)
@@ -517,7 +545,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
         }
       };
-      auto load_main = [&](const Tile& x, int kb) {
+      auto load_main = [&](const Tile& x, int kb_rel) {
+        const int kb = x.kb0 + kb_rel;  // K-block within d_in
         const int kx = kb * kElemsPerRow;
         // The CTAs of one weight tile (all row blocks of x) ask for the same
         // K-block at about the same time; the first of them warms L2 for
@@ -846,6 +875,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         continue;
       }
+      if (x.sidx >= 0) {
+        // a tile split along K (the last round): pieces > 0 hand their fp32
+        // partial to piece 0, which adds them before its epilogue
+        const int nranks = PAIR ? 2 : 1;
+        const uint32_t lq = static_cast<uint32_t>(quarter * 32) << 16;
+        auto slot = [&](int piece) {
+          const size_t sl =
+              (static_cast<size_t>(x.sidx) * (p.split_k - 1) + (piece - 1)) * nranks + rank;
+          return p.part_buf + sl * (static_cast<size_t>(kBM) * BN) + static_cast<size_t>(rr) * BN;
+        };
+        uint32_t* pflags = p.part_flags + static_cast<size_t>(x.sidx) * (p.split_k - 1);
+        if (x.piece > 0) {
+          float* dst = slot(x.piece);
+          for (int c = 0; c < BN; c += 32) {
+            uint32_t v[32];
+            sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
+            sm100::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              __stcg(reinterpret_cast<float4*>(dst + c + e),
+                     make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                 __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])));
+          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) {
+            arrive_leader(t_stored);  // this CTA's T tiles used phases 0 .. nt_mine-1
+            if (warp == 0 && leader) {
+              if (wait_cl(t_stored, nt_mine & 1))
+                st_release_u32(pflags + (x.piece - 1), p.epoch);
+              else
+                set_fault(kFaultEpilogue, &abort_flag);
+            }
+          }
+          __syncwarp();
+          break;  // a split piece is this CTA's last tile
+        }
+        // piece 0: wait for the other pieces, add their partials into TMEM
+        bool ready = true;
+        if (lane == 0)
+          for (int q = 1; q < p.split_k && ready; ++q) ready = wait_flag(pflags + (q - 1), p.epoch);
+        ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
+        __syncwarp();  // orders lane 0's acquire before the other lanes' loads
+        if (!ready) {
+          if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
+          break;
+        }
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
+          sm100::tmem_ld_wait();
+          for (int q = 1; q < p.split_k; ++q) {
+            const float* src = slot(q) + c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
+              v[e] = __float_as_uint(__uint_as_float(v[e]) + f.x);
+              v[e + 1] = __float_as_uint(__uint_as_float(v[e + 1]) + f.y);
+              v[e + 2] = __float_as_uint(__uint_as_float(v[e + 2]) + f.z);
+              v[e + 3] = __float_as_uint(__uint_as_float(v[e + 3]) + f.w);
+            }
+          }
+          sm100::tmem_st_32x32b_x32(acc + lq + c, v);
+        }
+        sm100::tmem_st_wait();
+      }
       if (adapter && li == nmine - 1) {
         // last tile: y_ar in this buffer, T Bm^T in the other; one pass
         if constexpr (PAIR && sizeof(T) == 2)
@@ -965,6 +1060,10 @@ uint32_t next_epoch() {
   return e;
 }
 
+int bn_for(int rows) { return rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256; }
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
 // Clusters of two that can be resident at once (cached per device).
 template <typename K>
 int max_pairs(K kern, int bytes) {
@@ -1006,9 +1105,34 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
       return UNO_ERR_CUDA;
     attr_done.fetch_or(bit, std::memory_order_relaxed);
   }
-  const long long tiles = static_cast<long long>(p.nT) * p.ngroups + p.main_tiles;
+  const long long units0 = static_cast<long long>(p.nT) * p.ngroups + p.main_tiles;
+  const long long resident = PAIR ? max_pairs(kern, bytes) : sm_count();
+  // Split the last, partial round of main tiles along K over the CTAs (or
+  // pairs) it would leave idle: 3 or 4 pieces, each of at least 2 K-blocks.
+  // (Two pieces do not pay for the hand-off of the fp32 partial: measured on
+  // 256 x 256 tiles, the round got slower.)
+  GemmParams q = p;
+  q.split_start = static_cast<int>(units0);
+  q.split_k = 1;
+  long long tiles = units0;
+  if (units0 > resident) {
+    const long long rem = units0 % resident;
+    int k = rem > 0 ? static_cast<int>(std::min<long long>(4, resident / rem)) : 1;
+    while (k > 1 && p.kb_total < 2 * k) --k;
+    const size_t per_slot = static_cast<size_t>(PAIR ? 2 : 1) * kBM * BN * sizeof(float);
+    const size_t slots = static_cast<size_t>(rem) * (k - 1);
+    const size_t need = slots * per_slot + align256(slots * sizeof(uint32_t));
+    if (k >= 3 && units0 - rem >= static_cast<long long>(p.nT) * p.ngroups &&
+        need <= p.part_capacity) {
+      q.split_k = k;
+      q.split_start = static_cast<int>(units0 - rem);
+      q.part_flags = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(p.part_buf) +
+                                                 slots * per_slot);
+      tiles = units0 - rem + rem * k;
+    }
+  }
   if constexpr (PAIR) {
-    long long pairs = max_pairs(kern, bytes);
+    long long pairs = resident;
     if (pairs > tiles) pairs = tiles;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
@@ -1024,9 +1148,9 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, maps, p) != cudaSuccess) return UNO_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, maps, q) != cudaSuccess) return UNO_ERR_CUDA;
   } else {
-    long long grid = sm_count();
+    long long grid = resident;
     if (grid > tiles) grid = tiles;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -1038,7 +1162,7 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, maps, p) != cudaSuccess) return UNO_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, maps, q) != cudaSuccess) return UNO_ERR_CUDA;
   }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
@@ -1053,9 +1177,6 @@ int launch_swapped(int bn, const DualMaps& maps, const GemmParams& p, cudaStream
   }
 }
 
-int bn_for(int rows) { return rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256; }
-
-size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 bool dual_sizes_ok(int M, int d_in, int d_out, int r, int dtype) {
   if (dtype != UNO_BF16 && dtype != UNO_F32) return false;
@@ -1069,8 +1190,14 @@ bool dual_sizes_ok(int M, int d_in, int d_out, int r, int dtype) {
 struct Plan {
   bool swap;
   int esize, kb_main, kb_adapt, nT;
-  size_t t_bytes, flag_bytes;
+  size_t t_bytes, flag_bytes;  // per projection
+  size_t part_bytes;           // per launch: partials of a K-split last round
 };
+
+// Partials of a split round: at most (resident - 1) slots of 128 x BN fp32
+// per CTA, sized for 148 SMs so that the size does not depend on the device
+// (a device that would need more simply splits less).
+constexpr int kSizingSms = 148;
 
 Plan make_plan(int M, int d_in, int r, int dtype) {
   Plan pl{};
@@ -1082,6 +1209,10 @@ Plan make_plan(int M, int d_in, int r, int dtype) {
   pl.nT = pl.swap ? (r + kBM - 1) / kBM : (M + 2 * kBM - 1) / (2 * kBM);
   pl.t_bytes = align256(static_cast<size_t>(M) * r * pl.esize);
   pl.flag_bytes = align256(static_cast<size_t>(pl.nT) * sizeof(uint32_t));
+  const int bn = pl.swap ? bn_for(M) : 256;
+  const size_t per_slot = static_cast<size_t>(pl.swap ? 1 : 2) * kBM * bn * sizeof(float);
+  const size_t slots = static_cast<size_t>(pl.swap ? kSizingSms : kSizingSms / 2) - 1;
+  pl.part_bytes = slots * per_slot + align256(slots * sizeof(uint32_t));
   return pl;
 }
 
@@ -1145,13 +1276,16 @@ int run_dualpath(int n, const void* x, const void* const* W, const void* const* 
   }
   if (!ok) return UNO_ERR_CUDA;
   gp.main_tiles = tile0;
-  if (adapter) {
+  gp.part_buf = reinterpret_cast<float*>(ws);  // after the n per-projection areas
+  gp.part_capacity = pl.part_bytes;
+  {
     // A captured launch replays with the epoch it was captured with, so under
-    // stream capture the flags are cleared by a node of their own first.
+    // stream capture the flags are cleared by nodes of their own first.
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return UNO_ERR_CUDA;
     if (cap != cudaStreamCaptureStatusNone &&
-        cudaMemsetAsync(workspace, 0, n * (pl.t_bytes + pl.flag_bytes), st) != cudaSuccess)
+        (cudaMemsetAsync(workspace, 0, n * (pl.t_bytes + pl.flag_bytes), st) != cudaSuccess ||
+         cudaMemsetAsync(ws, 0, pl.part_bytes, st) != cudaSuccess))
       return UNO_ERR_CUDA;
   }
   if (pl.swap) {
@@ -1189,7 +1323,7 @@ int check_dual_args(int n, const void* x, const void* const* W, const void* cons
   if (!workspace) return UNO_ERR_WORKSPACE;
   if (!uno_host::aligned(x, 16) || !uno_host::aligned(workspace, 16)) return UNO_ERR_ALIGN;
   const Plan pl = make_plan(M, d_in, r, dtype);
-  if (workspace_bytes < static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes))
+  if (workspace_bytes < static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes) + pl.part_bytes)
     return UNO_ERR_WORKSPACE;
   return 1;  // proceed
 }
@@ -1216,7 +1350,7 @@ int dispatch(int n, const void* x, const void* const* W, const void* const* A,
 extern "C" size_t uno_dualpath_workspace_bytes(int M, int d_in, int d_out, int r, int dtype) {
   if (!dual_sizes_ok(M, d_in, d_out, r, dtype)) return 0;
   const Plan pl = make_plan(M, d_in, r, dtype);
-  return pl.t_bytes + pl.flag_bytes;
+  return pl.t_bytes + pl.flag_bytes + pl.part_bytes;
 }
 
 extern "C" size_t uno_dualpath_grouped_workspace_bytes(int n, int M, int d_in, const int* d_out,
@@ -1225,7 +1359,7 @@ extern "C" size_t uno_dualpath_grouped_workspace_bytes(int n, int M, int d_in, c
   for (int g = 0; g < n; ++g)
     if (!dual_sizes_ok(M, d_in, d_out[g], r, dtype)) return 0;
   const Plan pl = make_plan(M, d_in, r, dtype);
-  return static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes);
+  return static_cast<size_t>(n) * (pl.t_bytes + pl.flag_bytes) + pl.part_bytes;
 }
 
 extern "C" int uno_dualpath_linear(const void* x, const void* W, const void* A, const void* Bm,

@@ -121,11 +121,15 @@ def test_argument_errors_need_no_gpu(lib):
                           fake, 1 << 30, None)] == "UNO_ERR_SIZE"
     assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_NULL"
+    # per-projection areas (T and its flags) plus one shared area for split partials
     need1 = lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 128, 0)
-    assert lib.uno_dualpath_grouped_workspace_bytes(3, 16, 4096, outs, 128, 0) == 3 * need1
+    need3 = lib.uno_dualpath_grouped_workspace_bytes(3, 16, 4096, outs, 128, 0)
+    need2 = lib.uno_dualpath_grouped_workspace_bytes(2, 16, 4096, outs, 128, 0)
+    assert need1 < need2 < need3 < 3 * need1
+    assert need3 - need2 == need2 - need1  # one more projection adds its own area
     assert lib.uno_dualpath_grouped_workspace_bytes(5, 16, 4096, outs, 128, 0) == 0
     assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
-                          fake, 3 * need1 - 1, None)] == "UNO_ERR_WORKSPACE"
+                          fake, need3 - 1, None)] == "UNO_ERR_WORKSPACE"
     assert grouped(3, None, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 0, 4096, outs, 128, 0, None, 0,
                    None) == 0
 

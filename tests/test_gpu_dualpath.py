@@ -46,6 +46,25 @@ def _run(api, d, **kw):
     return y
 
 
+@pytest.mark.parametrize("M,d_in,d_out,r,dtype", [
+    (1024, 512, 5120, 64, "bf16"),   # 84 tile units on 74 SM pairs: last round split 4 ways
+    (1024, 256, 5120, 32, "f32"),    # the same on the TF32 path (8 K-blocks: split in 4)
+    (100, 1024, 19000, 64, "bf16"),  # swapped: 150 units on 148 SMs, last round split 4 ways
+    (520, 640, 6904, 48, "bf16"),    # 3 x 27 + 3 units: ragged rows and columns, split round
+])
+def test_parity_split_last_round(api, M, d_in, d_out, r, dtype):
+    """Tiles of a last, partial round are split along K over idle SMs; the
+    pieces' fp32 partials are added before the epilogue."""
+    d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=r, alpha=2.0 * r, dtype=dtype,
+                        seed=M + d_out)
+    y_ar, y_dr = _run(api, d)
+    ref_ar, ref_dr, _ = _ref(d)
+    assert_dualpath_close(y_ar, ref_ar)
+    assert_dualpath_close(y_dr, ref_dr)
+    y_ar2, _ = _run(api, d, want_draft=False)
+    assert_dualpath_close(y_ar2, ref_ar)
+
+
 def test_tiny_configuration_tf32(api):
     d = dualpath_inputs(M=8, d_in=512, d_out=512, r=16, alpha=32.0, dtype="f32", b_std=0.01,
                         seed=0)
