@@ -62,9 +62,9 @@ def _peaks():
 # profiles/. A figure is reported only while the kernel source it was taken on
 # is unchanged (first 16 hex digits of its sha256), else traffic is null.
 MEASURED_TRAFFIC = {
-    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "03c916a1ad285bde", 75.5e6),
-    # stream 645.5 MB + decide 0.3 MB + draw 39.0 MB, per verifier call
-    ("batched_decode_b64_k16", "verify"): ("verify.cu", "656c525e118d8d7d", 684.9e6),
+    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "dfe88fefbff16324", 136.6e6),
+    # stream 646.5 MB + decide 0.3 MB + draw 39.1 MB, per verifier call
+    ("batched_decode_b64_k16", "verify"): ("verify.cu", "d55361a025a1b14b", 685.9e6),
 }
 
 
