@@ -202,3 +202,25 @@ def test_parity_full_vocabulary(api, B, K, dtype, dist, sigma, n_check):
     assert rep.compared + rep.accept_ties + rep.draw_ties == min(n_check, B)
     assert api.device_fault_flags() == 0
     torch.cuda.empty_cache()
+
+
+def _sweep_cases():
+    """Every (B, K) of the verifier sweep (B in {1..256}, K in {4..32}), V = 151936,
+    Gumbel-like logits with a boosted top-20; dtype and the draft noise sigma
+    cycle so that each value of each meets several B and K."""
+    cases = []
+    sigmas = (0.25, 1.0, 4.0)
+    for i, B in enumerate((1, 8, 32, 64, 128, 256)):
+        for j, K in enumerate((4, 8, 16, 32)):
+            dtype = "bf16" if (i + j) % 2 == 0 else "f32"
+            cases.append((B, K, dtype, sigmas[(i + 2 * j) % 3]))
+    return cases
+
+
+@pytest.mark.parametrize("B,K,dtype,sigma", _sweep_cases())
+def test_parity_verifier_sweep(api, B, K, dtype, sigma):
+    rep = _sampled_full_size(api, B, K, 151936, dtype, "gumbel", sigma, 2, seed=7 * B + K,
+                             step=B + K)
+    assert rep.compared + rep.accept_ties + rep.draw_ties == min(2, B)
+    assert api.device_fault_flags() == 0
+    torch.cuda.empty_cache()
