@@ -315,7 +315,7 @@ def verify_block(p_logits, q_logits, draft_tokens, seed: int, step: int):
 # --------------------------------------------------------------------------
 
 
-def dualpath_linear(x, W, A, Bm, scale: float, round_t_to_bf16: bool):
+def dualpath_linear(x, W, A, Bm, scale: float, round_t_to_bf16: bool, gate=None):
     """Dual-pathway linear of a diffusion-augmented layer, float64.
 
     x [M, d_in], W [d_out, d_in] (frozen AR weight, ``nn.Linear`` layout),
@@ -324,6 +324,12 @@ def dualpath_linear(x, W, A, Bm, scale: float, round_t_to_bf16: bool):
       y_AR    = x W^T                      (verification pathway)
       T       = scale * x A^T              (rounded to bf16 if asked, reading 8)
       y_draft = y_AR + T Bm^T              (drafting pathway, theta_AR + theta_Delta)
+
+    gate [M] (optional, nonzero = adapter on): the gated LoRA of the reader
+    page, "The Psi-Speculative Sampler" (logits of token 1 of a draft block
+    use the AR weights alone, tokens 2..B the gated LoRA-augmented weights) and
+    "Supplementary Details" (the first position's clean-token distribution uses
+    theta_AR only). A row with gate 0 has T = 0, so its y_draft is its y_AR.
 
     Returns (y_AR [M, d_out], y_draft [M, d_out], T [M, r]).
     """
@@ -335,5 +341,8 @@ def dualpath_linear(x, W, A, Bm, scale: float, round_t_to_bf16: bool):
     T = float(scale) * (x @ A.T)
     if round_t_to_bf16:
         T = round_to_bf16(T)
+    if gate is not None:
+        on = np.asarray(gate).reshape(-1) != 0
+        T = np.where(on[:, None], T, 0.0)
     y_draft = y_ar + T @ Bm.T
     return y_ar, y_draft, T

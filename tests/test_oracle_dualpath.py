@@ -120,3 +120,33 @@ def test_bf16_rounding_is_nearest():
     # Nearest: error at most half a spacing (spacing = 2^(e-8) for |x| in [2^(e-1), 2^e)).
     _, e = np.frexp(x)
     assert np.all(np.abs(r - x) <= np.ldexp(0.5, e - 8))
+
+
+def test_gate_rows_are_ar_only_and_open_rows_unchanged():
+    """Gated LoRA (reader page, "The Psi-Speculative Sampler"): a closed row's
+    draft output is its AR output exactly; an open row is the ungated result."""
+    rng = np.random.default_rng(5)
+    M, d_in, d_out, r = 7, 24, 16, 8
+    x = rng.standard_normal((M, d_in))
+    W = rng.standard_normal((d_out, d_in)) * 0.1
+    A = rng.standard_normal((r, d_in)) * 0.1
+    Bm = rng.standard_normal((d_out, r)) * 0.1
+    gate = np.array([0, 1, 1, 0, 1, 0, 1], dtype=np.uint8)
+    y_ar, y_dr, T = dualpath_linear(x, W, A, Bm, 2.0, False, gate=gate)
+    y_ar0, y_dr0, T0 = dualpath_linear(x, W, A, Bm, 2.0, False)
+    assert np.array_equal(y_ar, y_ar0)
+    for m in range(M):
+        if gate[m]:
+            assert np.array_equal(y_dr[m], y_dr0[m]) and np.array_equal(T[m], T0[m])
+        else:
+            assert np.array_equal(y_dr[m], y_ar[m]) and not np.any(T[m])
+    # brute force for one open row, written out as loops
+    m = 2
+    for j in range(d_out):
+        want = sum(x[m, k] * W[j, k] for k in range(d_in))
+        want += sum(2.0 * sum(x[m, k] * A[i, k] for k in range(d_in)) * Bm[j, i]
+                    for i in range(r))
+        assert abs(y_dr[m, j] - want) < 1e-12
+    # all-open gate is the ungated call; all-closed makes the adapter vanish
+    assert np.array_equal(dualpath_linear(x, W, A, Bm, 2.0, False, gate=np.ones(M))[1], y_dr0)
+    assert np.array_equal(dualpath_linear(x, W, A, Bm, 2.0, False, gate=np.zeros(M))[1], y_ar0)
