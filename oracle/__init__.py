@@ -7,11 +7,15 @@ never import it, and it imports nothing from them.
 
 from .uno_oracle import (  # noqa: F401
     PHILOX_WORD_ACCEPT,
+    PHILOX_WORD_DRAFT,
     PHILOX_WORD_SAMPLE,
     bf16_bits_to_f64,
+    draft_uniforms,
     dualpath_linear,
     philox4x32_10,
     round_to_bf16,
+    sample_drafts,
+    sample_drafts_u,
     softmax_rows,
     uniforms_for_block,
     verify_block,

@@ -105,6 +105,7 @@ _PHILOX_W1 = np.uint64(0xBB67AE85)
 
 PHILOX_WORD_ACCEPT = 0
 PHILOX_WORD_SAMPLE = 1
+PHILOX_WORD_DRAFT = 2  # drafting a block (sample_drafts), same counter and key
 
 
 def philox4x32_10(counter: np.ndarray, key: np.ndarray) -> np.ndarray:
@@ -346,3 +347,56 @@ def dualpath_linear(x, W, A, Bm, scale: float, round_t_to_bf16: bool, gate=None)
         T = np.where(on[:, None], T, 0.0)
     y_draft = y_ar + T @ Bm.T
     return y_ar, y_draft, T
+
+
+# --------------------------------------------------------------------------
+# Drafting: the linear sampler's proposal
+# --------------------------------------------------------------------------
+
+
+def draft_uniforms(B: int, K: int, seed: int, step: int):
+    """Uniforms of a draft call: word 2 of the Philox block of (sequence b,
+    position i) with the counter and key of uniforms_for_block; [B, K]."""
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    step = int(step) & 0xFFFFFFFFFFFFFFFF
+    bb, ii = np.meshgrid(np.arange(B, dtype=np.uint64), np.arange(K, dtype=np.uint64),
+                         indexing="ij")
+    ctr = np.empty((B, K, 4), dtype=np.uint32)
+    ctr[..., 0] = bb.astype(np.uint32)
+    ctr[..., 1] = ii.astype(np.uint32)
+    ctr[..., 2] = np.uint32(step & 0xFFFFFFFF)
+    ctr[..., 3] = np.uint32(step >> 32)
+    key = np.array([seed & 0xFFFFFFFF, seed >> 32], dtype=np.uint32)
+    return word_to_uniform(philox4x32_10(ctr, key)[..., PHILOX_WORD_DRAFT])
+
+
+def sample_drafts_u(q_logits, u):
+    """Drafted ids of the linear sampler for given uniforms u [B, K].
+
+    The linear sampler draws the block's tokens in parallel, each from its
+    own marginal (reader page, "The Psi-Speculative Sampler": sample a
+    candidate set from the joint proposal, linear or tree-based; the summary
+    page's "Psi-Speculative Sampler"): x_{b,i} ~ softmax(q_{b,i}), here by the
+    inverse CDF of reading 4 over exp(q - max) in index order. A row with no
+    finite logit has no distribution: its id is -1.
+
+    Returns (ids [B, K] int32, details) where details holds the CDF
+    boundaries of each draw (for near-tie accounting).
+    """
+    q = np.asarray(q_logits, dtype=np.float64)
+    B, K, V = q.shape
+    rows = q.reshape(B * K, V)
+    finite = np.isfinite(rows).any(axis=1)
+    m = np.where(finite, np.max(np.where(np.isfinite(rows), rows, -np.inf), axis=1), 0.0)
+    w = np.where(np.isfinite(rows), np.exp(rows - m[:, None]), 0.0)
+    idx, c_prev, c_at, t, total = _inverse_cdf(w, np.asarray(u, dtype=np.float64).reshape(-1))
+    idx = np.where(finite, idx, -1).astype(np.int32)
+    details = {"c_prev": c_prev.reshape(B, K), "c_at": c_at.reshape(B, K),
+               "threshold": t.reshape(B, K), "total": total.reshape(B, K)}
+    return idx.reshape(B, K), details
+
+
+def sample_drafts(q_logits, seed: int, step: int):
+    """Drafted ids for one block: sample_drafts_u with draft_uniforms."""
+    q = np.asarray(q_logits)
+    return sample_drafts_u(q, draft_uniforms(q.shape[0], q.shape[1], seed, step))
