@@ -165,6 +165,12 @@ size_t uno_dualpath_workspace_bytes(int M, int d_in, int d_out, int r, int dtype
  *            share a workspace must be ordered on one stream.
  * Returns UNO_OK or a negative uno_status. At least one of y_ar / y_draft
  * must be non-NULL.
+ *
+ * Schedule: one persistent launch; when its last round of tiles would leave
+ * most SMs idle, each tile of that round is accumulated as 3 or 4 K-pieces
+ * whose float32 partials are added before the epilogue. Results are
+ * deterministic for a given device and call; the split depends on the SM
+ * count, so the last bits of those tiles can differ between devices.
  */
 int uno_dualpath_linear(const void* x, const void* W, const void* A, const void* Bm,
                         float scale, void* y_ar, void* y_draft, int M, int d_in, int d_out,
@@ -182,8 +188,12 @@ int uno_dualpath_linear(const void* x, const void* W, const void* A, const void*
  * Bm[g] [d_out[g], r], scale[g], y_ar[g] and y_draft[g] [M, d_out[g]]; M,
  * d_in, r and dtype are shared, with the limits of uno_dualpath_linear.
  * Either every y_draft[g] is NULL (no adapter anywhere) or none is; y_ar[g]
- * may be NULL per projection. The results equal n separate
- * uno_dualpath_linear calls bit for bit.
+ * may be NULL per projection. gate [M] (or NULL) is the per-row adapter gate of
+ * uno_dualpath_linear_gated, shared by all projections. The results equal n
+ * separate single calls bit for bit, except when a last, partial round of
+ * tiles is split along K (see uno_dualpath_linear): the grouped launch may
+ * split other tiles than the single calls, and those tiles then differ in
+ * float32 summation order only.
  * workspace  at least uno_dualpath_grouped_workspace_bytes(...) bytes, 16-byte
  *            aligned, contents irrelevant on entry (n single-call workspaces
  *            back to back).
@@ -194,9 +204,46 @@ size_t uno_dualpath_grouped_workspace_bytes(int n, int M, int d_in, const int* d
                                             int dtype);
 int uno_dualpath_linear_grouped(int n, const void* x, const void* const* W,
                                 const void* const* A, const void* const* Bm,
-                                const float* scale, void* const* y_ar, void* const* y_draft,
-                                int M, int d_in, const int* d_out, int r, int dtype,
-                                void* workspace, size_t workspace_bytes, void* stream);
+                                const float* scale, const uint8_t* gate, void* const* y_ar,
+                                void* const* y_draft, int M, int d_in, const int* d_out,
+                                int r, int dtype, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
+ * Gated dual-pathway linear. gate [M] uint8 on the device (or NULL: every row
+ * on): a row with gate 0 gets no adapter, so its y_draft equals its y_ar bit
+ * for bit; a row with a nonzero gate is the ungated result. This is the gated
+ * LoRA of the reader page, "The Psi-Speculative Sampler": when a draft block
+ * is computed, token 1 uses the AR weights alone and tokens 2..B the gated
+ * LoRA-augmented weights ("Supplementary Details": the first position's
+ * clean-token distribution uses theta_AR only), so one pass serves the block.
+ * The grouped call above takes the same gate for all its projections.
+ * Everything else is as for uno_dualpath_linear.
+ */
+int uno_dualpath_linear_gated(const void* x, const void* W, const void* A, const void* Bm,
+                              float scale, const uint8_t* gate, void* y_ar, void* y_draft,
+                              int M, int d_in, int d_out, int r, int dtype, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * Drafting a block (linear Psi-Spec sampler)
+ *
+ * Reader page, "The Psi-Speculative Sampler": the block's candidates are
+ * sampled from the joint proposal; the linear sampler draws every position in
+ * parallel from its own marginal. Here draft_tokens[b][i] ~ softmax(q[b][i])
+ * (temperature 1) by the inverse CDF over exp(q - max) in index order: the
+ * smallest v with C_v > u * C_{V-1}. The uniform u is word 2 of the Philox
+ * block of counter (b, i, step lo, step hi), key (seed lo, seed hi); words 0
+ * and 1 of the same block are the accept test and the resample of
+ * uno_verify_block, so one (seed, step) gives independent uniforms to both.
+ *
+ * q_logits      [B, K, V] dtype (bf16 or f32), rows need not be aligned
+ * draft_tokens  [B, K] int32 output; -1 for a row with no finite logit
+ * Limits: 0 <= B <= 2^20, 1 <= K <= 256, 1 <= V <= 2^28. No workspace.
+ * Asynchronous on `stream`; returns UNO_OK or a negative uno_status.
+ * ------------------------------------------------------------------------ */
+int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype, uint64_t seed,
+                      uint64_t step, int32_t* draft_tokens, void* stream);
 
 /* ------------------------------------------------------------------------ *
  * Device fault flags

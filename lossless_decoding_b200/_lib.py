@@ -58,9 +58,14 @@ def _load() -> ctypes.CDLL:
     L.uno_dualpath_linear.restype = i32
     L.uno_dualpath_grouped_workspace_bytes.argtypes = [i32, i32, i32, vp, i32, i32]
     L.uno_dualpath_grouped_workspace_bytes.restype = sz
-    L.uno_dualpath_linear_grouped.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, i32,
-                                              i32, vp, sz, vp]
+    L.uno_dualpath_linear_grouped.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
+                                              i32, i32, vp, sz, vp]
+    L.uno_dualpath_linear_gated.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, i32, i32,
+                                            i32, i32, i32, vp, sz, vp]
+    L.uno_dualpath_linear_gated.restype = i32
     L.uno_dualpath_linear_grouped.restype = i32
+    L.uno_sample_drafts.argtypes = [vp, i32, i32, i32, i32, u64, u64, vp, vp]
+    L.uno_sample_drafts.restype = i32
     L.uno_device_fault_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint)]
     L.uno_device_fault_flags.restype = i32
     return L

@@ -168,14 +168,28 @@ def dualpath_workspace_bytes(M: int, d_in: int, d_out: int, r: int, dtype: torch
     return int(lib.uno_dualpath_workspace_bytes(M, d_in, d_out, r, _DT[dtype]))
 
 
+def _gate_arg(gate: Optional[torch.Tensor], M: int, dev) -> Optional[int]:
+    if gate is None:
+        return None
+    if gate.dtype not in (torch.uint8, torch.bool) or gate.numel() != M or not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous uint8/bool tensor with one entry per row")
+    _check_cuda(gate)
+    if gate.device != dev:
+        raise ValueError("gate must live on the same device")
+    return gate.data_ptr()
+
+
 def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor,
                     scale: float, *, want_ar: bool = True, want_draft: bool = True,
                     y_ar: Optional[torch.Tensor] = None, y_draft: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None):
+                    workspace: Optional[torch.Tensor] = None,
+                    gate: Optional[torch.Tensor] = None):
     """y_ar = x W^T and y_draft = y_ar + scale (x A^T) Bm^T in one pass over W.
 
     x [M, d_in], W [d_out, d_in], A [r, d_in], Bm [d_out, r], all bfloat16 or
-    all float32. Returns (y_ar, y_draft); an output not wanted is None.
+    all float32. gate [M] (uint8/bool, optional): rows with gate 0 get no
+    adapter (their y_draft equals y_ar). Returns (y_ar, y_draft); an output not
+    wanted is None.
     """
     if x.dim() != 2 or W.dim() != 2 or A.dim() != 2 or Bm.dim() != 2:
         raise ValueError("expected 2-D x, W, A, Bm")
@@ -199,9 +213,15 @@ def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch
     _check_cuda(y_ar, y_draft)
     need = int(lib.uno_dualpath_workspace_bytes(M, d_in, d_out, r, dt))
     ws = workspace if workspace is not None else _ws.get(dev, "dualpath", need)
-    st = lib.uno_dualpath_linear(_ptr(x), _ptr(W), _ptr(A), _ptr(Bm), ctypes.c_float(scale),
-                                 _ptr(y_ar), _ptr(y_draft), M, d_in, d_out, r, dt, _ptr(ws),
-                                 ws.numel(), _stream_handle(dev))
+    if gate is None:
+        st = lib.uno_dualpath_linear(_ptr(x), _ptr(W), _ptr(A), _ptr(Bm), ctypes.c_float(scale),
+                                     _ptr(y_ar), _ptr(y_draft), M, d_in, d_out, r, dt, _ptr(ws),
+                                     ws.numel(), _stream_handle(dev))
+    else:
+        st = lib.uno_dualpath_linear_gated(_ptr(x), _ptr(W), _ptr(A), _ptr(Bm),
+                                           ctypes.c_float(scale), _gate_arg(gate, M, dev),
+                                           _ptr(y_ar), _ptr(y_draft), M, d_in, d_out, r, dt,
+                                           _ptr(ws), ws.numel(), _stream_handle(dev))
     if st != 0:
         raise UnoError(st, "uno_dualpath_linear")
     return y_ar, y_draft
@@ -209,7 +229,8 @@ def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch
 
 def dualpath_linear_grouped(x: torch.Tensor, Ws, As, Bms, scales, *, want_ar: bool = True,
                             want_draft: bool = True, y_ars=None, y_drafts=None,
-                            workspace: Optional[torch.Tensor] = None):
+                            workspace: Optional[torch.Tensor] = None,
+                            gate: Optional[torch.Tensor] = None):
     """Several dual-path projections of the same x in one launch.
 
     Ws[g] [d_out_g, d_in], As[g] [r, d_in], Bms[g] [d_out_g, r], scales[g];
@@ -259,11 +280,42 @@ def dualpath_linear_grouped(x: torch.Tensor, Ws, As, Bms, scales, *, want_ar: bo
     st = lib.uno_dualpath_linear_grouped(
         n, _ptr(x), vpa(*[_ptr(t) for t in Ws]), vpa(*[_ptr(t) for t in As]),
         vpa(*[_ptr(t) for t in Bms]), (ctypes.c_float * n)(*[float(s) for s in scales]),
-        vpa(*[_ptr(t) for t in y_ars]), vpa(*[_ptr(t) for t in y_drafts]), M, d_in, c_dout, r,
+        _gate_arg(gate, M, dev), vpa(*[_ptr(t) for t in y_ars]), vpa(*[_ptr(t) for t in y_drafts]), M, d_in, c_dout, r,
         dt, _ptr(ws), ws.numel(), _stream_handle(dev))
     if st != 0:
         raise UnoError(st, "uno_dualpath_linear_grouped")
     return y_ars, y_drafts
+
+
+# ---------------------------------------------------------------------------
+# drafting a block
+# ---------------------------------------------------------------------------
+
+
+def sample_drafts(q_logits: torch.Tensor, seed: int, step: int, *,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Drafted ids of the linear sampler: out[b, i] ~ softmax(q_logits[b, i]).
+
+    q_logits [B, K, V] bfloat16 or float32 on a CUDA device; returns int32
+    [B, K] (-1 for a row with no finite logit). Uniform: Philox word 2 of
+    (b, i, step) under key `seed`, next to the verifier's words 0 and 1.
+    """
+    if q_logits.dim() != 3:
+        raise ValueError("q_logits must be [B, K, V]")
+    B, K, V = q_logits.shape
+    dt = _dtype_code(q_logits)
+    dev = _check_cuda(q_logits)
+    if out is None:
+        out = torch.empty((B, K), dtype=torch.int32, device=dev)
+    if out.dtype != torch.int32 or tuple(out.shape) != (B, K):
+        raise ValueError("out must be int32 [B, K]")
+    _check_cuda(out)
+    st = lib.uno_sample_drafts(_ptr(q_logits), B, K, V, dt, ctypes.c_uint64(seed & (2**64 - 1)),
+                               ctypes.c_uint64(step & (2**64 - 1)), _ptr(out),
+                               _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_sample_drafts")
+    return out
 
 
 def device_fault_flags(clear: bool = True) -> int:

@@ -1,0 +1,316 @@
+// Drafting a block with the linear Psi-Spec sampler on sm_100a.
+//
+// "Unlocking Lossless Speedups in LLMs via Discrete Diffusion", reader page,
+// "The Psi-Speculative Sampler": the block's candidate tokens are sampled from
+// the joint proposal; the linear sampler draws every position in parallel
+// from its own marginal. Here x_{b,i} ~ softmax(q_{b,i}) by the inverse CDF
+// over exp(q - max) in index order, with the uniform taken from word 2 of the
+// Philox block of (b, i, step) under the verifier's key (words 0 and 1 serve
+// the accept test and the resample), so drafting, verification and
+// resampling draw independent uniforms from one stream.
+//
+// One CTA per row (b, i), one pass over the row in HBM: each warp takes
+// chunks of the row (one 16-byte vector per lane per step), reduces each chunk
+// to (chunk max, sum of 2^(x - chunk max)) in the log2 domain and keeps it in
+// shared memory. The CTA then rescales the chunk sums to the row maximum,
+// takes their float64 running sum, finds the chunk where u * total is crossed
+// and scans only that chunk (in L2 by then) for the token.
+#include <climits>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "uno.h"
+#include "uno_device.cuh"
+#include "uno_host.h"
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxChunks = 2048;  // chunk table in shared memory (16 KB)
+constexpr int kInFlight = 4;      // chunks a warp loads before reducing them
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T>
+struct Row;
+
+template <>
+struct Row<uint16_t> {  // bfloat16 bits
+  static constexpr int kVec = 8;
+  __device__ static __forceinline__ float at(const uint16_t* p, long long i) {
+    return uno::bf16_bits_to_float(__ldg(p + i));
+  }
+  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <>
+struct Row<float> {
+  static constexpr int kVec = 4;
+  __device__ static __forceinline__ float at(const float* p, long long i) { return __ldg(p + i); }
+  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+};
+
+struct SampleParams {
+  const void* q;       // [B][K][V]
+  int B, K, V;
+  int chunk_len;       // elements per chunk (a multiple of 32 * kVec)
+  int nchunks;
+  uint64_t seed, step;
+  int32_t* out;        // [B][K]
+};
+
+struct Shared {
+  float cm[kMaxChunks];  // chunk maximum (log2 domain), -inf when empty
+  float cs[kMaxChunks];  // sum over the chunk of 2^(x log2 e - cm)
+  double warp_tot[kWarps];
+  float warp_max[kWarps];
+  double carry;
+  int chunk, last_pos, token;
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Exclusive running sum (float64, thread order) across the CTA; the total is
+// returned through *total.
+__device__ double block_exclusive_scan(double mine, Shared& sh, double* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double up = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += up;
+  }
+  if (lane == 31) sh.warp_tot[warp] = incl;
+  __syncthreads();
+  double before = 0.0, all = 0.0;
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) before += sh.warp_tot[w];
+    all += sh.warp_tot[w];
+  }
+  *total = all;
+  __syncthreads();
+  return before + incl - mine;
+}
+
+// Element v of the row, in the log2 domain (-inf stays -inf).
+template <typename T>
+__device__ __forceinline__ float l2(const T* row, long long v) {
+  return Row<T>::at(row, v) * kLog2e;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) sample_drafts_kernel(const SampleParams P) {
+  __shared__ Shared sh;
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
+  constexpr int kVec = Row<T>::kVec;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bi = blockIdx.x;  // b * K + i
+  const int b = bi / P.K, i = bi - b * P.K;
+  const T* row = static_cast<const T*>(P.q) + static_cast<size_t>(bi) * P.V;
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  const int V = P.V, L = P.chunk_len;
+
+  // ---- pass 1: per-chunk (max, sum of 2^(x - max)) ----
+  for (int c0 = warp; c0 < P.nchunks; c0 += kWarps * kInFlight) {
+    float cmax[kInFlight], csum[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      cmax[k] = -INFINITY;
+      csum[k] = 0.f;
+    }
+    // a chunk is L / (32 kVec) steps of one vector per lane
+    for (int s = 0; s < L; s += 32 * kVec) {
+      float f[kInFlight][kVec];
+#pragma unroll
+      for (int k = 0; k < kInFlight; ++k) {
+        const int c = c0 + k * kWarps;
+        const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
+        if (c < P.nchunks && vec && v0 + kVec <= V) {
+          Row<T>::unpack(__ldg(reinterpret_cast<const uint4*>(row + v0)), f[k]);
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) f[k][e] *= kLog2e;
+        } else {
+#pragma unroll
+          for (int e = 0; e < kVec; ++e)
+            f[k][e] = (c < P.nchunks && v0 + e < V) ? l2(row, v0 + e) : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kInFlight; ++k) {
+        float m = cmax[k];
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) m = fmaxf(m, f[k][e]);
+        m = warp_max(m);  // the chunk's running maximum, same in every lane
+        if (m > -INFINITY) {
+          csum[k] *= uno::ex2(cmax[k] - m);  // rescale what came before
+          float add = 0.f;
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) add += uno::ex2(f[k][e] - m);
+          csum[k] += add;
+          cmax[k] = m;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const int c = c0 + k * kWarps;
+      const float t = warp_sum(csum[k]);
+      if (lane == 0 && c < P.nchunks) {
+        sh.cm[c] = cmax[k];
+        sh.cs[c] = (cmax[k] > -INFINITY) ? t : 0.f;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- the row maximum and the rescaled chunk sums ----
+  float mx = -INFINITY;
+  for (int c = tid; c < P.nchunks; c += kThreads) mx = fmaxf(mx, sh.cm[c]);
+  mx = warp_max(mx);
+  if (lane == 0) sh.warp_max[warp] = mx;
+  if (tid == 0) {
+    sh.chunk = INT_MAX;
+    sh.last_pos = -1;
+    sh.token = INT_MAX;
+  }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sh.warp_max[w]);
+  if (M == -INFINITY) {  // no finite logit: no distribution
+    if (tid == 0) P.out[bi] = -1;
+    return;
+  }
+  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, i).z);
+  // thread t owns chunks [t * per, (t + 1) * per)
+  const int per = (P.nchunks + kThreads - 1) / kThreads;
+  const int c_lo = tid * per, c_hi = min(c_lo + per, P.nchunks);
+  double mine = 0.0;
+  int last_pos_chunk = -1;
+  for (int c = c_lo; c < c_hi; ++c) {
+    const double w = (sh.cm[c] > -INFINITY) ? static_cast<double>(sh.cs[c]) *
+                                                  static_cast<double>(uno::ex2(sh.cm[c] - M))
+                                            : 0.0;
+    mine += w;
+    if (w > 0.0) last_pos_chunk = c;
+  }
+  double total = 0.0;
+  const double before = block_exclusive_scan(mine, sh, &total);
+  const double t = static_cast<double>(u) * total;
+  {
+    double run = before;
+    int found = -1;
+    for (int c = c_lo; c < c_hi && found < 0; ++c) {
+      const double w = (sh.cm[c] > -INFINITY) ? static_cast<double>(sh.cs[c]) *
+                                                    static_cast<double>(uno::ex2(sh.cm[c] - M))
+                                              : 0.0;
+      if (run + w > t) found = c;
+      else run += w;
+    }
+    if (found >= 0) atomicMin(&sh.chunk, found);
+    if (last_pos_chunk >= 0) atomicMax(&sh.last_pos, last_pos_chunk);
+    __syncthreads();
+    if (found >= 0 && found == sh.chunk) sh.carry = run;  // running sum before that chunk
+  }
+  __syncthreads();
+  // Rounding can leave no crossing: then the last chunk with positive weight.
+  const bool crossed = sh.chunk != INT_MAX;
+  const int ch = crossed ? sh.chunk : sh.last_pos;
+  double carry = crossed ? sh.carry : 0.0;
+  __syncthreads();
+  if (tid == 0) sh.last_pos = -1;
+  __syncthreads();
+
+  // ---- scan the chosen chunk (whole CTA, kThreads elements per step) ----
+  const long long v_lo = static_cast<long long>(ch) * L;
+  const long long v_hi = min(v_lo + L, static_cast<long long>(V));
+  for (long long base = v_lo; base < v_hi; base += kThreads) {
+    const long long v = base + tid;
+    const float w = (v < v_hi) ? uno::ex2(l2(row, v) - M) : 0.f;
+    double step_total = 0.0;
+    const double bef = carry + block_exclusive_scan(static_cast<double>(w), sh, &step_total);
+    if (crossed && w > 0.f && bef + static_cast<double>(w) > t)
+      atomicMin(&sh.token, static_cast<int>(v));
+    if (w > 0.f) atomicMax(&sh.last_pos, static_cast<int>(v));
+    carry += step_total;
+    __syncthreads();
+    if (sh.token != INT_MAX) break;
+  }
+  if (tid == 0) P.out[bi] = (sh.token != INT_MAX) ? sh.token : sh.last_pos;
+}
+
+bool sample_sizes_ok(int B, int K, int V, int dtype) {
+  return (dtype == UNO_BF16 || dtype == UNO_F32) && B >= 0 && B <= (1 << 20) && K >= 1 &&
+         K <= 256 && V >= 1 && V <= (1 << 28) && static_cast<long long>(B) * K <= (1 << 28);
+}
+
+template <typename T>
+int run(const void* q, int B, int K, int V, uint64_t seed, uint64_t step, int32_t* out,
+        cudaStream_t st) {
+  constexpr int kStep = 32 * Row<T>::kVec;  // elements per vector step of a warp
+  SampleParams P{};
+  P.q = q;
+  P.B = B;
+  P.K = K;
+  P.V = V;
+  P.seed = seed;
+  P.step = step;
+  P.out = out;
+  const long long steps = (static_cast<long long>(V) + kStep - 1) / kStep;
+  const long long per_chunk = (steps + kMaxChunks - 1) / kMaxChunks;  // steps per chunk
+  P.chunk_len = static_cast<int>(per_chunk * kStep);
+  P.nchunks = static_cast<int>((V + P.chunk_len - 1) / P.chunk_len);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(B * K));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, sample_drafts_kernel<T>, P) != cudaSuccess) return UNO_ERR_CUDA;
+  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype,
+                                 uint64_t seed, uint64_t step, int32_t* draft_tokens,
+                                 void* stream) {
+  if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
+  if (!sample_sizes_ok(B, K, V, dtype)) return UNO_ERR_SIZE;
+  if (B == 0) return UNO_OK;
+  if (!q_logits || !draft_tokens) return UNO_ERR_NULL;
+  if (!uno_host::aligned(q_logits, dtype == UNO_BF16 ? 2 : 4) ||
+      !uno_host::aligned(draft_tokens, 4))
+    return UNO_ERR_ALIGN;
+  const int dev = uno_host::check_device();
+  if (dev != UNO_OK) return dev;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == UNO_BF16) return run<uint16_t>(q_logits, B, K, V, seed, step, draft_tokens, st);
+  return run<float>(q_logits, B, K, V, seed, step, draft_tokens, st);
+}

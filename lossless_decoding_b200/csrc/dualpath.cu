@@ -109,6 +109,7 @@ struct GemmParams {
   float* part_buf;    // [n_split][split_k - 1][CTAs per tile][128][BN] fp32
   uint32_t* part_flags;  // [n_split][split_k - 1]
   size_t part_capacity;  // bytes available at part_buf (host side: decides the split)
+  const uint8_t* gate;   // [M] per-row adapter gate (0: AR only), or null (all on)
   GroupArgs g[kMaxGroups];
 };
 
@@ -722,11 +723,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     T* tb = nullptr;
     int ncols = 0, gi = 0;
     // Drain accumulator columns [0, ncol) into y (row-major, ld columns, nrows rows).
+    // gate: for T tiles, the per-row adapter gate (rows of x: the A rows
+    // unswapped, the B rows swapped); a closed row stores T = 0.
     auto drain = [&](uint32_t acc, int a0, int b0, T* y, int ld, int nrows, int ncol,
-                     float mul) {
+                     float mul, const uint8_t* gate = nullptr) {
       if (!y) return;
       const uint32_t tq = acc + (static_cast<uint32_t>(quarter * 32) << 16);
       const int arow = a0 + rr;
+      if constexpr (!SWAP) {
+        if (gate && arow < nrows && gate[arow] == 0) mul = 0.f;
+      }
       for (int c = 0; c < ncol; c += 32) {
         uint32_t v[32];
         sm100::tmem_ld_32x32b_x32(tq + c, v);
@@ -735,6 +741,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * mul;
         const int brow = b0 + c;
+        if constexpr (SWAP) {
+          if (gate) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (brow + e < nrows && gate[brow + e] == 0) f[e] = 0.f;
+          }
+        }
         if constexpr (!SWAP) {
           // row = A row, column = B row
           if (arow < nrows && brow < ld)
@@ -851,8 +864,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (x.is_t) {
         // T = scale * x A^T: non-swapped, rows of x by r columns; swapped, r
         // rows (rows of A) by the M columns of x.
-        if constexpr (!SWAP) drain(acc, x.a0 + my_rows, 0, tb, p.r, p.M, p.r, p.g[gi].scale);
-        else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.g[gi].scale);
+        if constexpr (!SWAP) drain(acc, x.a0 + my_rows, 0, tb, p.r, p.M, p.r, p.g[gi].scale, p.gate);
+        else drain(acc, x.a0, 0, tb, p.r, p.M, BN, p.g[gi].scale, p.gate);
         sm100::tc_fence_before();
         __threadfence();
         __syncwarp();
@@ -1218,9 +1231,9 @@ Plan make_plan(int M, int d_in, int r, int dtype) {
 
 template <typename T>
 int run_dualpath(int n, const void* x, const void* const* W, const void* const* A,
-                 const void* const* Bm, const float* scale, void* const* y_ar,
-                 void* const* y_draft, int M, int d_in, const int* d_out, int r, int dtype,
-                 void* workspace, cudaStream_t st) {
+                 const void* const* Bm, const float* scale, const uint8_t* gate,
+                 void* const* y_ar, void* const* y_draft, int M, int d_in, const int* d_out,
+                 int r, int dtype, void* workspace, cudaStream_t st) {
   const Plan pl = make_plan(M, d_in, r, dtype);
   const bool adapter = (y_draft[0] != nullptr);
   const bool tf32 = (dtype == UNO_F32);
@@ -1231,6 +1244,7 @@ int run_dualpath(int n, const void* x, const void* const* W, const void* const* 
   gp.nT = adapter ? pl.nT : 0;
   gp.ngroups = n;
   gp.r = r;
+  gp.gate = gate;
   gp.epoch = next_epoch();
   DualMaps maps;
   const int bn = pl.swap ? bn_for(M) : 256;
@@ -1329,9 +1343,9 @@ int check_dual_args(int n, const void* x, const void* const* W, const void* cons
 }
 
 int dispatch(int n, const void* x, const void* const* W, const void* const* A,
-             const void* const* Bm, const float* scale, void* const* y_ar, void* const* y_draft,
-             int M, int d_in, const int* d_out, int r, int dtype, void* workspace,
-             size_t workspace_bytes, void* stream) {
+             const void* const* Bm, const float* scale, const uint8_t* gate, void* const* y_ar,
+             void* const* y_draft, int M, int d_in, const int* d_out, int r, int dtype,
+             void* workspace, size_t workspace_bytes, void* stream) {
   const int chk = check_dual_args(n, x, W, A, Bm, y_ar, y_draft, M, d_in, d_out, r, dtype,
                                   workspace, workspace_bytes);
   if (chk != 1) return chk;
@@ -1339,10 +1353,10 @@ int dispatch(int n, const void* x, const void* const* W, const void* const* A,
   if (dev != UNO_OK) return dev;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == UNO_BF16)
-    return run_dualpath<uint16_t>(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r,
+    return run_dualpath<uint16_t>(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r,
                                   dtype, workspace, st);
-  return run_dualpath<float>(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype,
-                             workspace, st);
+  return run_dualpath<float>(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r,
+                             dtype, workspace, st);
 }
 
 }  // namespace
@@ -1366,19 +1380,29 @@ extern "C" int uno_dualpath_linear(const void* x, const void* W, const void* A, 
                                    float scale, void* y_ar, void* y_draft, int M, int d_in,
                                    int d_out, int r, int dtype, void* workspace,
                                    size_t workspace_bytes, void* stream) {
-  return dispatch(1, x, &W, &A, &Bm, &scale, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
+  return dispatch(1, x, &W, &A, &Bm, &scale, nullptr, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
+                  workspace, workspace_bytes, stream);
+}
+
+extern "C" int uno_dualpath_linear_gated(const void* x, const void* W, const void* A,
+                                         const void* Bm, float scale, const uint8_t* gate,
+                                         void* y_ar, void* y_draft, int M, int d_in, int d_out,
+                                         int r, int dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  return dispatch(1, x, &W, &A, &Bm, &scale, gate, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
                   workspace, workspace_bytes, stream);
 }
 
 extern "C" int uno_dualpath_linear_grouped(int n, const void* x, const void* const* W,
                                            const void* const* A, const void* const* Bm,
-                                           const float* scale, void* const* y_ar,
-                                           void* const* y_draft, int M, int d_in,
-                                           const int* d_out, int r, int dtype, void* workspace,
-                                           size_t workspace_bytes, void* stream) {
+                                           const float* scale, const uint8_t* gate,
+                                           void* const* y_ar, void* const* y_draft, int M,
+                                           int d_in, const int* d_out, int r, int dtype,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream) {
   if (!scale) return UNO_ERR_NULL;
-  return dispatch(n, x, W, A, Bm, scale, y_ar, y_draft, M, d_in, d_out, r, dtype, workspace,
-                  workspace_bytes, stream);
+  return dispatch(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r, dtype,
+                  workspace, workspace_bytes, stream);
 }
 
 extern "C" int uno_device_fault_flags(int clear, unsigned int* flags) {

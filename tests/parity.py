@@ -102,3 +102,17 @@ def assert_dualpath_close(got: torch.Tensor, ref: np.ndarray, tol: float = 2e-2)
     bad = np.abs(g - ref) > tol * np.abs(ref) + tol * rms
     assert not bad.any(), f"{int(bad.sum())} elements outside the elementwise bound"
     return e
+
+
+def compare_drafts(got: np.ndarray, ids: np.ndarray, det: dict) -> tuple[int, int]:
+    """Drafted ids of the CUDA sampler against the oracle: equal except draws
+    whose threshold lies within TAU_ABS + TAU_REL * total of a CDF boundary
+    (the verifier's draw rule). Returns (compared, ties)."""
+    got = np.asarray(got)
+    assert got.shape == ids.shape
+    t, lo, hi, tot = det["threshold"], det["c_prev"], det["c_at"], det["total"]
+    tie = np.minimum(t - lo, hi - t) < TAU_ABS + TAU_REL * tot
+    tie &= ids >= 0
+    bad = (got != ids) & ~tie
+    assert not bad.any(), f"{int(bad.sum())} drafted ids differ, first at {np.argwhere(bad)[0]}"
+    return int((~tie).sum()), int(tie.sum())

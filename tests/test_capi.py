@@ -109,17 +109,17 @@ def test_argument_errors_need_no_gpu(lib):
     outs = (ctypes.c_int * 3)(4096, 1024, 1024)
     ptrs = vp3(fake, fake, fake)
     sc = (ctypes.c_float * 3)(2.0, 2.0, 2.0)
-    assert STATUS[grouped(0, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+    assert STATUS[grouped(0, fake, ptrs, ptrs, ptrs, sc, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_SIZE"
-    assert STATUS[grouped(5, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+    assert STATUS[grouped(5, fake, ptrs, ptrs, ptrs, sc, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_SIZE"
     mixed = vp3(fake, None, fake)  # y_draft for some projections only
-    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, mixed, 16, 4096, outs, 128, 0,
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, None, ptrs, mixed, 16, 4096, outs, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_NULL"
     bad = (ctypes.c_int * 3)(4096, 1020, 1024)  # d_out % 8
-    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, bad, 128, 0,
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, None, ptrs, ptrs, 16, 4096, bad, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_SIZE"
-    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, None, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
                           fake, 1 << 30, None)] == "UNO_ERR_NULL"
     # per-projection areas (T and its flags) plus one shared area for split partials
     need1 = lib.uno_dualpath_workspace_bytes(16, 4096, 4096, 128, 0)
@@ -128,9 +128,9 @@ def test_argument_errors_need_no_gpu(lib):
     assert need1 < need2 < need3 < 3 * need1
     assert need3 - need2 == need2 - need1  # one more projection adds its own area
     assert lib.uno_dualpath_grouped_workspace_bytes(5, 16, 4096, outs, 128, 0) == 0
-    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 16, 4096, outs, 128, 0,
+    assert STATUS[grouped(3, fake, ptrs, ptrs, ptrs, sc, None, ptrs, ptrs, 16, 4096, outs, 128, 0,
                           fake, need3 - 1, None)] == "UNO_ERR_WORKSPACE"
-    assert grouped(3, None, ptrs, ptrs, ptrs, sc, ptrs, ptrs, 0, 4096, outs, 128, 0, None, 0,
+    assert grouped(3, None, ptrs, ptrs, ptrs, sc, None, ptrs, ptrs, 0, 4096, outs, 128, 0, None, 0,
                    None) == 0
 
 

@@ -169,3 +169,41 @@ def test_batched_decode_projections_sampled_rows(api, name, d_in, d_out):
     assert_dualpath_close(y_ar[ri], ref_ar)
     assert_dualpath_close(y_dr[ri], ref_dr)
     assert api.device_fault_flags() == 0
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,dtype", [
+    (17, 512, 1000, 64, "bf16"),     # swapped layout: K = 16 drafts + bonus row
+    (520, 256, 384, 32, "bf16"),     # CTA-pair layout, ragged rows
+    (100, 1024, 19000, 64, "bf16"),  # swapped with a split last round
+    (300, 260, 136, 20, "f32"),      # TF32 pair layout
+])
+def test_gated_dual_path(api, M, d_in, d_out, r, dtype):
+    """Per-row adapter gate (gated LoRA): a closed row's y_draft is its y_ar bit
+    for bit, an open row is exactly the ungated result; parity with the gated
+    oracle. The gate closes the first position of each block of K+1 = 17 rows
+    (AR only) plus a few random rows."""
+    d = dualpath_inputs(M=M, d_in=d_in, d_out=d_out, r=r, alpha=2.0 * r, dtype=dtype, seed=M + r)
+    g = torch.ones(M, dtype=torch.uint8)
+    g[::17] = 0
+    g[torch.randperm(M, generator=torch.Generator().manual_seed(M))[: max(1, M // 10)]] = 0
+    gate = g.to(DEV)
+    y_ar, y_dr = _run(api, d, gate=gate)
+    y_ar0, y_dr0 = _run(api, d)
+    closed = g == 0
+    assert torch.equal(y_ar, y_ar0)
+    assert torch.equal(y_dr[closed.to(DEV)], y_ar[closed.to(DEV)])
+    assert torch.equal(y_dr[~closed.to(DEV)], y_dr0[~closed.to(DEV)])
+    ref_ar, ref_dr, _ = oracle.dualpath_linear(
+        widen(d.x), widen(d.W), widen(d.A), widen(d.Bm), d.scale,
+        round_t_to_bf16=(d.x.dtype == torch.bfloat16), gate=g.numpy())
+    assert_dualpath_close(y_dr, ref_dr)
+    # grouped launches take the same gate for every projection (their last
+    # round may be split along K differently from the single call, so the
+    # comparison is against the oracle, and closed rows stay exact)
+    ys_ar, ys_dr = api.dualpath_linear_grouped(d.x.to(DEV), [d.W.to(DEV)] * 2, [d.A.to(DEV)] * 2,
+                                               [d.Bm.to(DEV)] * 2, [d.scale] * 2, gate=gate)
+    torch.cuda.synchronize()
+    for ya, yd in zip(ys_ar, ys_dr):
+        assert torch.equal(yd[closed.to(DEV)], ya[closed.to(DEV)])
+        assert_dualpath_close(ya, ref_ar)
+        assert_dualpath_close(yd, ref_dr)

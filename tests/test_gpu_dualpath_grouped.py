@@ -1,8 +1,9 @@
 """Grouped dual-path launches (several projections of one x) on a B200.
 
 A grouped launch must give every projection exactly what a separate
-uno_dualpath_linear call gives (same tiles, same arithmetic: bit for bit) and
-both must match the float64 oracle within the dual-path criterion
+uno_dualpath_linear call gives (same tiles, same arithmetic: bit for bit; the
+shapes here are small enough that no launch splits its last round along K)
+and both must match the float64 oracle within the dual-path criterion
 (tests/parity.py). Covers the swapped (M <= 256) and the CTA-pair (M > 256)
 layouts, bf16 and f32, ragged output widths and projections without y_ar.
 """
