@@ -257,6 +257,29 @@ class BatchedDecode:
         if ev is not None:
             ev[3].record()
 
+    def extra_measurements(self, stream, reps=20):
+        """Rows beyond the step: the on-device draft sampler over this
+        workload's draft logits (B x K x V), timed alone with CUDA events on
+        the launching stream (inputs larger than L2), against the HBM peak."""
+        ids = torch.empty((self.B, self.K), dtype=torch.int32, device=self.out.out_tokens.device)
+        for i in range(3):
+            self.api.sample_drafts(self.v.q_logits, self.philox_seed, i, out=ids)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(reps):
+            self.api.sample_drafts(self.v.q_logits, self.philox_seed, 100 + i, out=ids)
+        b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / reps
+        nbytes = self.v.q_logits.numel() * self.v.q_logits.element_size() + ids.numel() * 4
+        gbs = nbytes / (us / 1e6) / 1e9
+        peak = _peaks()["hbm"]
+        return {"draft_sampler": {"kernel": "sample_drafts_kernel", "us": us, "achieved": gbs,
+                                  "unit": "GB/s", "peak": peak, "frac": gbs / peak,
+                                  "algorithmic_bytes": nbytes,
+                                  "rows": f"{self.B}x{self.K} rows of {self.V}"}}
+
     def make_events(self):
         n = len(self.layers)
         mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -353,6 +376,9 @@ class SingleSequence(BatchedDecode):
                          workspace=self.vws)
         if ev is not None:
             ev[3].record()
+
+    def extra_measurements(self, stream, reps=20):
+        return {}
 
     def host_inputs(self):
         _, x, *_ = self.layers[0]
@@ -542,6 +568,7 @@ def run_ours(args):
     gemm_ms = [wl.op_times(e)[0] for e in events]
     ver_ms = [wl.op_times(e)[1] for e in events]
     faults = api.device_fault_flags(clear=True)
+    extra = wl.extra_measurements(stream) if hasattr(wl, "extra_measurements") else {}
 
     rows_per_step = wl.B * wl.K
     value = whole_job_rate(rows_per_step, world, ms_step)
@@ -605,6 +632,7 @@ def run_ours(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "device_fault_flags": faults,
+            **extra,
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload)

@@ -26,7 +26,8 @@
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;     // 8 CTAs per SM: a 64 x 16 block of rows is one wave
+constexpr int kCtasPerSm = 8;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxChunks = 2048;  // chunk table in shared memory (16 KB)
 constexpr int kInFlight = 4;      // chunks a warp loads before reducing them
@@ -122,7 +123,7 @@ __device__ __forceinline__ float l2(const T* row, long long v) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) sample_drafts_kernel(const SampleParams P) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(const SampleParams P) {
   __shared__ Shared sh;
   uno::launch_dependents();
   uno::grid_dependency_wait();
@@ -135,53 +136,65 @@ __global__ void __launch_bounds__(kThreads) sample_drafts_kernel(const SamplePar
   const int V = P.V, L = P.chunk_len;
 
   // ---- pass 1: per-chunk (max, sum of 2^(x - max)) ----
+  // Each step a warp issues one 16-byte load per lane for kInFlight chunks
+  // before it reduces any of them. Every lane keeps its own reference (its
+  // running maximum, raised only when a larger value arrives) and sum; the
+  // warp combines them once per chunk.
   for (int c0 = warp; c0 < P.nchunks; c0 += kWarps * kInFlight) {
-    float cmax[kInFlight], csum[kInFlight];
+    float lm[kInFlight], ls[kInFlight];
 #pragma unroll
     for (int k = 0; k < kInFlight; ++k) {
-      cmax[k] = -INFINITY;
-      csum[k] = 0.f;
+      lm[k] = -INFINITY;
+      ls[k] = 0.f;
     }
     // a chunk is L / (32 kVec) steps of one vector per lane
     for (int s = 0; s < L; s += 32 * kVec) {
-      float f[kInFlight][kVec];
+      uint4 raw[kInFlight];
 #pragma unroll
       for (int k = 0; k < kInFlight; ++k) {
         const int c = c0 + k * kWarps;
         const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
-        if (c < P.nchunks && vec && v0 + kVec <= V) {
-          Row<T>::unpack(__ldg(reinterpret_cast<const uint4*>(row + v0)), f[k]);
-#pragma unroll
-          for (int e = 0; e < kVec; ++e) f[k][e] *= kLog2e;
-        } else {
-#pragma unroll
-          for (int e = 0; e < kVec; ++e)
-            f[k][e] = (c < P.nchunks && v0 + e < V) ? l2(row, v0 + e) : -INFINITY;
-        }
+        raw[k] = (c < P.nchunks && vec && v0 + kVec <= V)
+                     ? __ldg(reinterpret_cast<const uint4*>(row + v0))
+                     : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int k = 0; k < kInFlight; ++k) {
-        float m = cmax[k];
+        const int c = c0 + k * kWarps;
+        const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
+        float f[kVec];
+        if (c < P.nchunks && vec && v0 + kVec <= V) {
+          Row<T>::unpack(raw[k], f);
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) m = fmaxf(m, f[k][e]);
-        m = warp_max(m);  // the chunk's running maximum, same in every lane
-        if (m > -INFINITY) {
-          csum[k] *= uno::ex2(cmax[k] - m);  // rescale what came before
+          for (int e = 0; e < kVec; ++e) f[e] *= kLog2e;
+        } else {
+#pragma unroll
+          for (int e = 0; e < kVec; ++e)
+            f[e] = (c < P.nchunks && v0 + e < V) ? l2(row, v0 + e) : -INFINITY;
+        }
+        float mk = f[0];
+#pragma unroll
+        for (int e = 1; e < kVec; ++e) mk = fmaxf(mk, f[e]);
+        if (mk > lm[k]) {  // a larger value: move the reference up
+          ls[k] *= uno::ex2(lm[k] - mk);
+          lm[k] = mk;
+        }
+        if (lm[k] > -INFINITY) {
           float add = 0.f;
 #pragma unroll
-          for (int e = 0; e < kVec; ++e) add += uno::ex2(f[k][e] - m);
-          csum[k] += add;
-          cmax[k] = m;
+          for (int e = 0; e < kVec; ++e) add += uno::ex2(f[e] - lm[k]);
+          ls[k] += add;
         }
       }
     }
 #pragma unroll
     for (int k = 0; k < kInFlight; ++k) {
       const int c = c0 + k * kWarps;
-      const float t = warp_sum(csum[k]);
+      const float m = warp_max(lm[k]);
+      const float t = warp_sum((lm[k] > -INFINITY) ? ls[k] * uno::ex2(lm[k] - m) : 0.f);
       if (lane == 0 && c < P.nchunks) {
-        sh.cm[c] = cmax[k];
-        sh.cs[c] = (cmax[k] > -INFINITY) ? t : 0.f;
+        sh.cm[c] = m;
+        sh.cs[c] = (m > -INFINITY) ? t : 0.f;
       }
     }
   }
