@@ -22,3 +22,13 @@ from .uno_oracle import (  # noqa: F401
     verify_block_u,
     word_to_uniform,
 )
+from .tree_sampler import (  # noqa: F401,E402
+    tree_build,
+    tree_candidates,
+    tree_draft,
+    tree_max_nodes,
+    tree_topk,
+    tree_uniforms,
+    tree_verify,
+    tree_verify_u,
+)
