@@ -10,11 +10,15 @@
 // resampling draw independent uniforms from one stream.
 //
 // One CTA per row (b, i), one pass over the row in HBM: each warp takes
-// chunks of the row (one 16-byte vector per lane per step), reduces each chunk
-// to (chunk max, sum of 2^(x - chunk max)) in the log2 domain and keeps it in
-// shared memory. The CTA then rescales the chunk sums to the row maximum,
-// takes their float64 running sum, finds the chunk where u * total is crossed
-// and scans only that chunk (in L2 by then) for the token.
+// chunks of the row (at least kMinSteps 16-byte vectors per lane, so the warp
+// reduction is paid once per several vectors), reduces each chunk to (chunk
+// max, sum of 2^(x - chunk max)) in the log2 domain and keeps it in shared
+// memory. The CTA then rescales the chunk sums to the row maximum, takes their
+// float64 running sum, finds the chunk where u * total is crossed and scans
+// only that chunk (in L2 by then): each thread sums a contiguous segment, one
+// block scan places the segments, and the thread whose segment crosses finds
+// the token.
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 
@@ -31,6 +35,7 @@ constexpr int kCtasPerSm = 8;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxChunks = 2048;  // chunk table in shared memory (16 KB)
 constexpr int kInFlight = 4;      // chunks a warp loads before reducing them
+constexpr int kMinSteps = 8;      // vectors per lane in a chunk, at least
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <typename T>
@@ -65,12 +70,15 @@ struct Row<float> {
 };
 
 struct SampleParams {
-  const void* q;       // [B][K][V]
-  int B, K, V;
-  int chunk_len;       // elements per chunk (a multiple of 32 * kVec)
+  const void* q;       // [B][rows][V]
+  int B, rows, V;      // rows: rows per sequence
+  int chunk_len;       // elements per chunk (a multiple of 32 * kVec and of kThreads)
   int nchunks;
+  const int32_t* row_key;  // [B][rows] Philox position of each row (null: the row index)
+  const int32_t* n_rows;   // [B] rows in use per sequence (null: all)
+  int word;                // Philox output word of the uniform (1 or 2)
   uint64_t seed, step;
-  int32_t* out;        // [B][K]
+  int32_t* out;        // [B][rows]
 };
 
 struct Shared {
@@ -116,10 +124,10 @@ __device__ double block_exclusive_scan(double mine, Shared& sh, double* total) {
   return before + incl - mine;
 }
 
-// Element v of the row, in the log2 domain (-inf stays -inf).
-template <typename T>
-__device__ __forceinline__ float l2(const T* row, long long v) {
-  return Row<T>::at(row, v) * kLog2e;
+// 2^(x log2 e - ref) for a logit x and a reference in the log2 domain
+// (x = -inf gives 0).
+__device__ __forceinline__ float w2(float x, float ref) {
+  return uno::ex2(fmaf(x, kLog2e, -ref));
 }
 
 template <typename T>
@@ -129,8 +137,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
   uno::grid_dependency_wait();
   constexpr int kVec = Row<T>::kVec;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bi = blockIdx.x;  // b * K + i
-  const int b = bi / P.K, i = bi - b * P.K;
+  const int bi = blockIdx.x;  // b * rows + n
+  if (P.n_rows != nullptr && bi % P.rows >= P.n_rows[bi / P.rows]) {
+    if (tid == 0) P.out[bi] = -1;  // a row not in use: the whole CTA leaves
+    return;
+  }
   const T* row = static_cast<const T*>(P.q) + static_cast<size_t>(bi) * P.V;
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   const int V = P.V, L = P.chunk_len;
@@ -162,19 +173,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
       for (int k = 0; k < kInFlight; ++k) {
         const int c = c0 + k * kWarps;
         const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
-        float f[kVec];
+        float f[kVec];  // logits as read (natural log domain)
         if (c < P.nchunks && vec && v0 + kVec <= V) {
           Row<T>::unpack(raw[k], f);
-#pragma unroll
-          for (int e = 0; e < kVec; ++e) f[e] *= kLog2e;
         } else {
 #pragma unroll
           for (int e = 0; e < kVec; ++e)
-            f[e] = (c < P.nchunks && v0 + e < V) ? l2(row, v0 + e) : -INFINITY;
+            f[e] = (c < P.nchunks && v0 + e < V) ? Row<T>::at(row, v0 + e) : -INFINITY;
         }
         float mk = f[0];
 #pragma unroll
         for (int e = 1; e < kVec; ++e) mk = fmaxf(mk, f[e]);
+        mk *= kLog2e;
         if (mk > lm[k]) {  // a larger value: move the reference up
           ls[k] *= uno::ex2(lm[k] - mk);
           lm[k] = mk;
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
         if (lm[k] > -INFINITY) {
           float add = 0.f;
 #pragma unroll
-          for (int e = 0; e < kVec; ++e) add += uno::ex2(f[e] - lm[k]);
+          for (int e = 0; e < kVec; ++e) add += w2(f[e], lm[k]);
           ls[k] += add;
         }
       }
@@ -217,7 +227,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
     if (tid == 0) P.out[bi] = -1;
     return;
   }
-  const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, i).z);
+  const int b = bi / P.rows;
+  const int i = (P.row_key != nullptr) ? P.row_key[bi] : bi - b * P.rows;
+  const uint4 words = uno::verify_block_words(P.seed, P.step, b, static_cast<uint32_t>(i));
+  const float u = uno::uniform24(P.word == 1 ? words.y : words.z);
   // thread t owns chunks [t * per, (t + 1) * per)
   const int per = (P.nchunks + kThreads - 1) / kThreads;
   const int c_lo = tid * per, c_hi = min(c_lo + per, P.nchunks);
@@ -257,21 +270,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
   if (tid == 0) sh.last_pos = -1;
   __syncthreads();
 
-  // ---- scan the chosen chunk (whole CTA, kThreads elements per step) ----
+  // ---- scan the chosen chunk: thread t sums the contiguous segment
+  // [v_lo + t seg, v_lo + (t + 1) seg), a block scan places the segments, and
+  // the segment where the running sum crosses u * total holds the token ----
   const long long v_lo = static_cast<long long>(ch) * L;
   const long long v_hi = min(v_lo + L, static_cast<long long>(V));
-  for (long long base = v_lo; base < v_hi; base += kThreads) {
-    const long long v = base + tid;
-    const float w = (v < v_hi) ? uno::ex2(l2(row, v) - M) : 0.f;
-    double step_total = 0.0;
-    const double bef = carry + block_exclusive_scan(static_cast<double>(w), sh, &step_total);
-    if (crossed && w > 0.f && bef + static_cast<double>(w) > t)
-      atomicMin(&sh.token, static_cast<int>(v));
-    if (w > 0.f) atomicMax(&sh.last_pos, static_cast<int>(v));
-    carry += step_total;
-    __syncthreads();
-    if (sh.token != INT_MAX) break;
+  const int seg = L / kThreads;
+  const long long s_lo = min(v_lo + static_cast<long long>(tid) * seg, v_hi);
+  const long long s_hi = min(s_lo + seg, v_hi);
+  double seg_sum = 0.0;
+  int seg_last = -1;
+  for (long long v = s_lo; v < s_hi; ++v) {
+    const float w = w2(Row<T>::at(row, v), M);
+    seg_sum += static_cast<double>(w);
+    if (w > 0.f) seg_last = static_cast<int>(v);
   }
+  double chunk_total = 0.0;
+  double run = carry + block_exclusive_scan(seg_sum, sh, &chunk_total);
+  if (seg_last >= 0) atomicMax(&sh.last_pos, seg_last);
+  if (crossed && seg_sum > 0.0 && run + seg_sum > t) {
+    for (long long v = s_lo; v < s_hi; ++v) {
+      const float w = w2(Row<T>::at(row, v), M);
+      if (w > 0.f && run + static_cast<double>(w) > t) {
+        atomicMin(&sh.token, static_cast<int>(v));
+        break;
+      }
+      run += static_cast<double>(w);
+    }
+  }
+  __syncthreads();
   if (tid == 0) P.out[bi] = (sh.token != INT_MAX) ? sh.token : sh.last_pos;
 }
 
@@ -281,23 +308,27 @@ bool sample_sizes_ok(int B, int K, int V, int dtype) {
 }
 
 template <typename T>
-int run(const void* q, int B, int K, int V, uint64_t seed, uint64_t step, int32_t* out,
-        cudaStream_t st) {
+int run(const uno_host::RowDraws& r, cudaStream_t st) {
   constexpr int kStep = 32 * Row<T>::kVec;  // elements per vector step of a warp
+  const int V = r.V;
   SampleParams P{};
-  P.q = q;
-  P.B = B;
-  P.K = K;
+  P.q = r.logits;
+  P.B = r.B;
+  P.rows = r.rows_per_seq;
   P.V = V;
-  P.seed = seed;
-  P.step = step;
-  P.out = out;
+  P.row_key = r.row_key;
+  P.n_rows = r.n_rows;
+  P.word = r.word;
+  P.seed = r.seed;
+  P.step = r.step;
+  P.out = r.out;
   const long long steps = (static_cast<long long>(V) + kStep - 1) / kStep;
-  const long long per_chunk = (steps + kMaxChunks - 1) / kMaxChunks;  // steps per chunk
+  const long long per_chunk =
+      std::max<long long>(kMinSteps, (steps + kMaxChunks - 1) / kMaxChunks);  // steps per chunk
   P.chunk_len = static_cast<int>(per_chunk * kStep);
   P.nchunks = static_cast<int>((V + P.chunk_len - 1) / P.chunk_len);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(B * K));
+  cfg.gridDim = dim3(static_cast<unsigned>(r.B * r.rows_per_seq));
   cfg.blockDim = dim3(kThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -311,6 +342,11 @@ int run(const void* q, int B, int K, int V, uint64_t seed, uint64_t step, int32_
 
 }  // namespace
 
+int uno_host::sample_rows(const RowDraws& r, cudaStream_t st) {
+  if (r.B == 0 || r.rows_per_seq == 0) return UNO_OK;
+  return (r.dtype == UNO_BF16) ? run<uint16_t>(r, st) : run<float>(r, st);
+}
+
 extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype,
                                  uint64_t seed, uint64_t step, int32_t* draft_tokens,
                                  void* stream) {
@@ -323,7 +359,15 @@ extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int 
     return UNO_ERR_ALIGN;
   const int dev = uno_host::check_device();
   if (dev != UNO_OK) return dev;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == UNO_BF16) return run<uint16_t>(q_logits, B, K, V, seed, step, draft_tokens, st);
-  return run<float>(q_logits, B, K, V, seed, step, draft_tokens, st);
+  uno_host::RowDraws r{};
+  r.logits = q_logits;
+  r.B = B;
+  r.rows_per_seq = K;
+  r.V = V;
+  r.dtype = dtype;
+  r.word = 2;  // drafting: word 2 of the (b, i, step) block
+  r.seed = seed;
+  r.step = step;
+  r.out = draft_tokens;
+  return uno_host::sample_rows(r, static_cast<cudaStream_t>(stream));
 }

@@ -67,6 +67,7 @@ constexpr int kProducers = 2;
 constexpr int kGemmThreads = (kFirstProducer + kProducers) * 32;
 constexpr int kInsert = 6;         // main K-blocks of the next tile before an adapter
 constexpr int kPrefetch = 8;       // K-blocks of L2 prefetch ahead of the weight loads
+constexpr int kMaxSplit = 4;       // K-pieces of a split tile, at most
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum : unsigned { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
@@ -935,21 +936,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
           break;
         }
+        // every piece's loads of a 32-column chunk are issued before any is
+        // used (up to 24 x 16 bytes in flight per thread: one L2 round trip
+        // per chunk, not one per chunk and piece)
         for (int c = 0; c < BN; c += 32) {
+          float4 f[kMaxSplit - 1][8];
+#pragma unroll
+          for (int q = 1; q < kMaxSplit; ++q)
+            if (q < p.split_k) {
+              const float* src = slot(q) + c;
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                f[q - 1][e] = __ldcg(reinterpret_cast<const float4*>(src + 4 * e));
+            }
           uint32_t v[32];
           sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
           sm100::tmem_ld_wait();
-          for (int q = 1; q < p.split_k; ++q) {
-            const float* src = slot(q) + c;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 f = __ldcg(reinterpret_cast<const float4*>(src + e));
-              v[e] = __float_as_uint(__uint_as_float(v[e]) + f.x);
-              v[e + 1] = __float_as_uint(__uint_as_float(v[e + 1]) + f.y);
-              v[e + 2] = __float_as_uint(__uint_as_float(v[e + 2]) + f.z);
-              v[e + 3] = __float_as_uint(__uint_as_float(v[e + 3]) + f.w);
+          for (int q = 1; q < kMaxSplit; ++q)
+            if (q < p.split_k) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                v[4 * e] = __float_as_uint(__uint_as_float(v[4 * e]) + f[q - 1][e].x);
+                v[4 * e + 1] = __float_as_uint(__uint_as_float(v[4 * e + 1]) + f[q - 1][e].y);
+                v[4 * e + 2] = __float_as_uint(__uint_as_float(v[4 * e + 2]) + f[q - 1][e].z);
+                v[4 * e + 3] = __float_as_uint(__uint_as_float(v[4 * e + 3]) + f[q - 1][e].w);
+              }
             }
-          }
           sm100::tmem_st_32x32b_x32(acc + lq + c, v);
         }
         sm100::tmem_st_wait();
@@ -1130,7 +1143,7 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
   long long tiles = units0;
   if (units0 > resident) {
     const long long rem = units0 % resident;
-    int k = rem > 0 ? static_cast<int>(std::min<long long>(4, resident / rem)) : 1;
+    int k = rem > 0 ? static_cast<int>(std::min<long long>(kMaxSplit, resident / rem)) : 1;
     while (k > 1 && p.kb_total < 2 * k) --k;
     const size_t per_slot = static_cast<size_t>(PAIR ? 2 : 1) * kBM * BN * sizeof(float);
     const size_t slots = static_cast<size_t>(rem) * (k - 1);

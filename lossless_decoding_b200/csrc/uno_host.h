@@ -17,4 +17,20 @@ inline bool aligned(const void* p, uintptr_t a) {
 // answer is cached per device ordinal.
 int check_device();
 
+// One inverse-CDF draw per softmax row (draft_sample.cu): row n of sequence b
+// (logits + ((b * rows_per_seq + n) * V)) draws with the uniform of Philox
+// word `word` of the block (b, row_key[b][n] or n, step); rows with
+// n >= n_rows[b] are skipped and get -1 (n_rows null: all rows are used); a
+// row with no finite logit gets -1. Arguments are checked by the caller.
+struct RowDraws {
+  const void* logits;
+  int B, rows_per_seq, V, dtype;
+  const int32_t* row_key;
+  const int32_t* n_rows;
+  int word;
+  uint64_t seed, step;
+  int32_t* out;
+};
+int sample_rows(const RowDraws& r, cudaStream_t st);
+
 }  // namespace uno_host
