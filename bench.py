@@ -65,7 +65,9 @@ def _peaks():
 # profiles/. A figure is reported only while the kernel source it was taken on
 # is unchanged (first 16 hex digits of its sha256), else traffic is null.
 MEASURED_TRAFFIC = {
-    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "dfe88fefbff16324", 136.6e6),
+    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "86fe45781388d7ef", 137.6e6),
+    # sample_drafts_kernel over the 64 x 16 q rows: 314.9 MB read + 5.3 MB written
+    ("batched_decode_b64_k16", "draft"): ("draft_sample.cu", "9369b9644cfaf3fe", 320.2e6),
     # stream 646.5 MB + decide 0.3 MB + draw 39.1 MB, per verifier call
     ("batched_decode_b64_k16", "verify"): ("verify.cu", "d55361a025a1b14b", 685.9e6),
 }
@@ -284,6 +286,7 @@ class BatchedDecode:
         return {"draft_sampler": {"kernel": "sample_drafts_kernel", "us": us, "achieved": gbs,
                                   "unit": "GB/s", "peak": peak, "frac": gbs / peak,
                                   "algorithmic_bytes": nbytes,
+                                  "traffic": measured_traffic(self.name, "draft"),
                                   "rows": f"{self.B}x{self.K} rows of {self.V}"}}
 
     def make_events(self):
@@ -332,6 +335,69 @@ class BatchedDecode:
                 "lora_rank": RANK, "lora_alpha": ALPHA, "logits": "bf16",
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e9:.2f} GB distinct per step",
                 "global_batch": self.B, "parallelism": "replicas (one batch per GPU)"}
+
+
+def tree_measure(api, stream, B, D, top_k, budget, V, reps=20, sets=4):
+    """Time tree_draft (top-k + tree build) and tree_verify (node draws + walk)
+    on the device: `sets` calls of each are captured in a CUDA graph (host
+    overhead of the Python binding left out) and the graph is replayed `reps`
+    times between CUDA events. The `sets` copies of the logits rotate so that
+    the reads come from HBM (more than L2 in total)."""
+    from lossless_decoding_b200.inputs import verify_inputs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    N = api.tree_nodes(D, budget)
+    qs = [verify_inputs(B, D, V, dtype="bf16", seed=50 + i, device=dev).q_logits
+          for i in range(sets)]
+    ps = [verify_inputs(B, N - 1, V, dtype="bf16", seed=60 + i, device=dev).p_logits
+          for i in range(sets)]
+    ws = torch.empty(api.tree_draft_workspace_bytes(B, D, V, top_k), dtype=torch.uint8,
+                     device=dev)
+    trees = [api.tree_draft(q, top_k, budget, workspace=ws) for q in qs]
+    outs = [api.tree_verify(ps[i], trees[i], 1, 0) for i in range(sets)]
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):  # warm-up on the capture's stream kind
+        for i in range(sets):
+            api.tree_draft(qs[i], top_k, budget, workspace=ws)
+            api.tree_verify(ps[i], trees[i], 1, i, out=outs[i])
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    g_draft, g_verify = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_draft):
+        for i in range(sets):
+            api.tree_draft(qs[i], top_k, budget, workspace=ws)
+    with torch.cuda.graph(g_verify):
+        for i in range(sets):
+            api.tree_verify(ps[i], trees[i], 1, i, out=outs[i])
+    g_draft.replay()
+    g_verify.replay()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(cur)
+    for _ in range(reps):
+        g_draft.replay()
+    ev[1].record(cur)
+    for _ in range(reps):
+        g_verify.replay()
+    ev[2].record(cur)
+    torch.cuda.synchronize()
+    us_d = ev[0].elapsed_time(ev[1]) * 1e3 / (reps * sets)
+    us_v = ev[1].elapsed_time(ev[2]) * 1e3 / (reps * sets)
+    rows = sum(int(t.n_nodes.sum()) for t in trees) / sets
+    bytes_d = B * D * V * 2
+    bytes_v = rows * V * 2
+    peak = _peaks()["hbm"]
+    del g_draft, g_verify
+    return {"config": {"B": B, "D": D, "top_k": top_k, "budget": budget, "V": V,
+                       "node_rows": N, "dtype": "bf16"},
+            "timing": "CUDA graph of the calls, replayed between CUDA events",
+            "draft_us": us_d, "draft_gbs": bytes_d / (us_d / 1e6) / 1e9,
+            "verify_us": us_v, "verify_gbs": bytes_v / (us_v / 1e6) / 1e9,
+            "verify_rows_in_use": rows, "peak_gbs": peak,
+            "kernels": "tree_topk_part_kernel + tree_topk_merge_kernel + tree_build_kernel; "
+                       "sample_drafts_kernel (node rows) + tree_walk_kernel"}
 
 
 class SingleSequence(BatchedDecode):
@@ -384,7 +450,11 @@ class SingleSequence(BatchedDecode):
             ev[3].record()
 
     def extra_measurements(self, stream, reps=20):
-        return {}
+        """The tree sampler at this workload's batch: a block of 16 (D = 15
+        positions after the AR-only first token), top-4 per position, the 16
+        best sequences kept (241 node rows)."""
+        return {"tree_sampler": tree_measure(self.api, stream, B=self.B, D=self.K - 1, top_k=4,
+                                             budget=16, V=self.V, reps=reps)}
 
     def host_inputs(self):
         _, x, *_ = self.layers[0]

@@ -246,6 +246,75 @@ int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype, uint
                       uint64_t step, int32_t* draft_tokens, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * Tree sampler
+ *
+ * Reader page, "The Psi-Speculative Sampler" (worked example with
+ * (B, K, V) = (3, 2, 2): the K^(B-1) candidate sequences of the positions
+ * after the block's first token are ranked by joint log-probability, the top V
+ * are kept, every prefix is verified by the frozen AR model and the longest
+ * valid one is accepted) and "Sampler Extensions"; summary page,
+ * "Psi-Speculative Sampler" (top-K at each position). The pages' (B, K, V)
+ * are depth D = B - 1, top_k and budget here.
+ *
+ * uno_tree_nodes(D, budget) = 1 + D * budget: the node rows N of a tree
+ * (root + one node per position of every kept sequence, at most); 0 when D
+ * or budget is out of range.
+ *
+ * uno_tree_draft:
+ *   q_logits     [B, D, V] dtype: draft logits of positions 1..D
+ *   topk_ids     [B, D, top_k] int32 out: per position the top_k ids by
+ *                logit, larger first, ties to the smaller id; -inf logits
+ *                are never candidates (-1 fills missing slots)
+ *   topk_logq    [B, D, top_k] f32 out: log softmax(q)(id) (-inf when -1)
+ *   node_token   [B, N] int32 out: token of each node (root, padding: -1)
+ *   node_parent  [B, N] int32 out: parent node (root, padding: -1)
+ *   node_depth   [B, N] int32 out: 0 root, j for a prefix of length j
+ *                (padding: -1)
+ *   n_nodes      [B] int32 out
+ *   workspace    device scratch of at least
+ *                uno_tree_draft_workspace_bytes(B, D, V, top_k) bytes,
+ *                256-byte aligned (each row's logits are split over several
+ *                CTAs at small B; their partial lists meet there); contents
+ *                on entry do not matter
+ *   The kept set is the budget best of the top_k^D sequences by the sum of
+ *   topk_logq over positions (float32, position order), ties by the
+ *   sequence of ranks (lexicographic, smaller first); the nodes are their
+ *   distinct prefixes, by depth, then by rank sequence.
+ *   Limits: 0 <= B <= 2^20, 1 <= D <= 16, 1 <= top_k <= 16,
+ *   1 <= budget <= 64, 1 <= V <= 2^28.
+ *
+ * uno_tree_verify: the lossless walk of each sequence's tree.
+ *   p_logits     [B, N, V] dtype: AR logits after each node's prefix (rows
+ *                n >= n_nodes[b] are not read)
+ *   node_*, n_nodes  the tree (as uno_tree_draft writes it)
+ *   node_draw    [B, N] int32 out: the draw of every node in use (-1 for
+ *                rows not in use and rows with no finite logit)
+ *   out_tokens   [B, D+1] int32 out: accepted tree tokens, then the token
+ *                drawn where the walk stopped; -1 padding
+ *   accepted_len [B] int32 out: accepted tree tokens (0..D), -1 when a row
+ *                on the walk has no finite logit (then all tokens are -1)
+ *   At node n (depth j) the draw is the inverse CDF of softmax(p[b][n]) at
+ *   the uniform of Philox word 1 of the block (b, j, step) under (seed); the
+ *   walk follows it while it is the token of a child of the current node and
+ *   emits it either way, so every emitted token is an exact draw of the AR
+ *   distribution given the tokens before it.
+ *
+ * uno_tree_verify takes no workspace. Both are asynchronous on `stream` and
+ * return UNO_OK or a negative uno_status (UNO_ERR_WORKSPACE for a missing,
+ * short or misaligned draft workspace).
+ * ------------------------------------------------------------------------ */
+int uno_tree_nodes(int depth, int budget);
+size_t uno_tree_draft_workspace_bytes(int B, int D, int V, int top_k);
+int uno_tree_draft(const void* q_logits, int B, int D, int V, int dtype, int top_k, int budget,
+                   int32_t* topk_ids, float* topk_logq, int32_t* node_token,
+                   int32_t* node_parent, int32_t* node_depth, int32_t* n_nodes, void* workspace,
+                   size_t workspace_bytes, void* stream);
+int uno_tree_verify(const void* p_logits, const int32_t* node_token, const int32_t* node_parent,
+                    const int32_t* node_depth, const int32_t* n_nodes, int B, int D, int budget,
+                    int V, int dtype, uint64_t seed, uint64_t step, int32_t* node_draw,
+                    int32_t* out_tokens, int32_t* accepted_len, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * Device fault flags
  *
  * Every wait inside the kernels is bounded in time. A wait that gives up

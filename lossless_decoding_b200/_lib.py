@@ -66,6 +66,16 @@ def _load() -> ctypes.CDLL:
     L.uno_dualpath_linear_grouped.restype = i32
     L.uno_sample_drafts.argtypes = [vp, i32, i32, i32, i32, u64, u64, vp, vp]
     L.uno_sample_drafts.restype = i32
+    L.uno_tree_nodes.argtypes = [i32, i32]
+    L.uno_tree_nodes.restype = i32
+    L.uno_tree_draft_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.uno_tree_draft_workspace_bytes.restype = sz
+    L.uno_tree_draft.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                 sz, vp]
+    L.uno_tree_draft.restype = i32
+    L.uno_tree_verify.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, u64, u64, vp, vp,
+                                  vp, vp]
+    L.uno_tree_verify.restype = i32
     L.uno_device_fault_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint)]
     L.uno_device_fault_flags.restype = i32
     return L

@@ -318,6 +318,108 @@ def sample_drafts(q_logits: torch.Tensor, seed: int, step: int, *,
     return out
 
 
+# ---------------------------------------------------------------------------
+# tree sampler
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class DraftTree:
+    """A candidate tree per sequence (as ``uno_tree_draft`` writes it)."""
+
+    topk_ids: torch.Tensor     # [B, D, top_k] int32
+    topk_logq: torch.Tensor    # [B, D, top_k] float32
+    node_token: torch.Tensor   # [B, N] int32
+    node_parent: torch.Tensor  # [B, N] int32
+    node_depth: torch.Tensor   # [B, N] int32
+    n_nodes: torch.Tensor      # [B] int32
+    budget: int
+
+
+def tree_nodes(depth: int, budget: int) -> int:
+    """Node rows N of a tree of `depth` positions and `budget` kept sequences."""
+    n = lib.uno_tree_nodes(depth, budget)
+    if n <= 0:
+        raise ValueError("depth must be in [1, 16] and budget in [1, 64]")
+    return n
+
+
+def tree_draft_workspace_bytes(B: int, D: int, V: int, top_k: int) -> int:
+    return int(lib.uno_tree_draft_workspace_bytes(B, D, V, top_k))
+
+
+def tree_draft(q_logits: torch.Tensor, top_k: int, budget: int, *,
+               workspace: Optional[torch.Tensor] = None) -> DraftTree:
+    """Top-k candidates of each position and the tree of the `budget` best
+    sequences by joint log-probability. q_logits [B, D, V] bf16/f32."""
+    if q_logits.dim() != 3:
+        raise ValueError("q_logits must be [B, D, V]")
+    B, D, V = q_logits.shape
+    dt = _dtype_code(q_logits)
+    dev = _check_cuda(q_logits)
+    N = tree_nodes(D, budget)
+    i32 = dict(dtype=torch.int32, device=dev)
+    t = DraftTree(torch.empty((B, D, top_k), **i32),
+                  torch.empty((B, D, top_k), dtype=torch.float32, device=dev),
+                  torch.empty((B, N), **i32), torch.empty((B, N), **i32),
+                  torch.empty((B, N), **i32), torch.empty((B,), **i32), budget)
+    need = lib.uno_tree_draft_workspace_bytes(B, D, V, top_k)
+    if need == 0:
+        raise ValueError("sizes out of range for the tree sampler")
+    if workspace is None:
+        workspace = _ws.get(dev, "tree_draft", need)
+    if workspace.dtype != torch.uint8 or workspace.numel() < need:
+        raise ValueError(f"workspace must be uint8 with at least {need} bytes")
+    _check_cuda(workspace)
+    st = lib.uno_tree_draft(_ptr(q_logits), B, D, V, dt, top_k, budget, _ptr(t.topk_ids),
+                            _ptr(t.topk_logq), _ptr(t.node_token), _ptr(t.node_parent),
+                            _ptr(t.node_depth), _ptr(t.n_nodes), _ptr(workspace), need,
+                            _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_tree_draft")
+    return t
+
+
+@dataclass
+class TreeResult:
+    out_tokens: torch.Tensor    # [B, D+1] int32
+    accepted_len: torch.Tensor  # [B] int32
+    node_draw: torch.Tensor     # [B, N] int32
+
+
+def tree_verify(p_logits: torch.Tensor, tree: DraftTree, seed: int, step: int, *,
+                out: Optional[TreeResult] = None) -> TreeResult:
+    """The lossless walk of each tree with the AR rows p_logits [B, N, V]."""
+    if p_logits.dim() != 3:
+        raise ValueError("p_logits must be [B, N, V]")
+    B, N, V = p_logits.shape
+    D = tree.topk_ids.shape[1]
+    if N != tree_nodes(D, tree.budget) or tuple(tree.node_token.shape) != (B, N):
+        raise ValueError("p_logits must have one row per node slot of the tree")
+    dt = _dtype_code(p_logits)
+    dev = _check_cuda(p_logits, tree.node_token, tree.node_parent, tree.node_depth,
+                      tree.n_nodes)
+    for x in (tree.node_token, tree.node_parent, tree.node_depth, tree.n_nodes):
+        if x.dtype != torch.int32:
+            raise ValueError("tree arrays must be int32")
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = TreeResult(torch.empty((B, D + 1), **i32), torch.empty((B,), **i32),
+                         torch.empty((B, N), **i32))
+    _check_cuda(out.out_tokens, out.accepted_len, out.node_draw)
+    if (tuple(out.out_tokens.shape) != (B, D + 1) or tuple(out.accepted_len.shape) != (B,)
+            or tuple(out.node_draw.shape) != (B, N)):
+        raise ValueError("out tensors have the wrong shapes")
+    st = lib.uno_tree_verify(_ptr(p_logits), _ptr(tree.node_token), _ptr(tree.node_parent),
+                             _ptr(tree.node_depth), _ptr(tree.n_nodes), B, D, tree.budget, V, dt,
+                             ctypes.c_uint64(seed & (2**64 - 1)),
+                             ctypes.c_uint64(step & (2**64 - 1)), _ptr(out.node_draw),
+                             _ptr(out.out_tokens), _ptr(out.accepted_len), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_tree_verify")
+    return out
+
+
 def device_fault_flags(clear: bool = True) -> int:
     """Fault bits set by a kernel wait that gave up (0 = none). Synchronises."""
     flags = ctypes.c_uint(0)

@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG_DIR, "libuno.so")
 
-SOURCES = ["status.cu", "verify.cu", "verify_noalloc.cu", "dualpath.cu", "draft_sample.cu"]
+SOURCES = ["status.cu", "verify.cu", "verify_noalloc.cu", "dualpath.cu", "draft_sample.cu",
+           "tree_sampler.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          f"-I{INCLUDE}"]

@@ -30,44 +30,24 @@
 
 namespace {
 
-constexpr int kThreads = 128;     // 8 CTAs per SM: a 64 x 16 block of rows is one wave
-constexpr int kCtasPerSm = 8;
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxChunks = 2048;  // chunk table in shared memory (16 KB)
-constexpr int kInFlight = 4;      // chunks a warp loads before reducing them
 constexpr int kMinSteps = 8;      // vectors per lane in a chunk, at least
+
+// Launch shapes. Many rows (a 64 x 16 block of drafts): 128-thread CTAs, 8 per
+// SM, one wave. Few rows (a tree's node rows at batch 1): 512-thread CTAs, so
+// that a handful of rows still keeps enough loads in flight. Four chunks in
+// flight per warp either way (more spill registers).
+template <int THREADS, int IN_FLIGHT, int CTAS_PER_SM>
+struct Shape {
+  static constexpr int kThreads = THREADS;
+  static constexpr int kWarps = THREADS / 32;
+  static constexpr int kInFlight = IN_FLIGHT;  // chunks a warp loads before reducing them
+  static constexpr int kCtasPerSm = CTAS_PER_SM;
+};
+using Narrow = Shape<128, 4, 8>;
+using Wide = Shape<512, 4, 2>;
+constexpr int kWideRows = 2 * 148;  // at most this many rows: the wide shape
 constexpr float kLog2e = 1.4426950408889634f;
-
-template <typename T>
-struct Row;
-
-template <>
-struct Row<uint16_t> {  // bfloat16 bits
-  static constexpr int kVec = 8;
-  __device__ static __forceinline__ float at(const uint16_t* p, long long i) {
-    return uno::bf16_bits_to_float(__ldg(p + i));
-  }
-  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      f[2 * k] = __uint_as_float(w[k] << 16);
-      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-    }
-  }
-};
-
-template <>
-struct Row<float> {
-  static constexpr int kVec = 4;
-  __device__ static __forceinline__ float at(const float* p, long long i) { return __ldg(p + i); }
-  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
-    f[0] = __uint_as_float(v.x);
-    f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z);
-    f[3] = __uint_as_float(v.w);
-  }
-};
 
 struct SampleParams {
   const void* q;       // [B][rows][V]
@@ -81,6 +61,7 @@ struct SampleParams {
   int32_t* out;        // [B][rows]
 };
 
+template <int kWarps>
 struct Shared {
   float cm[kMaxChunks];  // chunk maximum (log2 domain), -inf when empty
   float cs[kMaxChunks];  // sum over the chunk of 2^(x log2 e - cm)
@@ -104,7 +85,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Exclusive running sum (float64, thread order) across the CTA; the total is
 // returned through *total.
-__device__ double block_exclusive_scan(double mine, Shared& sh, double* total) {
+template <int kWarps>
+__device__ double block_exclusive_scan(double mine, Shared<kWarps>& sh, double* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double incl = mine;
 #pragma unroll
@@ -130,12 +112,14 @@ __device__ __forceinline__ float w2(float x, float ref) {
   return uno::ex2(fmaf(x, kLog2e, -ref));
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(const SampleParams P) {
-  __shared__ Shared sh;
+template <typename T, typename S>
+__global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
+    sample_drafts_kernel(const SampleParams P) {
+  constexpr int kThreads = S::kThreads, kWarps = S::kWarps, kInFlight = S::kInFlight;
+  __shared__ Shared<kWarps> sh;
   uno::launch_dependents();
   uno::grid_dependency_wait();
-  constexpr int kVec = Row<T>::kVec;
+  constexpr int kVec = uno::LogitRow<T>::kVec;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bi = blockIdx.x;  // b * rows + n
   if (P.n_rows != nullptr && bi % P.rows >= P.n_rows[bi / P.rows]) {
@@ -175,11 +159,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
         const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
         float f[kVec];  // logits as read (natural log domain)
         if (c < P.nchunks && vec && v0 + kVec <= V) {
-          Row<T>::unpack(raw[k], f);
+          uno::LogitRow<T>::unpack(raw[k], f);
         } else {
 #pragma unroll
           for (int e = 0; e < kVec; ++e)
-            f[e] = (c < P.nchunks && v0 + e < V) ? Row<T>::at(row, v0 + e) : -INFINITY;
+            f[e] = (c < P.nchunks && v0 + e < V) ? uno::LogitRow<T>::at(row, v0 + e) : -INFINITY;
         }
         float mk = f[0];
 #pragma unroll
@@ -281,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
   double seg_sum = 0.0;
   int seg_last = -1;
   for (long long v = s_lo; v < s_hi; ++v) {
-    const float w = w2(Row<T>::at(row, v), M);
+    const float w = w2(uno::LogitRow<T>::at(row, v), M);
     seg_sum += static_cast<double>(w);
     if (w > 0.f) seg_last = static_cast<int>(v);
   }
@@ -290,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_drafts_kernel(con
   if (seg_last >= 0) atomicMax(&sh.last_pos, seg_last);
   if (crossed && seg_sum > 0.0 && run + seg_sum > t) {
     for (long long v = s_lo; v < s_hi; ++v) {
-      const float w = w2(Row<T>::at(row, v), M);
+      const float w = w2(uno::LogitRow<T>::at(row, v), M);
       if (w > 0.f && run + static_cast<double>(w) > t) {
         atomicMin(&sh.token, static_cast<int>(v));
         break;
@@ -307,9 +291,11 @@ bool sample_sizes_ok(int B, int K, int V, int dtype) {
          K <= 256 && V >= 1 && V <= (1 << 28) && static_cast<long long>(B) * K <= (1 << 28);
 }
 
-template <typename T>
+template <typename T, typename S>
 int run(const uno_host::RowDraws& r, cudaStream_t st) {
-  constexpr int kStep = 32 * Row<T>::kVec;  // elements per vector step of a warp
+  constexpr int kStep = 32 * uno::LogitRow<T>::kVec;  // elements per vector step of a warp
+  // a chunk is a whole number of warp steps and of CTA-wide segments
+  constexpr int kStepsMult = (S::kThreads > kStep) ? S::kThreads / kStep : 1;
   const int V = r.V;
   SampleParams P{};
   P.q = r.logits;
@@ -323,20 +309,22 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
   P.step = r.step;
   P.out = r.out;
   const long long steps = (static_cast<long long>(V) + kStep - 1) / kStep;
-  const long long per_chunk =
+  long long per_chunk =
       std::max<long long>(kMinSteps, (steps + kMaxChunks - 1) / kMaxChunks);  // steps per chunk
+  per_chunk = (per_chunk + kStepsMult - 1) / kStepsMult * kStepsMult;
   P.chunk_len = static_cast<int>(per_chunk * kStep);
   P.nchunks = static_cast<int>((V + P.chunk_len - 1) / P.chunk_len);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(r.B * r.rows_per_seq));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(S::kThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, sample_drafts_kernel<T>, P) != cudaSuccess) return UNO_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, sample_drafts_kernel<T, S>, P) != cudaSuccess)
+    return UNO_ERR_CUDA;
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
@@ -344,7 +332,9 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
 
 int uno_host::sample_rows(const RowDraws& r, cudaStream_t st) {
   if (r.B == 0 || r.rows_per_seq == 0) return UNO_OK;
-  return (r.dtype == UNO_BF16) ? run<uint16_t>(r, st) : run<float>(r, st);
+  if (static_cast<long long>(r.B) * r.rows_per_seq <= kWideRows)
+    return (r.dtype == UNO_BF16) ? run<uint16_t, Wide>(r, st) : run<float, Wide>(r, st);
+  return (r.dtype == UNO_BF16) ? run<uint16_t, Narrow>(r, st) : run<float, Narrow>(r, st);
 }
 
 extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype,

@@ -72,4 +72,37 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
   return static_cast<uint16_t>(u >> 16);
 }
 
+// A row of logits in memory: element reads and 16-byte vector unpacking for
+// bfloat16 (raw bits, 8 per vector) and float32 (4 per vector).
+template <typename T>
+struct LogitRow;
+
+template <>
+struct LogitRow<uint16_t> {
+  static constexpr int kVec = 8;
+  __device__ static __forceinline__ float at(const uint16_t* p, long long i) {
+    return bf16_bits_to_float(__ldg(p + i));
+  }
+  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <>
+struct LogitRow<float> {
+  static constexpr int kVec = 4;
+  __device__ static __forceinline__ float at(const float* p, long long i) { return __ldg(p + i); }
+  __device__ static __forceinline__ void unpack(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+};
+
 }  // namespace uno

@@ -57,6 +57,7 @@ T6. A node row on the walk with no finite logit marks the sequence invalid:
 
 from __future__ import annotations
 
+import heapq
 import itertools
 
 import numpy as np
@@ -83,30 +84,61 @@ def tree_topk(q_logits, top_k: int):
                 continue
             m = row[fin].max()
             lse = m + np.log(np.sum(np.exp(row[fin] - m)))
-            order = sorted(np.flatnonzero(fin), key=lambda v: (-row[v], v))
+            cand = np.flatnonzero(fin)
+            # sort by logit (larger first), then by id (smaller first)
+            order = cand[np.lexsort((cand, -row[cand]))]
             for s, v in enumerate(order[:top_k]):
                 ids[b, i, s] = v
                 logq[b, i, s] = row[v] - lse
     return ids, logq
 
 
-def tree_candidates(logq_b, budget: int):
+ENUMERATE_LIMIT = 200_000  # combinations enumerated outright, at most
+
+
+def tree_candidates(logq_b, budget: int, method: str = "auto"):
     """The kept sequences of one sequence's block (reading T3).
 
-    logq_b [D, top_k] (slots with -inf are absent). Enumerates every
-    combination of one candidate per position, ranks them by joint
-    log-probability (larger first; ties by rank tuple, smaller first) and
-    keeps ``budget``. Returns a list of (rank tuple, joint log-probability).
+    logq_b [D, top_k] (slots with -inf are absent). The pages' definition:
+    enumerate every combination of one candidate per position, rank them by
+    joint log-probability (larger first; ties by rank tuple, smaller first)
+    and keep ``budget`` ("enumerate"). When there are more than
+    ENUMERATE_LIMIT combinations (top_k^D grows fast) the same total order is
+    walked best first ("best_first"): the successors of a rank tuple raise one
+    coordinate at or after its last raised one, so every tuple has exactly one
+    predecessor, which precedes it in the order (the per-position lists are
+    sorted, so its score is not smaller, and on equal scores its tuple is
+    smaller). "auto" picks by the count. Returns a list of (rank tuple, joint
+    log-probability) in rank order.
     """
     logq_b = np.asarray(logq_b, dtype=np.float64)
     D, k = logq_b.shape
     per_pos = [[s for s in range(k) if np.isfinite(logq_b[i, s])] for i in range(D)]
-    combos = []
-    for tup in itertools.product(*per_pos):
-        score = float(sum(logq_b[i, s] for i, s in enumerate(tup)))
-        combos.append((tup, score))
-    combos.sort(key=lambda c: (-c[1], c[0]))
-    return combos[:budget]
+
+    def score(tup):
+        return float(sum(logq_b[i, s] for i, s in enumerate(tup)))
+
+    count = int(np.prod([len(c) for c in per_pos], dtype=np.float64))
+    if method == "auto":
+        method = "enumerate" if count <= ENUMERATE_LIMIT else "best_first"
+    if method == "enumerate":
+        combos = [(tup, score(tup)) for tup in itertools.product(*per_pos)]
+        combos.sort(key=lambda c: (-c[1], c[0]))
+        return combos[:budget]
+    if count == 0:
+        return []
+    avail = [len(c) for c in per_pos]  # finite slots come first in each row
+    start = (0,) * D
+    heap = [(-score(start), start, 0)]
+    out = []
+    while heap and len(out) < budget:
+        neg, tup, last = heapq.heappop(heap)
+        out.append((tup, -neg))
+        for j in range(last, D):
+            if tup[j] + 1 < avail[j]:
+                nxt = tup[:j] + (tup[j] + 1,) + tup[j + 1:]
+                heapq.heappush(heap, (-score(nxt), nxt, j))
+    return out
 
 
 def tree_max_nodes(depth: int, budget: int) -> int:

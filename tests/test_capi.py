@@ -143,3 +143,54 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(4, 8)
     with pytest.raises(ValueError):
         api.dualpath_linear(x, torch.zeros(8, 8), torch.zeros(8, 8), torch.zeros(8, 8), 1.0)
+
+
+def test_tree_argument_errors_need_no_gpu(lib):
+    from lossless_decoding_b200._lib import STATUS
+    fake = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4096 + 2)
+    u64 = ctypes.c_uint64
+    assert lib.uno_tree_nodes(15, 16) == 1 + 15 * 16
+    assert lib.uno_tree_nodes(0, 4) == 0 and lib.uno_tree_nodes(17, 4) == 0
+    assert lib.uno_tree_nodes(4, 0) == 0 and lib.uno_tree_nodes(4, 65) == 0
+    draft = lib.uno_tree_draft
+    need = lib.uno_tree_draft_workspace_bytes(2, 15, 1000, 4)
+    assert need > 0 and lib.uno_tree_draft_workspace_bytes(2, 17, 1000, 4) == 0
+    assert lib.uno_tree_draft_workspace_bytes(2, 15, 1000, 17) == 0
+    # small batches split each row over more CTAs: more partial lists
+    assert lib.uno_tree_draft_workspace_bytes(1, 15, 151936, 4) > 15 * 4 * 8
+    ok = (fake, 2, 15, 1000, 0, 4, 16, fake, fake, fake, fake, fake, fake, fake, need, None)
+
+    def d(**kw):
+        args = list(ok)
+        for i, name in enumerate(("q", "B", "D", "V", "dtype", "top_k", "budget", "ids", "logq",
+                                  "tok", "par", "dep", "n", "ws", "ws_bytes")):
+            if name in kw:
+                args[i] = kw[name]
+        return STATUS[draft(*args)]
+
+    assert d(dtype=3) == "UNO_ERR_DTYPE"
+    assert d(D=0) == "UNO_ERR_SIZE" and d(D=17) == "UNO_ERR_SIZE"
+    assert d(top_k=0) == "UNO_ERR_SIZE" and d(top_k=17) == "UNO_ERR_SIZE"
+    assert d(budget=0) == "UNO_ERR_SIZE" and d(budget=65) == "UNO_ERR_SIZE"
+    assert d(V=0) == "UNO_ERR_SIZE" and d(B=-1) == "UNO_ERR_SIZE"
+    assert d(q=None) == "UNO_ERR_NULL" and d(n=None) == "UNO_ERR_NULL"
+    odd1 = ctypes.c_void_p(4096 + 1)
+    assert d(q=odd1) == "UNO_ERR_ALIGN" and d(logq=odd) == "UNO_ERR_ALIGN"
+    assert d(ws=None) == "UNO_ERR_WORKSPACE" and d(ws_bytes=need - 1) == "UNO_ERR_WORKSPACE"
+    assert d(ws=ctypes.c_void_p(4096 + 128)) == "UNO_ERR_WORKSPACE"  # not 256-byte aligned
+    assert d(B=0, q=None, ids=None) == "UNO_OK"
+    ver = lib.uno_tree_verify
+    good = [fake, fake, fake, fake, fake, 2, 15, 16, 1000, 0, u64(0), u64(0), fake, fake, fake,
+            None]
+
+    def v(i, val):
+        args = list(good)
+        args[i] = val
+        return STATUS[ver(*args)]
+
+    assert v(9, 4) == "UNO_ERR_DTYPE"
+    assert v(6, 0) == "UNO_ERR_SIZE" and v(7, 65) == "UNO_ERR_SIZE" and v(8, 0) == "UNO_ERR_SIZE"
+    assert v(0, None) == "UNO_ERR_NULL" and v(12, None) == "UNO_ERR_NULL"
+    assert v(0, odd1) == "UNO_ERR_ALIGN" and v(13, odd) == "UNO_ERR_ALIGN"
+    assert v(5, 0) == "UNO_OK"

@@ -9,9 +9,9 @@ picx.dev summary, Methodology / Psi-Speculative Sampler (tree sampler: top-K
 at each position). The pins never compare the oracle with itself:
 
 * hand-worked trees and walks (tests/golden/tree_hand.json);
-* the kept set against an independent best-first enumeration of the product
-  of sorted lists (a different algorithm from the oracle's full
-  enumeration), with ties;
+* the kept set: the oracle's full enumeration (the pages' definition) and
+  its best-first search (used when top_k^D is large) agree, with ties, and
+  best-first matches a numpy argsort of all 6^6 joint scores;
 * closed forms: the best sequence is the per-position argmax, a depth-1 tree
   is the top-budget tokens of q_1, budget = top_k^D keeps every combination;
 * invariants: parents precede children, every kept sequence is a root-leaf
@@ -21,7 +21,6 @@ at each position). The pins never compare the oracle with itself:
   the chain-rule product of the AR rows along its prefix.
 """
 
-import heapq
 import json
 import os
 
@@ -89,33 +88,11 @@ def test_golden_walks():
 # --------------------------------------------------------------------------
 
 
-def _best_first(logq_b, budget):
-    """k-best combinations of sorted lists by best-first search: a tuple's
-    successors raise one coordinate at or after its last raised one, so every
-    tuple has one predecessor and is pushed once."""
-    D, k = logq_b.shape
-    avail = [int(np.isfinite(logq_b[i]).sum()) for i in range(D)]
-    if min(avail) == 0:
-        return []
-
-    def score(t):
-        return float(sum(logq_b[i, s] for i, s in enumerate(t)))
-
-    start = (0,) * D
-    heap = [(-score(start), start, 0)]
-    out = []
-    while heap and len(out) < budget:
-        neg, t, last = heapq.heappop(heap)
-        out.append((t, -neg))
-        for j in range(last, D):
-            if t[j] + 1 < avail[j]:
-                u = t[:j] + (t[j] + 1,) + t[j + 1:]
-                heapq.heappush(heap, (-score(u), u, j))
-    return out
-
-
 @pytest.mark.parametrize("seed", range(12))
-def test_kept_set_matches_best_first_search(seed):
+def test_kept_set_enumeration_equals_best_first_search(seed):
+    """The oracle's two routes to the kept set (full enumeration, the pages'
+    definition; best-first search, used when top_k^D is large) agree,
+    including exact ties and rows with few candidates."""
     rng = np.random.default_rng(seed)
     D, k, budget = int(rng.integers(1, 5)), int(rng.integers(1, 5)), int(rng.integers(1, 12))
     V = 12
@@ -124,10 +101,26 @@ def test_kept_set_matches_best_first_search(seed):
     if seed % 3 == 0:
         q[0, 0, rng.integers(0, V, size=V - 2)] = -np.inf  # a row with few candidates
     ids, logq = tree_topk(q, k)
-    got = tree_candidates(logq[0], budget)
-    want = _best_first(logq[0], budget)
+    got = tree_candidates(logq[0], budget, method="enumerate")
+    want = tree_candidates(logq[0], budget, method="best_first")
     assert [t for t, _ in got] == [t for t, _ in want]
     assert np.allclose([s for _, s in got], [s for _, s in want], rtol=0, atol=1e-12)
+
+
+def test_best_first_against_sorted_brute_force_list():
+    """Best-first at a size where enumeration is the textbook check: the
+    first 50 of 6^6 = 46656 sequences, every joint score recomputed from the
+    per-position log-probabilities with numpy broadcasting and argsort."""
+    rng = np.random.default_rng(77)
+    D, k = 6, 6
+    logq = np.sort(rng.normal(-3, 1, size=(D, k)), axis=1)[:, ::-1]
+    grids = np.meshgrid(*[np.arange(k)] * D, indexing="ij")
+    tup = np.stack([g.reshape(-1) for g in grids], axis=1)
+    total = sum(logq[i][tup[:, i]] for i in range(D))
+    order = np.lexsort(tuple(tup[:, i] for i in reversed(range(D))) + (-total,))
+    want = [tuple(int(x) for x in tup[o]) for o in order[:50]]
+    got = [t for t, _ in tree_candidates(logq, 50, method="best_first")]
+    assert got == want
 
 
 def test_topk_order_ties_and_masks():
