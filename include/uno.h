@@ -226,6 +226,52 @@ int uno_dualpath_linear_gated(const void* x, const void* W, const void* A, const
                               size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * LM head with the verifier's row statistics, and the verifier that uses them
+ *
+ * The last dual-path linear of a decode step is the LM head: y_ar holds the
+ * verifier's logits p, y_draft the draft logits q (reader page, "The Uno
+ * Framework": drafting uses theta_AR + theta_Delta, verification theta_AR
+ * alone). uno_dualpath_linear_stats is uno_dualpath_linear_gated (same
+ * arguments, same outputs bit for bit) that also writes, for every output
+ * row and every 256-column tile, the softmax partial of the values it
+ * stored: m = max(value) * log2(e) and z = sum of 2^(value * log2(e) - m)
+ * (float pairs). uno_verify_block_head then verifies without reading every
+ * logit again: it merges those partials instead of streaming the rows and
+ * reads only the logits at the drafted ids and the one p (and q) row that
+ * the final draw needs per sequence.
+ *
+ * uno_dualpath_stats_tiles(M, d_out) = ceil(d_out / 256) when M > 256 (the
+ *   statistics come from the CTA-pair layout), else 0.
+ * uno_dualpath_linear_stats: as uno_dualpath_linear_gated, plus
+ *   stats_ar     [M, T, 2] f32 out (T = uno_dualpath_stats_tiles), or null;
+ *                needs y_ar
+ *   stats_draft  [M, T, 2] f32 out, or null; needs y_draft
+ *   M must exceed 256 (UNO_ERR_SIZE otherwise).
+ * uno_verify_block_head: as uno_verify_block, with
+ *   y_ar         [B, K+1, V] dtype: p, row i of sequence b = LM-head row
+ *                b * (K+1) + i
+ *   y_draft      [B, K+1, V] dtype: q_i of sequence b = row b * (K+1) + i for
+ *                i < K (row K, the bonus position, is not read)
+ *   stats_ar, stats_draft  the partials of those rows, stats_tiles per row
+ *   The accept tests, the draw and every output follow uno_verify_block;
+ *   the row statistics are summed in tile order instead of slab order, so
+ *   probabilities can differ from uno_verify_block's by float32 rounding.
+ *   Workspace: uno_verify_workspace_bytes(B, K, V, dtype).
+ * ------------------------------------------------------------------------ */
+int uno_dualpath_stats_tiles(int M, int d_out);
+int uno_dualpath_linear_stats(const void* x, const void* W, const void* A, const void* Bm,
+                              float scale, const uint8_t* gate, void* y_ar, void* y_draft,
+                              float* stats_ar, float* stats_draft, int M, int d_in, int d_out,
+                              int r, int dtype, void* workspace, size_t workspace_bytes,
+                              void* stream);
+int uno_verify_block_head(const void* y_ar, const void* y_draft, const float* stats_ar,
+                          const float* stats_draft, int stats_tiles, const int32_t* draft_tokens,
+                          int B, int K, int V, int dtype, uint64_t seed, uint64_t step,
+                          int32_t* out_tokens, int32_t* accepted_len, float* p_at_draft,
+                          float* q_at_draft, float* row_lse, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * Drafting a block (linear Psi-Spec sampler)
  *
  * Reader page, "The Psi-Speculative Sampler": the block's candidates are

@@ -66,6 +66,14 @@ def _load() -> ctypes.CDLL:
     L.uno_dualpath_linear_grouped.restype = i32
     L.uno_sample_drafts.argtypes = [vp, i32, i32, i32, i32, u64, u64, vp, vp]
     L.uno_sample_drafts.restype = i32
+    L.uno_dualpath_stats_tiles.argtypes = [i32, i32]
+    L.uno_dualpath_stats_tiles.restype = i32
+    L.uno_dualpath_linear_stats.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp,
+                                            i32, i32, i32, i32, i32, vp, sz, vp]
+    L.uno_dualpath_linear_stats.restype = i32
+    L.uno_verify_block_head.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, u64, u64,
+                                        vp, vp, vp, vp, vp, vp, sz, vp]
+    L.uno_verify_block_head.restype = i32
     L.uno_tree_nodes.argtypes = [i32, i32]
     L.uno_tree_nodes.restype = i32
     L.uno_tree_draft_workspace_bytes.argtypes = [i32, i32, i32, i32]

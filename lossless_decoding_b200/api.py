@@ -227,6 +227,103 @@ def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch
     return y_ar, y_draft
 
 
+def dualpath_stats_tiles(M: int, d_out: int) -> int:
+    """Column tiles of the row statistics of ``dualpath_linear_stats`` (0 when
+    M <= 256: not available)."""
+    return int(lib.uno_dualpath_stats_tiles(M, d_out))
+
+
+def dualpath_linear_stats(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor,
+                          scale: float, *, gate: Optional[torch.Tensor] = None,
+                          y_ar: Optional[torch.Tensor] = None,
+                          y_draft: Optional[torch.Tensor] = None,
+                          stats_ar: Optional[torch.Tensor] = None,
+                          stats_draft: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None):
+    """The LM head: ``dualpath_linear`` (both outputs) that also writes each
+    output row's softmax partials per 256-column tile, float32 [M, T, 2] as
+    (max * log2 e, sum of 2^(x log2 e - that)). M must exceed 256. Returns
+    (y_ar, y_draft, stats_ar, stats_draft)."""
+    if x.dim() != 2 or W.dim() != 2 or A.dim() != 2 or Bm.dim() != 2:
+        raise ValueError("expected 2-D x, W, A, Bm")
+    M, d_in = x.shape
+    d_out = W.shape[0]
+    r = A.shape[0]
+    if W.shape[1] != d_in or A.shape[1] != d_in or tuple(Bm.shape) != (d_out, r):
+        raise ValueError("shape mismatch: x [M,d_in], W [d_out,d_in], A [r,d_in], Bm [d_out,r]")
+    if not (x.dtype == W.dtype == A.dtype == Bm.dtype):
+        raise TypeError("x, W, A and Bm must share a dtype")
+    T = dualpath_stats_tiles(M, d_out)
+    if T == 0:
+        raise ValueError("row statistics need M > 256")
+    dt = _dtype_code(x)
+    dev = _check_cuda(x, W, A, Bm)
+    if y_ar is None:
+        y_ar = torch.empty((M, d_out), dtype=x.dtype, device=dev)
+    if y_draft is None:
+        y_draft = torch.empty((M, d_out), dtype=x.dtype, device=dev)
+    if stats_ar is None:
+        stats_ar = torch.empty((M, T, 2), dtype=torch.float32, device=dev)
+    if stats_draft is None:
+        stats_draft = torch.empty((M, T, 2), dtype=torch.float32, device=dev)
+    for t in (stats_ar, stats_draft):
+        if t.dtype != torch.float32 or tuple(t.shape) != (M, T, 2):
+            raise ValueError(f"stats must be float32 [{M}, {T}, 2]")
+    _check_cuda(y_ar, y_draft, stats_ar, stats_draft)
+    need = int(lib.uno_dualpath_workspace_bytes(M, d_in, d_out, r, dt))
+    ws = workspace if workspace is not None else _ws.get(dev, "dualpath", need)
+    st = lib.uno_dualpath_linear_stats(_ptr(x), _ptr(W), _ptr(A), _ptr(Bm), ctypes.c_float(scale),
+                                       None if gate is None else _gate_arg(gate, M, dev),
+                                       _ptr(y_ar), _ptr(y_draft), _ptr(stats_ar),
+                                       _ptr(stats_draft), M, d_in, d_out, r, dt, _ptr(ws),
+                                       ws.numel(), _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_dualpath_linear_stats")
+    return y_ar, y_draft, stats_ar, stats_draft
+
+
+def verify_block_head(y_ar: torch.Tensor, y_draft: torch.Tensor, stats_ar: torch.Tensor,
+                      stats_draft: torch.Tensor, draft_tokens: torch.Tensor, seed: int,
+                      step: int, *, want_probs: bool = False, want_lse: bool = False,
+                      out: Optional[VerifyResult] = None,
+                      workspace: Optional[torch.Tensor] = None) -> VerifyResult:
+    """Verify from the LM head's outputs and row statistics: y_ar, y_draft
+    [B*(K+1), V] (or [B, K+1, V]) with p = y_ar rows and q_i = y_draft row
+    b*(K+1)+i for i < K; stats from ``dualpath_linear_stats``."""
+    B, K = draft_tokens.shape
+    V = y_ar.shape[-1]
+    if y_ar.numel() != B * (K + 1) * V or y_draft.shape != y_ar.shape:
+        raise ValueError("y_ar and y_draft must hold B*(K+1) rows of V logits")
+    if stats_ar.dim() != 3 or stats_ar.shape[0] != B * (K + 1) or stats_ar.shape[2] != 2 \
+            or stats_draft.shape != stats_ar.shape:
+        raise ValueError("stats must be float32 [B*(K+1), T, 2]")
+    if draft_tokens.dtype != torch.int32:
+        raise TypeError("draft_tokens must be int32")
+    T = stats_ar.shape[1]
+    dt = _dtype_code(y_ar)
+    dev = _check_cuda(y_ar, y_draft, stats_ar, stats_draft, draft_tokens)
+    if out is None:
+        out = VerifyResult(
+            torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+            torch.empty((B,), dtype=torch.int32, device=dev),
+            torch.empty((B, K), dtype=torch.float32, device=dev) if want_probs else None,
+            torch.empty((B, K), dtype=torch.float32, device=dev) if want_probs else None,
+            torch.empty((B, 2 * K + 1), dtype=torch.float32, device=dev) if want_lse else None,
+        )
+    _check_cuda(out.out_tokens, out.accepted_len, out.p_at_draft, out.q_at_draft, out.row_lse)
+    need = int(lib.uno_verify_workspace_bytes(B, K, V, dt))
+    ws = workspace if workspace is not None else _ws.get(dev, "verify", need)
+    st = lib.uno_verify_block_head(
+        _ptr(y_ar), _ptr(y_draft), _ptr(stats_ar), _ptr(stats_draft), T, _ptr(draft_tokens),
+        B, K, V, dt, ctypes.c_uint64(int(seed) & (2**64 - 1)),
+        ctypes.c_uint64(int(step) & (2**64 - 1)), _ptr(out.out_tokens), _ptr(out.accepted_len),
+        _ptr(out.p_at_draft), _ptr(out.q_at_draft), _ptr(out.row_lse), _ptr(ws), ws.numel(),
+        _stream_handle(dev))
+    if st != 0:
+        raise UnoError(st, "uno_verify_block_head")
+    return out
+
+
 def dualpath_linear_grouped(x: torch.Tensor, Ws, As, Bms, scales, *, want_ar: bool = True,
                             want_draft: bool = True, y_ars=None, y_drafts=None,
                             workspace: Optional[torch.Tensor] = None,

@@ -87,6 +87,9 @@ struct GroupArgs {
   void* y_draft;      // may be null (then for every projection)
   void* t_buf;        // T [M][r]
   uint32_t* t_flags;  // [nT]
+  float2* stats_ar;     // [M][stats_tiles] row softmax partials of y_ar (may be null)
+  float2* stats_draft;  // [M][stats_tiles] the same for y_draft (may be null)
+  int stats_tiles;      // column tiles of the projection: ceil(d_out / BN)
 };
 
 struct GemmParams {
@@ -191,6 +194,45 @@ __device__ __forceinline__ void store_one(T* dst, float v) {
   } else {
     *dst = v;
   }
+}
+
+// Softmax statistics of one output row over a tile's columns, as the
+// verifier merges them: m = the largest stored value times log2(e), z = the
+// sum of 2^(value log2 e - m), over the values as stored (bfloat16-rounded
+// for bfloat16 outputs). The reference m moves up only when a larger value
+// arrives.
+struct RowStats {
+  float m, z;
+  __device__ __forceinline__ void init() {
+    m = -INFINITY;
+    z = 0.f;
+  }
+  __device__ __forceinline__ void add(const float* v, int n) {  // the first n of 32 values
+    constexpr float kL2e = 1.4426950408889634f;
+    float mk = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (e < n) mk = fmaxf(mk, v[e]);
+    mk *= kL2e;
+    if (mk > m) {
+      z *= uno::ex2(m - mk);
+      m = mk;
+    }
+    if (m > -INFINITY) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (e < n) s += uno::ex2(fmaf(v[e], kL2e, -m));
+      z += s;
+    }
+  }
+};
+
+// The value a store of v into T keeps.
+template <typename T>
+__device__ __forceinline__ float stored_value(float v) {
+  if constexpr (sizeof(T) == 2) return __uint_as_float(pack_bf16x2(v, 0.f) << 16);
+  else return v;
 }
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -727,13 +769,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // gate: for T tiles, the per-row adapter gate (rows of x: the A rows
     // unswapped, the B rows swapped); a closed row stores T = 0.
     auto drain = [&](uint32_t acc, int a0, int b0, T* y, int ld, int nrows, int ncol,
-                     float mul, const uint8_t* gate = nullptr) {
+                     float mul, const uint8_t* gate = nullptr, float2* stats = nullptr,
+                     int stats_tiles = 0) {
       if (!y) return;
       const uint32_t tq = acc + (static_cast<uint32_t>(quarter * 32) << 16);
       const int arow = a0 + rr;
       if constexpr (!SWAP) {
         if (gate && arow < nrows && gate[arow] == 0) mul = 0.f;
       }
+      RowStats rs;
+      rs.init();
       for (int c = 0; c < ncol; c += 32) {
         uint32_t v[32];
         sm100::tmem_ld_32x32b_x32(tq + c, v);
@@ -753,6 +798,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // row = A row, column = B row
           if (arow < nrows && brow < ld)
             store_row32<T>(y + static_cast<size_t>(arow) * ld + brow, f, ld - brow);
+          if (stats && brow < ld) {
+            float sv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[e] = stored_value<T>(f[e]);
+            rs.add(sv, min(32, ld - brow));
+          }
         } else {
           // row = B row, column = A row
           if (arow < ld) {
@@ -762,6 +813,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 store_one<T>(y + static_cast<size_t>(brow + e) * ld + arow, f[e]);
           }
         }
+      }
+      if constexpr (!SWAP) {
+        if (stats && arow < nrows)
+          stats[static_cast<size_t>(arow) * stats_tiles + b0 / BN] = make_float2(rs.m, rs.z);
       }
     };
     // Drain y_ar = acc and y_draft = acc + adp (both BN columns wide).
@@ -775,12 +830,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint8_t* stage_ar = smem + quarter * 32768;
       uint8_t* stage_dr = stage_ar + 16384;
       const uint32_t sw = static_cast<uint32_t>(lane & 7);
+      float2* st_ar = p.g[gi].stats_ar;
+      float2* st_dr = p.g[gi].stats_draft;
+      RowStats rs_ar, rs_dr;
+      rs_ar.init();
+      rs_dr.init();
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32], w[32];
         sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
         sm100::tmem_ld_32x32b_x32(adp + lq + c, w);
         sm100::tmem_ld_wait();
         // columns c..c+31 = 4 chunks of 16 bytes in box c/64, chunks (c%64)/8..+3
+        float sva[32], svd[32];
         const int box = c >> 6;
         const uint32_t chunk0 = static_cast<uint32_t>((c & 63) >> 3);
 #pragma unroll
@@ -802,6 +863,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                (((chunk0 + g) ^ sw) << 4);
           *reinterpret_cast<uint4*>(stage_ar + off) = a;
           *reinterpret_cast<uint4*>(stage_dr + off) = d;
+          if (st_ar || st_dr) {  // the stored (rounded) values, unpacked again
+            const uint32_t pa[4] = {a.x, a.y, a.z, a.w}, pd[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              sva[8 * g + 2 * h] = __uint_as_float(pa[h] << 16);
+              sva[8 * g + 2 * h + 1] = __uint_as_float(pa[h] & 0xFFFF0000u);
+              svd[8 * g + 2 * h] = __uint_as_float(pd[h] << 16);
+              svd[8 * g + 2 * h + 1] = __uint_as_float(pd[h] & 0xFFFF0000u);
+            }
+          }
+        }
+        if (st_ar || st_dr) {
+          const int nvalid = min(32, ncols - (b0 + c));
+          if (st_ar) rs_ar.add(sva, nvalid);
+          if (st_dr) rs_dr.add(svd, nvalid);
+        }
+      }
+      {
+        const int arow = a0 + lane;
+        if (arow < p.M) {
+          const size_t at = static_cast<size_t>(arow) * p.g[gi].stats_tiles + b0 / BN;
+          if (st_ar) st_ar[at] = make_float2(rs_ar.m, rs_ar.z);
+          if (st_dr) st_dr[at] = make_float2(rs_dr.m, rs_dr.z);
         }
       }
       fence_proxy_async_shared();
@@ -820,6 +904,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto drain2 = [&](uint32_t acc, uint32_t adp, int a0, int b0) {
       const uint32_t lq = static_cast<uint32_t>(quarter * 32) << 16;
       const int arow = a0 + rr;
+      float2* st2[2] = {p.g[gi].stats_ar, p.g[gi].stats_draft};
+      RowStats rs2[2];
+      rs2[0].init();
+      rs2[1].init();
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32], w[32];
         sm100::tmem_ld_32x32b_x32(acc + lq + c, v);
@@ -837,6 +925,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if constexpr (!SWAP) {
             if (arow < p.M && brow < ncols)
               store_row32<T>(y + static_cast<size_t>(arow) * ncols + brow, f, ncols - brow);
+            if (st2[pass] && brow < ncols) {
+              float sv[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) sv[e] = stored_value<T>(f[e]);
+              rs2[pass].add(sv, min(32, ncols - brow));
+            }
           } else {
             if (arow < ncols) {
 #pragma unroll
@@ -844,6 +938,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * ncols + arow, f[e]);
             }
           }
+        }
+      }
+      if constexpr (!SWAP) {
+        if (arow < p.M) {
+          const size_t at = static_cast<size_t>(arow) * p.g[gi].stats_tiles + b0 / BN;
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass)
+            if (st2[pass]) st2[pass][at] = make_float2(rs2[pass].m, rs2[pass].z);
         }
       }
     };
@@ -976,7 +1078,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           drain2(acc, tmem + static_cast<uint32_t>((buf ^ 1) * kAcc), x.a0 + my_rows, x.b0);
         break;
       }
-      drain(acc, x.a0 + my_rows, x.b0, ya, ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, ya, ncols, p.M, BN, 1.f, nullptr, p.g[gi].stats_ar,
+            p.g[gi].stats_tiles);
       sm100::tc_fence_before();
       __syncwarp();
       const int mo = li - nt_mine;
@@ -988,7 +1091,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       sm100::tc_fence_after();
-      drain(acc, x.a0 + my_rows, x.b0, yd, ncols, p.M, BN, 1.f);
+      drain(acc, x.a0 + my_rows, x.b0, yd, ncols, p.M, BN, 1.f, nullptr, p.g[gi].stats_draft,
+            p.g[gi].stats_tiles);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(&acc_empty[buf]);
@@ -1246,7 +1350,8 @@ template <typename T>
 int run_dualpath(int n, const void* x, const void* const* W, const void* const* A,
                  const void* const* Bm, const float* scale, const uint8_t* gate,
                  void* const* y_ar, void* const* y_draft, int M, int d_in, const int* d_out,
-                 int r, int dtype, void* workspace, cudaStream_t st) {
+                 int r, int dtype, void* workspace, cudaStream_t st,
+                 float* const* stats_ar = nullptr, float* const* stats_draft = nullptr) {
   const Plan pl = make_plan(M, d_in, r, dtype);
   const bool adapter = (y_draft[0] != nullptr);
   const bool tf32 = (dtype == UNO_F32);
@@ -1271,6 +1376,9 @@ int run_dualpath(int n, const void* x, const void* const* W, const void* const* 
     a.scale = scale[g];
     a.y_ar = y_ar[g];
     a.y_draft = y_draft[g];
+    a.stats_ar = stats_ar ? reinterpret_cast<float2*>(stats_ar[g]) : nullptr;
+    a.stats_draft = stats_draft ? reinterpret_cast<float2*>(stats_draft[g]) : nullptr;
+    a.stats_tiles = (d_out[g] + 255) / 256;
     a.t_buf = ws;
     a.t_flags = reinterpret_cast<uint32_t*>(ws + pl.t_bytes);
     ws += pl.t_bytes + pl.flag_bytes;
@@ -1358,7 +1466,8 @@ int check_dual_args(int n, const void* x, const void* const* W, const void* cons
 int dispatch(int n, const void* x, const void* const* W, const void* const* A,
              const void* const* Bm, const float* scale, const uint8_t* gate, void* const* y_ar,
              void* const* y_draft, int M, int d_in, const int* d_out, int r, int dtype,
-             void* workspace, size_t workspace_bytes, void* stream) {
+             void* workspace, size_t workspace_bytes, void* stream,
+             float* const* stats_ar = nullptr, float* const* stats_draft = nullptr) {
   const int chk = check_dual_args(n, x, W, A, Bm, y_ar, y_draft, M, d_in, d_out, r, dtype,
                                   workspace, workspace_bytes);
   if (chk != 1) return chk;
@@ -1367,9 +1476,9 @@ int dispatch(int n, const void* x, const void* const* W, const void* const* A,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == UNO_BF16)
     return run_dualpath<uint16_t>(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r,
-                                  dtype, workspace, st);
+                                  dtype, workspace, st, stats_ar, stats_draft);
   return run_dualpath<float>(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r,
-                             dtype, workspace, st);
+                             dtype, workspace, st, stats_ar, stats_draft);
 }
 
 }  // namespace
@@ -1416,6 +1525,24 @@ extern "C" int uno_dualpath_linear_grouped(int n, const void* x, const void* con
   if (!scale) return UNO_ERR_NULL;
   return dispatch(n, x, W, A, Bm, scale, gate, y_ar, y_draft, M, d_in, d_out, r, dtype,
                   workspace, workspace_bytes, stream);
+}
+
+extern "C" int uno_dualpath_stats_tiles(int M, int d_out) {
+  if (M <= 256 || d_out < 1) return 0;  // row statistics come from the CTA-pair layout
+  return (d_out + 255) / 256;
+}
+
+extern "C" int uno_dualpath_linear_stats(const void* x, const void* W, const void* A,
+                                         const void* Bm, float scale, const uint8_t* gate,
+                                         void* y_ar, void* y_draft, float* stats_ar,
+                                         float* stats_draft, int M, int d_in, int d_out, int r,
+                                         int dtype, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  if (M <= 256) return UNO_ERR_SIZE;
+  if ((stats_ar && !y_ar) || (stats_draft && !y_draft)) return UNO_ERR_NULL;
+  if (!uno_host::aligned(stats_ar, 8) || !uno_host::aligned(stats_draft, 8)) return UNO_ERR_ALIGN;
+  return dispatch(1, x, &W, &A, &Bm, &scale, gate, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
+                  workspace, workspace_bytes, stream, &stats_ar, &stats_draft);
 }
 
 extern "C" int uno_device_fault_flags(int clear, unsigned int* flags) {

@@ -88,6 +88,14 @@ struct VerifyParams {
   float* chunk_sums;  // [B][nchunks]
   int* draw_count;    // [B], set to 0 by the decision launch
   Decision* decisions;  // [B]
+  // Rows of q per sequence in memory: K (q is [B][K][V]) or K+1 (q is the
+  // draft-pathway output of the same B x (K+1) rows as p, bonus rows unused).
+  int q_rows = 0;
+  // Row statistics written by the LM-head GEMM (null: the stream launch
+  // computes them): ext_T partials per logit row, in the partial convention.
+  const Partial* ext_p = nullptr;  // [B][K+1][ext_T]
+  const Partial* ext_q = nullptr;  // [B][q_rows][ext_T]
+  int ext_T = 0;
 };
 
 // ---- element access -----------------------------------------------------------
@@ -211,7 +219,7 @@ __device__ __forceinline__ const T* row_ptr(const VerifyParams& P, int b, int j,
     row = static_cast<size_t>(b) * (K + 1) + j;
     base = static_cast<const T*>(P.p_logits);
   } else {
-    row = static_cast<size_t>(b) * K + (j - K - 1);
+    row = static_cast<size_t>(b) * P.q_rows + (j - K - 1);
     base = static_cast<const T*>(P.q_logits);
   }
   *off = row * static_cast<size_t>(P.V);
@@ -437,19 +445,52 @@ __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyPar
   const int K = P.K, R = 2 * K + 1, S = P.S, V = P.V;
 
   // row statistics: merge the slab partials of every row in slab order
-  for (int j = tid; j < R; j += kThreads) {
-    const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
-    float m = -INFINITY, z = 0.f;
-    for (int s0 = 0; s0 < S; s0 += 8) {  // eight loads in flight, merged in slab order
-      Partial v[8];
+  if (P.ext_p == nullptr) {
+    for (int j = tid; j < R; j += kThreads) {
+      const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
+      float m = -INFINITY, z = 0.f;
+      for (int s0 = 0; s0 < S; s0 += 8) {  // eight loads in flight, merged in slab order
+        Partial v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? pp[s0 + k] : Partial{-INFINITY, 0.f};
+        for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? pp[s0 + k] : Partial{-INFINITY, 0.f};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) merge(m, z, v[k].m, v[k].z);
+        for (int k = 0; k < 8; ++k) merge(m, z, v[k].m, v[k].z);
+      }
+      sh.row_m[j] = m;
+      sh.row_z[j] = z;
+      if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
     }
-    sh.row_m[j] = m;
-    sh.row_z[j] = z;
-    if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
+  } else {
+    // the LM head's column-tile partials (hundreds per row): one warp per row,
+    // lanes over the tiles, then a shuffle reduction
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int j = warp; j < R; j += kWarps) {
+      const Partial* pp = (j <= K)
+          ? P.ext_p + (static_cast<size_t>(b) * (K + 1) + j) * P.ext_T
+          : P.ext_q + (static_cast<size_t>(b) * P.q_rows + (j - K - 1)) * P.ext_T;
+      float m = -INFINITY, z = 0.f;
+      for (int t0 = lane; t0 < P.ext_T; t0 += 32 * 4) {  // four loads in flight per lane
+        Partial v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int t = t0 + 32 * k;
+          v[k] = (t < P.ext_T) ? pp[t] : Partial{-INFINITY, 0.f};
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) merge(m, z, v[k].m, v[k].z);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+        const float z2 = __shfl_xor_sync(0xFFFFFFFFu, z, o);
+        merge(m, z, m2, z2);
+      }
+      if (lane == 0) {
+        sh.row_m[j] = m;
+        sh.row_z[j] = z;
+        if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
+      }
+    }
   }
   if (tid == 0) {
     sh.first_reject = K;
@@ -729,7 +770,9 @@ int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P
 
 template <typename T>
 int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
-  if (launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  if (P.ext_p == nullptr &&
+      launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK)
+    return UNO_ERR_CUDA;
   if (launch_pdl(verify_decide_kernel<T>, P.B, st, P) != UNO_OK) return UNO_ERR_CUDA;
   if (launch_pdl(verify_draw_kernel<T>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
@@ -789,6 +832,66 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
   P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
   P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
+  P.q_rows = K;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return (dtype == UNO_BF16) ? launch<uint16_t>(P, g, st) : launch<float>(P, g, st);
+}
+
+extern "C" int uno_verify_block_head(const void* y_ar, const void* y_draft, const float* stats_ar,
+                                     const float* stats_draft, int stats_tiles,
+                                     const int32_t* draft_tokens, int B, int K, int V, int dtype,
+                                     uint64_t seed, uint64_t step, int32_t* out_tokens,
+                                     int32_t* accepted_len, float* p_at_draft, float* q_at_draft,
+                                     float* row_lse, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
+  if (!verify_sizes_ok(B, K, V, dtype) || stats_tiles < 1 || stats_tiles > (1 << 20))
+    return UNO_ERR_SIZE;
+  if (B == 0) return UNO_OK;
+  if (!y_ar || !y_draft || !stats_ar || !stats_draft || !draft_tokens || !out_tokens ||
+      !accepted_len)
+    return UNO_ERR_NULL;
+  if (!workspace) return UNO_ERR_WORKSPACE;
+  if (!uno_host::aligned(y_ar, 16) || !uno_host::aligned(y_draft, 16) ||
+      !uno_host::aligned(stats_ar, 8) || !uno_host::aligned(stats_draft, 8) ||
+      !uno_host::aligned(workspace, 16) || !uno_host::aligned(draft_tokens, 4) ||
+      !uno_host::aligned(out_tokens, 4) || !uno_host::aligned(accepted_len, 4) ||
+      !uno_host::aligned(p_at_draft, 4) || !uno_host::aligned(q_at_draft, 4) ||
+      !uno_host::aligned(row_lse, 4))
+    return UNO_ERR_ALIGN;
+  const Geometry g = geometry(B, K, V, dtype);
+  if (workspace_bytes < g.bytes) return UNO_ERR_WORKSPACE;
+  if (g.draw_ctas > INT_MAX) return UNO_ERR_SIZE;
+  const int dev_status = uno_host::check_device();
+  if (dev_status != UNO_OK) return dev_status;
+
+  char* ws = static_cast<char*>(workspace);
+  VerifyParams P;
+  P.p_logits = y_ar;
+  P.q_logits = y_draft;
+  P.draft = draft_tokens;
+  P.B = B;
+  P.K = K;
+  P.V = V;
+  P.S = g.S;
+  P.nchunks = g.nchunks;
+  P.chunk_len = g.chunk_len;
+  P.SD = g.SD;
+  P.seed = seed;
+  P.step = step;
+  P.out_tokens = out_tokens;
+  P.accepted_len = accepted_len;
+  P.p_at_draft = p_at_draft;
+  P.q_at_draft = q_at_draft;
+  P.row_lse = row_lse;
+  P.draw_count = reinterpret_cast<int*>(ws + g.off_counts);
+  P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
+  P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
+  P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
+  P.q_rows = K + 1;
+  P.ext_p = reinterpret_cast<const Partial*>(stats_ar);
+  P.ext_q = reinterpret_cast<const Partial*>(stats_draft);
+  P.ext_T = stats_tiles;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return (dtype == UNO_BF16) ? launch<uint16_t>(P, g, st) : launch<float>(P, g, st);
 }

@@ -194,3 +194,36 @@ def test_tree_argument_errors_need_no_gpu(lib):
     assert v(0, None) == "UNO_ERR_NULL" and v(12, None) == "UNO_ERR_NULL"
     assert v(0, odd1) == "UNO_ERR_ALIGN" and v(13, odd) == "UNO_ERR_ALIGN"
     assert v(5, 0) == "UNO_OK"
+
+
+def test_head_argument_errors_need_no_gpu(lib):
+    from lossless_decoding_b200._lib import STATUS
+    fake = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4096 + 4)
+    u64 = ctypes.c_uint64
+    assert lib.uno_dualpath_stats_tiles(1088, 151936) == 594
+    assert lib.uno_dualpath_stats_tiles(256, 151936) == 0
+    st = lib.uno_dualpath_linear_stats
+    # statistics need the CTA-pair layout (M > 256)
+    assert STATUS[st(fake, fake, fake, fake, 2.0, None, fake, fake, fake, fake, 256, 4096, 4096,
+                     128, 0, fake, 1 << 30, None)] == "UNO_ERR_SIZE"
+    # statistics of an output that is not written
+    assert STATUS[st(fake, fake, fake, fake, 2.0, None, None, fake, fake, fake, 1088, 4096, 4096,
+                     128, 0, fake, 1 << 30, None)] == "UNO_ERR_NULL"
+    assert STATUS[st(fake, fake, fake, fake, 2.0, None, fake, fake, odd, fake, 1088, 4096, 4096,
+                     128, 0, fake, 1 << 30, None)] == "UNO_ERR_ALIGN"
+    vh = lib.uno_verify_block_head
+    args = [fake, fake, fake, fake, 594, fake, 64, 16, 151936, 0, u64(0), u64(0), fake, fake,
+            None, None, None, fake, 1 << 30, None]
+
+    def v(i, val):
+        a = list(args)
+        a[i] = val
+        return STATUS[vh(*a)]
+
+    assert v(9, 7) == "UNO_ERR_DTYPE"
+    assert v(4, 0) == "UNO_ERR_SIZE" and v(7, 0) == "UNO_ERR_SIZE"
+    assert v(2, None) == "UNO_ERR_NULL" and v(5, None) == "UNO_ERR_NULL"
+    assert v(2, odd) == "UNO_ERR_ALIGN"
+    assert v(17, None) == "UNO_ERR_WORKSPACE" and v(18, 8) == "UNO_ERR_WORKSPACE"
+    assert v(6, 0) == "UNO_OK"
