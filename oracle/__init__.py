@@ -18,7 +18,10 @@ from .uno_oracle import (  # noqa: F401
     sample_drafts_u,
     softmax_rows,
     uniforms_for_block,
+    merge_row_stats,
+    row_stat_partials,
     verify_block,
+    verify_block_head,
     verify_block_u,
     word_to_uniform,
 )

@@ -37,6 +37,11 @@ What each function follows:
   accepts the whole block or replaces the tail with a single token drawn
   from the verifier), with the accept and residual rules of [SD].
 * ``philox4x32_10``: [SC11].
+* ``row_stat_partials`` / ``merge_row_stats`` / ``verify_block_head``: the
+  verifier's row normalisers split into per-column-tile partials (the form in
+  which the LM head can produce them) and the verifier on the LM head's row
+  layout (p = a block's K+1 AR rows, q_i = its draft row i < K); no new
+  arithmetic, the definitions above rearranged.
 
 Readings of the pages that this module fixes (each one is listed with its
 reason in the repository's design notes):
@@ -400,3 +405,63 @@ def sample_drafts(q_logits, seed: int, step: int):
     """Drafted ids for one block: sample_drafts_u with draft_uniforms."""
     q = np.asarray(q_logits)
     return sample_drafts_u(q, draft_uniforms(q.shape[0], q.shape[1], seed, step))
+
+
+# --------------------------------------------------------------------------
+# The LM head feeding the verifier (the fused row): row statistics per column
+# tile and the verifier on the LM head's row layout
+# --------------------------------------------------------------------------
+
+
+def row_stat_partials(y, tile: int = 256):
+    """Softmax partials of each row of y [M, N] per column tile, float64.
+
+    Tile t covers columns [t*tile, (t+1)*tile). Its partial is
+    (m, z) = (max(y) * log2(e), sum of 2^(y * log2(e) - m)) over the tile's
+    finite entries, (-inf, 0) when it has none. Merging the partials of a row
+    gives its normaliser: log Z = ln 2 * (M + log2 sum_t z_t 2^(m_t - M)),
+    M = max_t m_t. Returns an array [M, T, 2].
+    """
+    y = np.asarray(y, dtype=np.float64)
+    M, N = y.shape
+    T = (N + tile - 1) // tile
+    out = np.empty((M, T, 2))
+    log2e = 1.0 / np.log(2.0)
+    for t in range(T):
+        blk = y[:, t * tile:(t + 1) * tile] * log2e
+        fin = np.isfinite(blk)
+        m = np.where(fin, blk, -np.inf).max(axis=1)
+        has = np.isfinite(m)
+        ref = np.where(has, m, 0.0)
+        z = np.where(fin, np.exp2(np.where(fin, blk, 0.0) - ref[:, None]), 0.0).sum(axis=1)
+        out[:, t, 0] = m
+        out[:, t, 1] = np.where(has, z, 0.0)
+    return out
+
+
+def merge_row_stats(partials):
+    """Natural-log normaliser of each row from its [T, 2] partials."""
+    p = np.asarray(partials, dtype=np.float64)
+    m, z = p[..., 0], p[..., 1]
+    top = m.max(axis=-1)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w = np.where(np.isfinite(m), z * np.exp2(m - safe[..., None]), 0.0).sum(axis=-1)
+    ok = np.isfinite(top)
+    return np.where(ok, (top + np.log2(np.where(ok, w, 1.0))) * np.log(2.0), -np.inf)
+
+
+def verify_block_head(y_ar, y_draft, draft_tokens, seed: int, step: int):
+    """The verifier on the LM head's outputs, as the fused entry reads them.
+
+    y_ar, y_draft [B*(K+1), V]: one block of K+1 rows per sequence. The
+    verifier's p is the block's K+1 AR rows; q_i is the block's draft row i
+    for i < K (the bonus position's draft row is not a draft distribution of
+    any drafted token). Then ``verify_block``.
+    """
+    x = np.asarray(draft_tokens)
+    B, K = x.shape
+    y_ar = np.asarray(y_ar, dtype=np.float64)
+    V = y_ar.shape[-1]
+    p = y_ar.reshape(B, K + 1, V)
+    q = np.asarray(y_draft, dtype=np.float64).reshape(B, K + 1, V)[:, :K]
+    return verify_block(p, q, x, seed=seed, step=step)
