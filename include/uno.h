@@ -7,7 +7,9 @@
  * linear; the reader's "The Psi-Speculative Sampler" and "Sampler Extensions"
  * (linear sampler) define the verification step, with the standard speculative
  * rejection-sampling rule the pages cite (Leviathan et al. 2023; Chen et al.
- * 2023).
+ * 2023). The same sections, with the worked (B, K, V) = (3, 2, 2) example and
+ * the summary page's "Psi-Speculative Sampler", define drafting and the tree
+ * sampler. Each entry point below names its passage.
  *
  * Conventions shared by every entry point:
  *  - Every buffer argument is a DEVICE pointer owned by the caller. The library
@@ -17,7 +19,9 @@
  *    errors (checked on the host before anything is launched) and launch errors.
  *  - Matrices are dense and row-major with no padding between rows.
  *  - Base pointers of logits, activations, weights and outputs must be 16-byte
- *    aligned (cudaMalloc and PyTorch allocations are 256-byte aligned).
+ *    aligned (cudaMalloc and PyTorch allocations are 256-byte aligned); the
+ *    draft and tree samplers need only element alignment. Workspaces must be
+ *    16-byte aligned (the tree draft's 256-byte aligned).
  *  - On an error nothing is launched and no output is written.
  */
 #ifndef UNO_H_
