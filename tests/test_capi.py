@@ -227,3 +227,35 @@ def test_head_argument_errors_need_no_gpu(lib):
     assert v(2, odd) == "UNO_ERR_ALIGN"
     assert v(17, None) == "UNO_ERR_WORKSPACE" and v(18, 8) == "UNO_ERR_WORKSPACE"
     assert v(6, 0) == "UNO_OK"
+
+
+def test_valid_calls_without_a_device_report_an_error(lib):
+    """On a host with no CUDA device, a call whose arguments all pass the
+    checks stops at the device check (UNO_ERR_CUDA or UNO_ERR_DEVICE): nothing
+    is launched and no pointer is touched. Skipped where a GPU exists, since
+    the fake pointers would then reach a launch."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    from lossless_decoding_b200._lib import STATUS
+    fake = ctypes.c_void_p(1 << 20)  # 256-byte aligned, never dereferenced
+    u64 = ctypes.c_uint64
+    bad = {"UNO_ERR_CUDA", "UNO_ERR_DEVICE"}
+    need_v = lib.uno_verify_workspace_bytes(2, 4, 1000, 0)
+    assert STATUS[lib.uno_verify_block(fake, fake, fake, 2, 4, 1000, 0, u64(0), u64(0), fake,
+                                       fake, None, None, None, fake, need_v, None)] in bad
+    assert STATUS[lib.uno_verify_block_head(fake, fake, fake, fake, 4, fake, 2, 4, 1000, 0,
+                                            u64(0), u64(0), fake, fake, None, None, None, fake,
+                                            need_v, None)] in bad
+    need_d = lib.uno_dualpath_workspace_bytes(512, 256, 512, 32, 0)
+    assert STATUS[lib.uno_dualpath_linear(fake, fake, fake, fake, 2.0, fake, fake, 512, 256, 512,
+                                          32, 0, fake, need_d, None)] in bad
+    assert STATUS[lib.uno_dualpath_linear_stats(fake, fake, fake, fake, 2.0, None, fake, fake,
+                                                fake, fake, 512, 256, 512, 32, 0, fake, need_d,
+                                                None)] in bad
+    assert STATUS[lib.uno_sample_drafts(fake, 2, 4, 1000, 0, u64(0), u64(0), fake, None)] in bad
+    need_t = lib.uno_tree_draft_workspace_bytes(2, 3, 1000, 2)
+    assert STATUS[lib.uno_tree_draft(fake, 2, 3, 1000, 0, 2, 2, fake, fake, fake, fake, fake,
+                                     fake, fake, need_t, None)] in bad
+    assert STATUS[lib.uno_tree_verify(fake, fake, fake, fake, fake, 2, 3, 2, 1000, 0, u64(0),
+                                      u64(0), fake, fake, fake, None)] in bad
