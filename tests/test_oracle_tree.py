@@ -400,3 +400,47 @@ def test_build_accepts_precomputed_topk():
     b = tree_draft(q, 3, 5)
     for f in ("node_token", "node_parent", "node_depth", "n_nodes"):
         assert np.array_equal(a[f], b[f])
+
+
+def test_walk_draws_at_every_node_follow_its_row():
+    """Monte Carlo over Philox uniforms: among walks that reach a node, the
+    token drawn there is distributed as softmax of that node's AR row
+    (chi-square per node), so each depth's uniform is independent of the
+    path and the walk reads the right row."""
+    from scipy import stats as st
+    rng = np.random.default_rng(21)
+    V, D = 5, 2
+    q = rng.normal(0, 1, size=(1, D, V))
+    tree = tree_draft(q, 2, 3)
+    N = tree["node_token"].shape[1]
+    p = rng.normal(0, 0.8, size=(1, N, V))
+    for c in range(1, int(tree["n_nodes"][0])):  # make the tree's tokens likely
+        p[0, tree["node_parent"][0, c], tree["node_token"][0, c]] += 1.5
+    n_draws = 40000
+    pb = np.broadcast_to(p, (n_draws, N, V))
+    tb = {f: np.broadcast_to(tree[f], (n_draws,) + tree[f].shape[1:]) for f in
+          ("node_token", "node_parent", "n_nodes")}
+    res = tree_verify_u(pb, tb["node_token"], tb["node_parent"], tb["n_nodes"],
+                        tree_uniforms(n_draws, D, seed=17, step=4))
+    out = res["out_tokens"]
+    tok, par = tree["node_token"][0], tree["node_parent"][0]
+    P = special.softmax(p[0], axis=-1)
+    # node reached by each walk at each depth, found from the emitted tokens
+    node = np.zeros(n_draws, dtype=np.int64)
+    checked = 0
+    for j in range(D + 1):
+        live = out[:, j] >= 0
+        for n in np.unique(node[live]):
+            sel = live & (node == n)
+            if sel.sum() < 500:
+                continue
+            counts = np.bincount(out[sel, j], minlength=V)
+            assert st.chisquare(counts, P[n] * sel.sum()).pvalue > 1e-4, (j, n)
+            checked += 1
+        # advance along accepted tokens
+        nxt = np.full(n_draws, -1)
+        for c in range(1, int(tree["n_nodes"][0])):
+            hit = live & (par[c] == node) & (out[:, j] == tok[c]) & (res["accepted_len"] > j)
+            nxt[hit] = c
+        node = np.where(nxt >= 0, nxt, node)  # stopped walks are -1 from here on
+    assert checked >= 3
