@@ -1,13 +1,17 @@
 """Pins of the oracle's Philox4x32-10 and uniform mapping.
 
 Philox4x32-10 is the counter-based generator of Salmon et al., "Parallel
-Random Numbers: As Easy as 1, 2, 3" (SC'11). Its published known-answer
-vectors are not available here, so whether the oracle reproduces the
-canonical stream bit for bit is *parity unpinned*; what these tests pin is
-the structure (10 invertible rounds with the stated key schedule, checked by
-running the rounds backwards) and the statistical quality the sampler's
-losslessness needs (uniform, independent words and counters).
+Random Numbers: As Easy as 1, 2, 3" (SC'11). The oracle's stream is pinned to
+the known-answer vectors published with that paper's Random123 library
+(tests/golden/philox_kat.json), so a wrong multiplier, Weyl constant, word
+order or round count fails here. The other tests pin the structure (10
+invertible rounds with the stated key schedule, checked by running the rounds
+backwards) and the statistical quality the sampler's losslessness needs
+(uniform, independent words and counters).
 """
+
+import json
+import os
 
 import numpy as np
 import pytest
@@ -16,6 +20,39 @@ from scipy import stats
 from oracle import philox4x32_10, uniforms_for_block, word_to_uniform
 
 MASK = (1 << 32) - 1
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "philox_kat.json")
+
+
+def _kat_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _kat_cases(), ids=lambda c: c["name"])
+def test_published_known_answer_vectors(case):
+    ctr = np.array([int(w, 16) for w in case["counter"]], dtype=np.uint32)
+    key = np.array([int(w, 16) for w in case["key"]], dtype=np.uint32)
+    out = philox4x32_10(ctr, key)
+    assert [f"{int(w):08x}" for w in out] == case["out"]
+    # batched calls see the same block
+    both = philox4x32_10(np.stack([ctr, ctr]), key)
+    assert np.array_equal(both[0], out) and np.array_equal(both[1], out)
+
+
+def test_block_words_map_to_the_documented_counter_and_key():
+    # counter (b, i, step lo, step hi), key (seed lo, seed hi): the all-zero
+    # known answer is sequence 0, position 0, step 0 under seed 0
+    zeros = next(c for c in _kat_cases() if c["name"] == "zeros")
+    u_acc, u_smp = uniforms_for_block(B=1, K=1, seed=0, step=0)
+    assert u_acc[0, 0] == (int(zeros["out"][0], 16) >> 8) * 2.0**-24
+    assert u_smp[0, 0] == (int(zeros["out"][1], 16) >> 8) * 2.0**-24
+    pi = next(c for c in _kat_cases() if c["name"] == "pi digits")
+    seed = int(pi["key"][0], 16) | (int(pi["key"][1], 16) << 32)
+    step = int(pi["counter"][2], 16) | (int(pi["counter"][3], 16) << 32)
+    ctr = np.array([[int(pi["counter"][0], 16), int(pi["counter"][1], 16),
+                     step & MASK, step >> 32]], dtype=np.uint32)
+    key = np.array([seed & MASK, seed >> 32], dtype=np.uint32)
+    assert [f"{int(w):08x}" for w in philox4x32_10(ctr, key)[0]] == pi["out"]
 
 
 def _inv_mod32(a: int) -> int:
