@@ -117,16 +117,19 @@ int uno_verify_block(const void* p_logits, const void* q_logits, const int32_t* 
  * synchronise the device), or a caller from another language with no device
  * allocator at hand.
  *
- * Scratch: one fixed 4 MiB array in the library's device memory, reserved on
- * every GPU that loads the library until the process exits. Calls whose
+ * Scratch: one fixed 4 MiB array in the library's device memory. It is
+ * reserved on a device once the library's module is loaded there -- with
+ * CUDA's default lazy module loading, at this entry point's first call on that
+ * device -- and stays reserved until the process exits. Calls whose
  * uno_verify_workspace_bytes(B, K, V, dtype) exceeds 4 MiB are rejected with
  * UNO_ERR_SIZE (for example B = 64, K = 16, V = 151936 needs about 51 KB).
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
- * Every call clears the part of the array it uses on `stream` before its
- * kernels run. All calls on a device share the array, so calls that may
- * overlap on the GPU (different streams, or different host threads without
- * ordering) race and corrupt each other's results: order them on one stream.
+ * The array keeps the previous call's contents; the verifier does not depend
+ * on them (it rewrites whatever it reads), so nothing is cleared. All calls
+ * on a device share the array, so calls that may overlap on the GPU
+ * (different streams, or different host threads without ordering) race and
+ * corrupt each other's results: order them on one stream.
  * The library calls no cudaMalloc, cudaFree or other allocating routine here.
  * Arguments, outputs and errors are those of uno_verify_block.
  */

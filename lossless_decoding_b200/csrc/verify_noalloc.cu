@@ -9,9 +9,10 @@
 // the verifier with its scratch in a fixed array that lives in the library's
 // own device memory, so the call allocates nothing.
 //
-// The scratch is one file-scope array of kNoAllocScratchBytes per device that
-// loads the library; it stays reserved until the process exits. All calls on
-// a device share it.
+// The scratch is one file-scope array of kNoAllocScratchBytes per device. It
+// is reserved on a device once the module that holds it is loaded there (with
+// CUDA's default lazy loading: at this entry point's first use on that device)
+// and stays reserved until the process exits. All calls on a device share it.
 #include <atomic>
 #include <cstdint>
 #include <mutex>
@@ -62,10 +63,13 @@ extern "C" int uno_verify_block_noalloc(const void* p_logits, const void* q_logi
                                         float* p_at_draft, float* q_at_draft, float* row_lse,
                                         void* stream) {
   if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
-  if (B == 0 && K >= 1 && V >= 1) return UNO_OK;
+  // Sizes are checked before B = 0 returns, exactly as uno_verify_block does
+  // (the workspace size of one sequence is 0 only for bad K, V or dtype).
+  if (B < 0 || B > (1 << 20) || uno_verify_workspace_bytes(1, K, V, dtype) == 0)
+    return UNO_ERR_SIZE;
+  if (B == 0) return UNO_OK;
   const size_t need = uno_verify_workspace_bytes(B, K, V, dtype);
-  if (need == 0) return UNO_ERR_SIZE;
-  if (need > kNoAllocScratchBytes) return UNO_ERR_SIZE;  // problem larger than the fixed scratch
+  if (need == 0 || need > kNoAllocScratchBytes) return UNO_ERR_SIZE;  // beyond the fixed scratch
   // Check the caller's pointers before any work is queued.
   if (!p_logits || !q_logits || !draft_tokens || !out_tokens || !accepted_len)
     return UNO_ERR_NULL;
@@ -79,10 +83,9 @@ extern "C" int uno_verify_block_noalloc(const void* p_logits, const void* q_logi
   void* scratch = nullptr;
   const int st = scratch_for_current_device(&scratch);
   if (st != UNO_OK) return st;
-  // The array keeps whatever the previous call left; clear the part this call
-  // uses on the caller's stream so every call starts from the same state.
-  if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return UNO_ERR_CUDA;
+  // The array keeps whatever the previous call left. uno_verify_block does
+  // not depend on the contents of its workspace on entry (every counter and
+  // record it reads is rewritten by the same call first), so nothing is cleared.
   return uno_verify_block(p_logits, q_logits, draft_tokens, B, K, V, dtype, seed, step,
                           out_tokens, accepted_len, p_at_draft, q_at_draft, row_lse, scratch,
                           kNoAllocScratchBytes, stream);

@@ -259,3 +259,15 @@ def test_valid_calls_without_a_device_report_an_error(lib):
                                      fake, fake, need_t, None)] in bad
     assert STATUS[lib.uno_tree_verify(fake, fake, fake, fake, fake, 2, 3, 2, 1000, 0, u64(0),
                                       u64(0), fake, fake, fake, None)] in bad
+
+
+def test_noalloc_checks_sizes_before_the_empty_batch(lib):
+    # B = 0 is accepted only with valid K and V, as for uno_verify_block
+    for K, V, want in ((4, 100, "UNO_OK"), (257, 100, "UNO_ERR_SIZE"), (4, 0, "UNO_ERR_SIZE")):
+        st = lib.uno_verify_block_noalloc(None, None, None, 0, K, V, 0, ctypes.c_uint64(0),
+                                          ctypes.c_uint64(0), None, None, None, None, None, None)
+        assert lib.uno_status_string(st).decode().startswith(want)
+        ref = lib.uno_verify_block(None, None, None, 0, K, V, 0, ctypes.c_uint64(0),
+                                   ctypes.c_uint64(0), None, None, None, None, None, None, 0,
+                                   None)
+        assert ref == st

@@ -82,3 +82,31 @@ def test_noalloc_rejects_problems_beyond_its_scratch(libs):
                                       ctypes.c_uint64(0), fake, fake, None, None, None, None)
     assert lib.uno_status_string(st).decode().startswith("UNO_ERR_SIZE")
     assert lib.uno_verify_workspace_bytes(4096, 64, 151936, 0) > (4 << 20)
+
+
+def test_noalloc_call_allocates_no_device_memory(libs):
+    """After a first call on the device (module load, symbol look-up), a call
+    changes neither the device's free memory nor PyTorch's allocations."""
+    _, lib = libs
+    v = verify_inputs(8, 6, 3001, dtype="bf16", seed=3, device=DEV)
+    out = _outputs(8, 6)
+
+    def call(step):
+        st = lib.uno_verify_block_noalloc(
+            v.p_logits.data_ptr(), v.q_logits.data_ptr(), v.draft_tokens.data_ptr(), 8, 6, 3001,
+            0, ctypes.c_uint64(5), ctypes.c_uint64(step), out[0].data_ptr(), out[1].data_ptr(),
+            out[2].data_ptr(), out[3].data_ptr(), out[4].data_ptr(),
+            torch.cuda.current_stream().cuda_stream)
+        assert st == 0, lib.uno_status_string(st).decode()
+
+    call(0)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for step in range(1, 4):
+        call(step)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert int(out[1].min().item()) >= 0
+
