@@ -8,6 +8,7 @@ and both must match the float64 oracle within the dual-path criterion
 layouts, bf16 and f32, ragged output widths and projections without y_ar.
 """
 
+import numpy as np
 import pytest
 import torch
 
@@ -94,3 +95,55 @@ def test_grouped_without_adapter_and_partial_outputs(api):
         assert torch.equal(y_drs[g], yd)
         if y_ars[g] is not None:
             assert torch.equal(y_ars[g], ya)
+
+
+def _sampled_rows(M, seed, n=64, tail=16):
+    rows = np.random.default_rng(seed).choice(M - tail, size=n, replace=False)
+    return np.sort(np.concatenate([rows, np.arange(M - tail, M)]))
+
+
+# The grouped launches the benchmark times, at their full sizes: batched decode
+# (64 x 16 = 1024 rows, q/k/v and gate/up of a Qwen3-8B-shaped layer, rank 128,
+# alpha 256) and the whole-stack step (64 x 17 = 1088 rows, every launch with
+# the row gate closing the first position of each block of 17, weights of
+# standard deviation d_in^-1/2 and Bm of 0.004).
+FULL_SIZE = [
+    ("qkv_1024", 1024, 4096, (4096, 1024, 1024), False),
+    ("gate_up_1024", 1024, 4096, (12288, 12288), False),
+    ("qkv_1088_gated", 1088, 4096, (4096, 1024, 1024), True),
+    ("o_1088_gated", 1088, 4096, (4096,), True),
+    ("gate_up_1088_gated", 1088, 4096, (12288, 12288), True),
+    ("down_1088_gated", 1088, 12288, (4096,), True),
+]
+
+
+@pytest.mark.parametrize("name,M,d_in,d_outs,gated", FULL_SIZE, ids=[c[0] for c in FULL_SIZE])
+def test_benchmarked_grouped_launches_sampled_rows(api, name, M, d_in, d_outs, gated):
+    kw = dict(w_std=d_in ** -0.5, b_std=0.004) if gated else {}
+    ds = [dualpath_inputs(M=M, d_in=d_in, d_out=o, r=128, alpha=256.0, seed=M + 11 * g + d_in,
+                          device=DEV, **kw) for g, o in enumerate(d_outs)]
+    x = ds[0].x
+    gate = None
+    g_np = None
+    if gated:
+        g_np = np.ones(M, dtype=np.uint8)
+        g_np[::17] = 0
+        gate = torch.from_numpy(g_np).to(DEV)
+    y_ars, y_drs = api.dualpath_linear_grouped(x, [d.W for d in ds], [d.A for d in ds],
+                                               [d.Bm for d in ds], [d.scale for d in ds],
+                                               gate=gate)
+    torch.cuda.synchronize()
+    rows = _sampled_rows(M, seed=M + d_in)
+    ri = torch.from_numpy(rows).to(DEV)
+    for g, d in enumerate(ds):
+        ref_ar, ref_dr, _ = oracle.dualpath_linear(
+            widen(x[ri]), widen(d.W), widen(d.A), widen(d.Bm), d.scale, round_t_to_bf16=True,
+            gate=None if g_np is None else g_np[rows])
+        assert_dualpath_close(y_ars[g][ri], ref_ar)
+        assert_dualpath_close(y_drs[g][ri], ref_dr)
+        if gated:
+            closed = torch.from_numpy(g_np == 0).to(DEV)
+            assert torch.equal(y_drs[g][closed], y_ars[g][closed])
+    assert api.device_fault_flags() == 0
+    del ds, y_ars, y_drs
+    torch.cuda.empty_cache()
