@@ -134,16 +134,30 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-// Bytes of one ring stage per CTA: a 128-row box of the A side and the B
-// rows this CTA holds (all BN, or half of them with the CTA pair).
+// Bytes of one K-block per CTA: a 128-row box of the A side and the B rows
+// this CTA holds (all BN, or half of them with the CTA pair).
+template <int BN, bool PAIR>
+__host__ __device__ constexpr int kblock_bytes() {
+  return (kBM + (PAIR ? BN / 2 : BN)) * kRowBytes;
+}
+
+// K-blocks per ring item. Every item costs its MMA issuer a wait on the
+// item's data, a hand-over and a commit, and its producer a wait for the
+// stage; the CTA pair moves two K-blocks per item (a 64 KB stage per CTA) so
+// that these costs are paid once per 1024 cycles of tensor work, not 512.
+template <bool PAIR>
+__host__ __device__ constexpr int kblocks_per_item() {
+  return PAIR ? 2 : 1;
+}
+
 template <int BN, bool PAIR>
 __host__ __device__ constexpr int stage_bytes() {
-  return (kBM + (PAIR ? BN / 2 : BN)) * kRowBytes;
+  return kblocks_per_item<PAIR>() * kblock_bytes<BN, PAIR>();
 }
 
 template <int BN, bool PAIR>
 __host__ __device__ constexpr int stages_for() {
-  return PAIR ? 6 : (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8));
+  return PAIR ? 3 : (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8));
 }
 
 template <int BN, bool PAIR>
@@ -382,6 +396,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int STAGES = stages_for<BN, PAIR>();
   constexpr int kAbytes = kBM * kRowBytes;
   constexpr int kBrows = PAIR ? BN / 2 : BN;   // rows of W (B side) per CTA and K-block
+  constexpr int KBI = kblocks_per_item<PAIR>();  // K-blocks per ring item
+  constexpr int kKb = kblock_bytes<BN, PAIR>();   // bytes of one K-block in a stage
   constexpr int kStage = stage_bytes<BN, PAIR>();
   constexpr int kRows = PAIR ? 2 * kBM : kBM;  // output rows of a tile (both CTAs)
   constexpr bool kTf32 = sizeof(T) == 4;
@@ -426,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = p.kb_total;
   const bool adapter = p.nkb_adapt > 0;
   const int nad = adapter ? p.nkb_adapt : 0;
-  const int ins = min(kInsert, nkb);
+  constexpr int kInsertItems = (kInsert + KBI - 1) / KBI;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -524,14 +540,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     return x;
   };
-  // Ring items of local tile li: the first ins main K-blocks of tile li,
-  // the adapter K-blocks of tile li-1 (if that was a main tile other than the
-  // last: its adapter accumulates in place onto its drained y_ar), the
-  // remaining main K-blocks, and for this CTA's last tile (a main tile) its
-  // own adapter K-blocks into the other accumulator buffer, so that one drain
-  // writes both outputs.
+  // Ring items of local tile li (KBI K-blocks each, the last of a kind may
+  // hold fewer): the first main items of tile li, the adapter items of tile
+  // li-1 (if that was a main tile other than the last: its adapter
+  // accumulates in place onto its drained y_ar), the remaining main items,
+  // and for this CTA's last tile (a main tile) its own adapter items into the
+  // other accumulator buffer, so that one drain writes both outputs.
   struct Counts {
-    int nmain, nprev, nself;
+    int nmain, nprev, nself;  // K-blocks of each kind
+    int imain, iprev, iself;  // ring items of each kind
   };
   auto counts = [&](int li) {
     Counts c;
@@ -539,17 +556,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.nmain = x.kb1 - x.kb0;
     c.nprev = (li > 0 && adapter && !tile_at(li - 1).is_t) ? nad : 0;
     c.nself = (li == nmine - 1 && adapter && !x.is_t && x.piece == 0) ? nad : 0;
+    c.imain = (c.nmain + KBI - 1) / KBI;
+    c.iprev = (c.nprev + KBI - 1) / KBI;
+    c.iself = (c.nself + KBI - 1) / KBI;
     return c;
   };
   // Item q of tile li: kind (0 main, 1 previous tile's adapter, 2 own adapter)
-  // and its K-block index within that kind.
+  // and its item index j within that kind (K-blocks j * KBI onwards).
   auto item_of = [&](const Counts& c, int q) -> int2 {
-    const int head = min(ins, c.nmain);
+    const int head = min(kInsertItems, c.imain);
     if (q < head) return make_int2(0, q);
-    if (q < head + c.nprev) return make_int2(1, q - head);
-    if (q < c.nmain + c.nprev) return make_int2(0, q - c.nprev);
-    return make_int2(2, q - c.nmain - c.nprev);
+    if (q < head + c.iprev) return make_int2(1, q - head);
+    if (q < c.imain + c.iprev) return make_int2(0, q - c.iprev);
+    return make_int2(2, q - c.imain - c.iprev);
   };
+  // K-blocks in item j of a kind that has n K-blocks.
+  auto item_kbs = [&](int j, int n) { return min(KBI, n - j * KBI); };
 
   if (warp >= kFirstProducer) {
     if (lane == 0) {
@@ -562,49 +584,67 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       int t_ready = -1;  // (projection, row block) whose T this producer saw published
-      // b_rows: rows of the B box (both CTAs of a pair load the same shape;
-      // the leader expects the bytes of both).
-      auto load = [&](const CUtensorMap* ma, int ay, const CUtensorMap* mb, int by, int kx,
-                      int b_rows) {
+      // Stage of the current ring item, once it is free (null on failure).
+      // b_rows: rows of the B box; nk: K-blocks in the item (both CTAs of a
+      // pair load the same shapes; the leader expects the bytes of both).
+      uint32_t bar_pair = 0;
+      auto begin_item = [&](int b_rows, int nk) -> uint8_t* {
         const int s = it % STAGES;
         if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
           set_fault(kFaultProducer, &abort_flag);
           ok = false;
-          return;
+          return nullptr;
         }
         if (abort_flag) {
           ok = false;
-          return;
+          return nullptr;
         }
-        uint8_t* sa = smem + s * kStage;
-        const uint32_t bytes = static_cast<uint32_t>(kAbytes + b_rows * kRowBytes);
+        const uint32_t bytes = static_cast<uint32_t>(nk * (kAbytes + b_rows * kRowBytes));
         if constexpr (PAIR) {
           if (leader) sm100::mbar_arrive_expect_tx(&full_bar[s], 2 * bytes);
-          const uint32_t bar = cluster_addr(&full_bar[s], 0);
-          tma_load_2d_pair(sa, ma, bar, kx, ay);
-          tma_load_2d_pair(sa + kAbytes, mb, bar, kx, by);
+          bar_pair = cluster_addr(&full_bar[s], 0);
         } else {
           sm100::mbar_arrive_expect_tx(&full_bar[s], bytes);
+        }
+        return smem + s * kStage;
+      };
+      // The A and B boxes of one K-block, at K-block slot j of the stage.
+      auto load_kb = [&](uint8_t* stage, int j, const CUtensorMap* ma, int ay,
+                         const CUtensorMap* mb, int by, int kx) {
+        uint8_t* sa = stage + j * kKb;
+        const int s = it % STAGES;
+        if constexpr (PAIR) {
+          tma_load_2d_pair(sa, ma, bar_pair, kx, ay);
+          tma_load_2d_pair(sa + kAbytes, mb, bar_pair, kx, by);
+        } else {
           sm100::tma_load_2d(sa, ma, &full_bar[s], kx, ay);
           sm100::tma_load_2d(sa + kAbytes, mb, &full_bar[s], kx, by);
         }
       };
-      auto load_main = [&](const Tile& x, int kb_rel) {
-        const int kb = x.kb0 + kb_rel;  // K-block within d_in
-        const int kx = kb * kElemsPerRow;
-        // The CTAs of one weight tile (all row blocks of x) ask for the same
-        // K-block at about the same time; the first of them warms L2 for
-        // K-block kb + kPrefetch so that none of them waits on DRAM.
-        if constexpr (!SWAP) {
-          if (!x.is_t && x.a0 == 0 && kb + kPrefetch < nkb)
-            sm100::tma_prefetch_l2_2d(&m.w[x.g], kx + kPrefetch * kElemsPerRow, x.b0 + my_brows);
-        }
-        if (x.is_t) {
-          if constexpr (SWAP) load(&m.l[x.g], x.a0, &m.x, 0, kx, kBrows);
-          else load(&m.x, x.a0 + my_rows, &m.l[x.g], static_cast<int>(rank) * p.t_brows, kx, p.t_brows);
-        } else {
-          if constexpr (SWAP) load(&m.w[x.g], x.a0, &m.x, x.b0, kx, kBrows);
-          else load(&m.x, x.a0 + my_rows, &m.w[x.g], x.b0 + my_brows, kx, kBrows);
+      // Main item j of tile x: K-blocks x.kb0 + j * KBI onwards.
+      auto load_main = [&](const Tile& x, int j, int nk) {
+        const int b_rows = (x.is_t && !SWAP) ? p.t_brows : kBrows;
+        uint8_t* stage = begin_item(b_rows, nk);
+        if (!stage) return;
+        for (int jj = 0; jj < nk; ++jj) {
+          const int kb = x.kb0 + j * KBI + jj;  // K-block within d_in
+          const int kx = kb * kElemsPerRow;
+          // The CTAs of one weight tile (all row blocks of x) ask for the same
+          // K-block at about the same time; the first of them warms L2 for
+          // K-block kb + kPrefetch so that none of them waits on DRAM.
+          if constexpr (!SWAP) {
+            if (!x.is_t && x.a0 == 0 && kb + kPrefetch < nkb)
+              sm100::tma_prefetch_l2_2d(&m.w[x.g], kx + kPrefetch * kElemsPerRow,
+                                        x.b0 + my_brows);
+          }
+          if (x.is_t) {
+            if constexpr (SWAP) load_kb(stage, jj, &m.l[x.g], x.a0, &m.x, 0, kx);
+            else load_kb(stage, jj, &m.x, x.a0 + my_rows, &m.l[x.g],
+                         static_cast<int>(rank) * p.t_brows, kx);
+          } else {
+            if constexpr (SWAP) load_kb(stage, jj, &m.w[x.g], x.a0, &m.x, x.b0, kx);
+            else load_kb(stage, jj, &m.x, x.a0 + my_rows, &m.w[x.g], x.b0 + my_brows, kx);
+          }
         }
       };
       int last_mine = -1;  // this producer's last ring item
@@ -612,14 +652,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const Counts c = counts(li);
         const Tile cur = tile_at(li);
         const Tile prev = (li > 0) ? tile_at(li - 1) : cur;
-        const int items = c.nmain + c.nprev + c.nself;
+        const int items = c.imain + c.iprev + c.iself;
         for (int q = 0; q < items && ok; ++q, ++it) {
           if (it % kProducers != pr) continue;
           last_mine = it;
           const int2 ik = item_of(c, q);
-          const int kind = ik.x, kb = ik.y;
+          const int kind = ik.x, j = ik.y;
           if (kind == 0) {
-            load_main(cur, kb);
+            load_main(cur, j, item_kbs(j, c.nmain));
             continue;
           }
           const Tile owner = (kind == 1) ? prev : cur;
@@ -641,11 +681,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_global();
             t_ready = key;
           }
-          if constexpr (SWAP)
-            load(&m.bm[owner.g], owner.a0, &m.t[owner.g], owner.b0, kb * kElemsPerRow, kBrows);
-          else
-            load(&m.t[owner.g], owner.a0 + my_rows, &m.bm[owner.g], owner.b0 + my_brows,
-                 kb * kElemsPerRow, kBrows);
+          const int nk = item_kbs(j, nad);
+          uint8_t* stage = begin_item(kBrows, nk);
+          if (!stage) break;
+          for (int jj = 0; jj < nk; ++jj) {
+            const int kx = (j * KBI + jj) * kElemsPerRow;
+            if constexpr (SWAP)
+              load_kb(stage, jj, &m.bm[owner.g], owner.a0, &m.t[owner.g], owner.b0, kx);
+            else
+              load_kb(stage, jj, &m.t[owner.g], owner.a0 + my_rows, &m.bm[owner.g],
+                      owner.b0 + my_brows, kx);
+          }
         }
       }
       // No copy may still be landing when the CTA exits: wait for this
@@ -676,7 +722,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if constexpr (PAIR) commit_pair(bar);
         else sm100::mma_commit(bar);
       };
-      auto issue = [&](uint32_t d, uint32_t idesc, bool accumulate_first) {
+      // The MMAs of ring item `it` (nk K-blocks of 4 MMAs each); the first
+      // MMA overwrites the accumulator unless accumulate_first.
+      auto issue = [&](uint32_t d, uint32_t idesc, bool accumulate_first, int nk) {
         const int s = it % STAGES;
         if (!wait_order(order, it, &abort_flag) ||
             !sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
@@ -685,14 +733,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         sm100::tc_fence_after();
         const uint32_t sa = sm100::smem_addr(smem + s * kStage);
-        const uint64_t da = sm100::smem_desc_k_sw128(sa);
-        const uint64_t db = sm100::smem_desc_k_sw128(sa + kAbytes);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if constexpr (PAIR)
-            mma_pair<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
-          else
-            sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, accumulate_first || (k > 0));
+        for (int jj = 0; jj < KBI; ++jj) {
+          if (jj < nk) {
+            const uint64_t da = sm100::smem_desc_k_sw128(sa + jj * kKb);
+            const uint64_t db = sm100::smem_desc_k_sw128(sa + jj * kKb + kAbytes);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const bool acc = accumulate_first || (jj > 0) || (k > 0);
+              if constexpr (PAIR)
+                mma_pair<kTf32>(d, da + 2 * k, db + 2 * k, idesc, acc);
+              else
+                sm100::mma<kTf32>(d, da + 2 * k, db + 2 * k, idesc, acc);
+            }
+          }
         }
         sm100::tc_fence_before();
         st_release_shared(order, it + 1);
@@ -704,27 +758,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d = tmem + static_cast<uint32_t>(buf * kAcc);
         const uint32_t pd = tmem + static_cast<uint32_t>(pbuf * kAcc);
         const uint32_t idesc = (tile_at(li).is_t && !SWAP) ? p.idesc_t : kIdesc;
-        const int items = c.nmain + c.nprev + c.nself;
+        const int items = c.imain + c.iprev + c.iself;
         const int mo = li - 1 - nt_mine;  // main ordinal of the previous tile
         for (int q = 0; q < items && ok; ++q, ++it) {
           const bool mine = (it & 1) == e;
           const int2 ik = item_of(c, q);
-          const int kind = ik.x, kb = ik.y;
+          const int kind = ik.x, j = ik.y;
           if (kind == 1) {
             if (mine) {
-              if (kb == 0) {
+              if (j == 0) {
                 if (!wait_cl(&ar_read[mo & 1], (mo >> 1) & 1)) {
                   fail();
                   break;
                 }
                 sm100::tc_fence_after();
               }
-              issue(pd, kIdesc, true);  // adds T Bm^T onto y_ar of the previous tile
+              // adds T Bm^T onto y_ar of the previous tile
+              issue(pd, kIdesc, true, item_kbs(j, c.nprev));
             }
-            if (ok && kb == c.nprev - 1) commit(&draft_full[mo & 1]);
+            if (ok && j == c.iprev - 1) commit(&draft_full[mo & 1]);
           } else if (kind == 2) {
             if (mine) {
-              if (kb == 0 && li >= 1) {
+              if (j == 0 && li >= 1) {
                 // the other buffer is free once tile li-1 has been drained
                 if (!wait_cl(&acc_empty[pbuf], ((li - 1) >> 1) & 1)) {
                   fail();
@@ -732,21 +787,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 sm100::tc_fence_after();
               }
-              issue(pd, kIdesc, kb > 0);  // T Bm^T of this tile, on its own
+              issue(pd, kIdesc, j > 0, item_kbs(j, c.nself));  // T Bm^T of this tile, on its own
             }
-            if (ok && kb == c.nself - 1) commit(&acc_full[buf]);
+            if (ok && j == c.iself - 1) commit(&acc_full[buf]);
           } else {
             if (mine) {
-              if (kb == 0 && li >= 2) {
+              if (j == 0 && li >= 2) {
                 if (!wait_cl(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
                   fail();
                   break;
                 }
                 sm100::tc_fence_after();
               }
-              issue(d, idesc, kb > 0);
+              issue(d, idesc, j > 0, item_kbs(j, c.nmain));
             }
-            if (ok && kb == c.nmain - 1 && c.nself == 0) commit(&acc_full[buf]);
+            if (ok && j == c.imain - 1 && c.nself == 0) commit(&acc_full[buf]);
           }
         }
       }
@@ -879,6 +934,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (st_ar) rs_ar.add(sva, nvalid);
           if (st_dr) rs_dr.add(svd, nvalid);
         }
+        if ((c & 63) == 32) {
+          // a 64-column box of this warp's 32 rows is staged: store it now,
+          // so the stores overlap the rest of the drain
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            if (ya) sm100::tma_store_2d(&m.ya[gi], stage_ar + box * 4096, b0 + 64 * box, a0);
+            sm100::tma_store_2d(&m.yd[gi], stage_dr + box * 4096, b0 + 64 * box, a0);
+            sm100::bulk_commit_group();
+          }
+        }
       }
       {
         const int arow = a0 + lane;
@@ -888,17 +954,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (st_dr) st_dr[at] = make_float2(rs_dr.m, rs_dr.z);
         }
       }
-      fence_proxy_async_shared();
-      __syncwarp();
-      if (lane == 0) {
-        const int row = a0;  // first of this warp's 32 rows
-        for (int box = 0; box < BN / 64; ++box) {
-          if (ya) sm100::tma_store_2d(&m.ya[gi], stage_ar + box * 4096, b0 + 64 * box, row);
-          sm100::tma_store_2d(&m.yd[gi], stage_dr + box * 4096, b0 + 64 * box, row);
-        }
-        sm100::bulk_commit_group();
-        sm100::bulk_wait_group_0();
-      }
+      // the staging buffers must stay intact until the stores have read them
+      if (lane == 0) sm100::bulk_wait_group_read_0();
       __syncwarp();
     };
     auto drain2 = [&](uint32_t acc, uint32_t adp, int a0, int b0) {

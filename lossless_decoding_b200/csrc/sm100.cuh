@@ -108,6 +108,13 @@ __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// Wait until every committed bulk group of this thread has finished reading
+// its shared-memory source (the global writes may still be in flight; they
+// are complete when the grid is).
+__device__ __forceinline__ void bulk_wait_group_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Wait until every committed bulk group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_group_0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
