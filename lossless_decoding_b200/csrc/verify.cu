@@ -8,24 +8,32 @@
 // from the verifier), with the standard speculative accept rule
 // u < p(x)/q(x) and residual max(0, p - q) that the pages cite.
 //
-// Three launches per call; no CTA ever waits for another:
+// Two launches per call; no CTA ever waits for another:
 //  1. verify_stream_kernel streams every logit row once. One CTA per slab
 //     (up to 256 KB of one row, a whole number of 16 KB rounds) issues 16-byte
 //     loads, four per thread in flight plus the next four prefetched, folds
 //     them into a running (reference, sum of 2^(x - reference)) in the log2
 //     domain and writes one partial per slab. Nothing else happens on this
 //     path.
-//  2. verify_decide_kernel, one CTA per sequence, merges the slab partials of
-//     the sequence's 2K+1 rows in slab order, evaluates the accept tests with
-//     Philox uniforms, finds the first rejection by ballot and records what the
-//     draw needs (which rows, their statistics).
-//  3. verify_draw_kernel runs SD CTAs per sequence; each sums the residual
-//     weights max(0, p_n - q_n) (or the bonus row p_K) over its range of
-//     fixed-size vocabulary chunks with 16-byte loads. The CTA that completes a
-//     sequence (atomic counter) takes the float64 running sum of the chunk
-//     sums, finds the chunk where u' * total is crossed, scans it with warp
-//     prefix sums to pick the token and writes the outputs.
-#include <atomic>
+//  2. verify_draw_kernel runs SD CTAs per sequence. Each first decides the
+//     sequence (the same decision in every one of them, so that none waits for
+//     another): it merges the slab partials of the sequence's 2K+1 rows,
+//     evaluates the accept tests with Philox uniforms and finds the first
+//     rejection by ballot. It then sums, over its range of fixed-size
+//     vocabulary chunks, the weights of the final draw -- the residual
+//     max(0, p_n - q_n) or the bonus row p_K -- with 16-byte loads. The CTA
+//     that completes a sequence (atomic counter) takes the running sum of the
+//     chunk sums, finds the chunk where u' * total is crossed, scans it token
+//     by token and writes the outputs.
+// With the LM head's row statistics (uno_verify_block_head) the stream launch
+// is replaced by verify_decide_kernel, one CTA per sequence, which merges the
+// head's per-tile partials, decides and records the decision for the draw.
+//
+// Precision of the draw: a token's weight is 2^(x log2 e - L) on the SFU, L
+// the row's log2-sum-exp from the decision (two floats) and the argument
+// formed by FMAs with log2 e in two parts, so its error is three float32
+// roundings of the argument; a vector's weights are summed in float32, all
+// longer sums in float64.
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -49,7 +57,7 @@ constexpr int kMaxK = 256;
 constexpr int kMaxRows = 2 * kMaxK + 1;
 constexpr int kChunkMin = 256;            // vocabulary entries per inverse-CDF chunk
 constexpr int kMaxChunks = 4096;          // chunks per row (the chunk length grows beyond)
-constexpr int kDrawCtasPerSm = 2;
+constexpr int kDrawCtasPerSm = 3;
 constexpr int kDrawCtasTarget = 148 * kDrawCtasPerSm;  // one wave of draw CTAs
 constexpr int kSizingSms = 148;           // fixed, so the workspace size is device-independent
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,8 +73,8 @@ struct __align__(16) Decision {
   int n;        // first rejected position (K: all accepted)
   int invalid;  // a draft id was out of range
   int mode;     // 0: residual max(0, p_n - q_n); 1: the row p_n itself
-  float mp, izp, mq, izq;  // draw rows: reference (log2 domain) and 1 / sum
-  float c;                 // residual sign threshold (log2 domain)
+  int pad;
+  double lp, lq;  // log2-sum-exp of the draw rows (lq unused in mode 1)
 };
 
 struct VerifyParams {
@@ -84,10 +92,10 @@ struct VerifyParams {
   float* p_at_draft;
   float* q_at_draft;
   float* row_lse;
-  Partial* partials;  // [B][2K+1][S]
-  float* chunk_sums;  // [B][nchunks]
-  int* draw_count;    // [B], set to 0 by the decision launch
-  Decision* decisions;  // [B]
+  Partial* partials;    // [B][2K+1][S]
+  double* chunk_sums;   // [B][nchunks] draw-weight sums of the chunks
+  int* draw_count;      // [B], set to 0 before the draw launch
+  Decision* decisions;  // [B] (the LM-head path: written by the decision launch)
   // Rows of q per sequence in memory: K (q is [B][K][V]) or K+1 (q is the
   // draft-pathway output of the same B x (K+1) rows as p, bonus rows unused).
   int q_rows = 0;
@@ -307,145 +315,33 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     m = (lane < kWarps) ? red_m[lane] : -INFINITY;
     z = (lane < kWarps) ? red_z[lane] : 0.f;
     warp_merge(m, z);
-    if (lane == 0) P.partials[static_cast<size_t>(blockIdx.x)] = Partial{m, z};
-  }
-}
-
-// ---- launch 2: decision and draw ----------------------------------------------------------
-
-using DrawRows = Decision;
-
-// Weight of token v. mode 0: max(0, p(v) - q(v)), skipping both exponentials
-// where the log-domain test shows p(v) < q(v) by a clear margin; mode 1: p(v).
-template <typename T>
-__device__ __forceinline__ float weight(const DrawRows& d, const T* rp, const T* rq, int v) {
-  const float lp = Elem<T>::at(rp, v) * kLog2e;
-  if (d.mode) return uno::ex2(lp - d.mp) * d.izp;
-  const float lq = Elem<T>::at(rq, v) * kLog2e;
-  if (lp - lq < d.c - 1e-3f) return 0.f;
-  const float pv = uno::ex2(lp - d.mp) * d.izp;
-  const float qv = uno::ex2(lq - d.mq) * d.izq;
-  return fmaxf(0.f, pv - qv);
-}
-
-// Sums of chunks c0 + w0, c0 + w0 + wstep, ... (< c1) of the draw rows of
-// sequence b, one warp per chunk, stored to the workspace. Returns this lane's
-// largest positive-weight index, or -1. When both rows are 16-byte aligned and
-// V and the chunk length are whole vectors, each lane loads 16-byte vectors,
-// all of the warp's chunks at once; otherwise it falls back to scalar loads.
-template <typename T>
-__device__ int chunk_sums(const VerifyParams& P, int b, const DrawRows& d, const T* rp,
-                          const T* rq, int c0, int c1, int w0, int wstep) {
-  constexpr int kVec = Elem<T>::kVec;
-  constexpr int kMaxVecs = 8;  // vectors per lane held in flight per row
-  const int lane = threadIdx.x & 31;
-  int last = -1;
-  const int vpl = P.chunk_len / (32 * kVec);  // vectors per lane per chunk
-  const bool vec_ok = ((reinterpret_cast<uintptr_t>(rp) | reinterpret_cast<uintptr_t>(rq)) & 15) == 0 &&
-                      (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0 && vpl >= 1 &&
-                      vpl <= kMaxVecs;
-  if (vec_ok) {
-    const uint4* vp = reinterpret_cast<const uint4*>(rp);
-    const uint4* vq = reinterpret_cast<const uint4*>(rq);
-    const int cvec = P.chunk_len / kVec;  // vectors per chunk
-    const int nvec_row = P.V / kVec;      // vectors per row (V is a multiple of kVec here)
-    // Each pass covers up to kMaxVecs (chunk, vector) pairs per lane: all loads
-    // of a pass are issued before any is used.
-    const int per_pass_chunks = max(1, kMaxVecs / vpl);
-    for (int cb = c0 + w0; cb < c1; cb += wstep * per_pass_chunks) {
-      uint4 a[kMaxVecs], bq[kMaxVecs];
-#pragma unroll
-      for (int k = 0; k < kMaxVecs; ++k) {
-        const int c = cb + (k / vpl) * wstep;
-        const int q = k % vpl;
-        const int vi = c * cvec + q * 32 + lane;
-        const bool in = (k < per_pass_chunks * vpl) && (c < c1) && (q < vpl) && (vi < nvec_row);
-        a[k] = in ? __ldg(vp + vi) : make_uint4(0, 0, 0, 0);
-        bq[k] = (in && d.mode == 0) ? __ldg(vq + vi) : make_uint4(0, 0, 0, 0);
-      }
-      float s[kMaxVecs / 1];
-#pragma unroll
-      for (int k = 0; k < kMaxVecs; ++k) {
-        const int c = cb + (k / vpl) * wstep;
-        const int q = k % vpl;
-        s[k] = 0.f;
-        const int vi = c * cvec + q * 32 + lane;
-        if (!((k < per_pass_chunks * vpl) && (c < c1) && (q < vpl) && (vi < nvec_row))) continue;
-        float fp[kVec], fq[kVec];
-        Elem<T>::unpack(a[k], fp);
-        Elem<T>::unpack(bq[k], fq);
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) {
-          float w;
-          const float lp = fp[e] * kLog2e;
-          if (d.mode) {
-            w = uno::ex2(lp - d.mp) * d.izp;
-          } else {
-            const float lq = fq[e] * kLog2e;
-            w = (lp - lq < d.c - 1e-3f)
-                    ? 0.f
-                    : fmaxf(0.f, uno::ex2(lp - d.mp) * d.izp - uno::ex2(lq - d.mq) * d.izq);
-          }
-          s[k] += w;
-          if (w > 0.f) last = max(last, vi * kVec + e);
-        }
-      }
-      // one sum per chunk of this pass
-#pragma unroll
-      for (int k0 = 0; k0 < kMaxVecs; k0 += 1) {
-        if (k0 % vpl != 0 || k0 >= per_pass_chunks * vpl) continue;
-        float t = 0.f;
-        for (int q = 0; q < vpl && k0 + q < kMaxVecs; ++q) t += s[k0 + q];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
-        const int c = cb + (k0 / vpl) * wstep;
-        if (lane == 0 && c < c1) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = t;
-      }
+    if (lane == 0) {
+      P.partials[static_cast<size_t>(blockIdx.x)] = Partial{m, z};
+      // the draw launch counts its CTAs of this sequence from 0
+      if (j == 0 && s == 0) P.draw_count[b] = 0;
     }
-    return last;
   }
-  for (int c = c0 + w0; c < c1; c += wstep) {
-    const int v0 = c * P.chunk_len;
-    const int v1 = min(v0 + P.chunk_len, P.V);
-    float s = 0.f;
-    for (int base = v0; base < v1; base += 32 * 8) {
-      float w[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int v = base + k * 32 + lane;
-        w[k] = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        s += w[k];
-        if (w[k] > 0.f) last = max(last, base + k * 32 + lane);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (lane == 0) P.chunk_sums[static_cast<size_t>(b) * P.nchunks + c] = s;
-  }
-  return last;
 }
 
-// ---- launch 2: the decision of each sequence (one CTA per sequence) ---------------------
+// ---- the decision of one sequence (a whole CTA) ------------------------------------
 
 struct DecideShared {
   float row_m[kMaxRows], row_z[kMaxRows];
   int first_reject, invalid;
+  Decision d;
 };
 
+// Merges the row statistics of sequence b (the slab partials, or the LM head's
+// tile partials when P.ext_p is set), runs the K accept tests, finds the first
+// rejection and leaves the decision in sh.d. With `outputs`, also writes
+// row_lse, p/q at the drafts and the outputs of a sequence with an invalid
+// draft id (the draw writes the others).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyParams P) {
-  __shared__ DecideShared sh;
-  uno::launch_dependents();
-  uno::grid_dependency_wait();
+__device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, bool outputs) {
   const int tid = threadIdx.x;
-  const int b = blockIdx.x;
-  const int K = P.K, R = 2 * K + 1, S = P.S, V = P.V;
-
-  // row statistics: merge the slab partials of every row in slab order
+  const int K = P.K, R = 2 * K + 1, V = P.V;
   if (P.ext_p == nullptr) {
+    const int S = P.S;
     for (int j = tid; j < R; j += kThreads) {
       const Partial* pp = P.partials + (static_cast<size_t>(b) * R + j) * S;
       float m = -INFINITY, z = 0.f;
@@ -458,7 +354,6 @@ __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyPar
       }
       sh.row_m[j] = m;
       sh.row_z[j] = z;
-      if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
     }
   } else {
     // the LM head's column-tile partials (hundreds per row): one warp per row,
@@ -479,25 +374,21 @@ __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyPar
 #pragma unroll
         for (int k = 0; k < 4; ++k) merge(m, z, v[k].m, v[k].z);
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-        const float z2 = __shfl_xor_sync(0xFFFFFFFFu, z, o);
-        merge(m, z, m2, z2);
-      }
+      warp_merge(m, z);
       if (lane == 0) {
         sh.row_m[j] = m;
         sh.row_z[j] = z;
-        if (P.row_lse) P.row_lse[static_cast<size_t>(b) * R + j] = (m + log2f(z)) * kLn2;
       }
     }
   }
   if (tid == 0) {
     sh.first_reject = K;
     sh.invalid = 0;
-    P.draw_count[b] = 0;
   }
   __syncthreads();
+  if (outputs && P.row_lse)
+    for (int j = tid; j < R; j += kThreads)
+      P.row_lse[static_cast<size_t>(b) * R + j] = (sh.row_m[j] + log2f(sh.row_z[j])) * kLn2;
 
   // accept tests, one thread per position; first rejection by ballot
   for (int i0 = 0; i0 < K; i0 += kThreads) {
@@ -516,8 +407,8 @@ __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyPar
                          sh.row_z[K + 1 + i];
         const uint4 w = uno::verify_block_words(P.seed, P.step, b, i);
         rejected = !(uno::uniform24(w.x) * qq < pp);
-        if (P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
-        if (P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
+        if (outputs && P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
+        if (outputs && P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
       }
     }
     const unsigned ballot = __ballot_sync(0xFFFFFFFFu, rejected);
@@ -526,29 +417,155 @@ __global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyPar
   }
   __syncthreads();
   const int n = sh.first_reject;
-  if (sh.invalid) {
+  if (outputs && sh.invalid) {
     int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
     for (int i = tid; i <= K; i += kThreads) out[i] = -1;
+    if (tid == 0) P.accepted_len[b] = -1;
   }
   if (tid == 0) {
     Decision d{};
     d.n = n;
     d.invalid = sh.invalid;
     d.mode = (n < K) ? 0 : 1;
-    d.mp = sh.row_m[n];
-    d.izp = 1.f / sh.row_z[n];
-    if (n < K) {
-      d.mq = sh.row_m[K + 1 + n];
-      d.izq = 1.f / sh.row_z[K + 1 + n];
-      d.c = (sh.row_m[n] + log2f(sh.row_z[n])) -
-            (sh.row_m[K + 1 + n] + log2f(sh.row_z[K + 1 + n]));
-    }
-    P.decisions[b] = d;
-    if (sh.invalid) P.accepted_len[b] = -1;
+    d.lp = static_cast<double>(sh.row_m[n]) + static_cast<double>(log2f(sh.row_z[n]));
+    // a q row with no finite logit has q = 0 everywhere: max(0, p - q) = p
+    if (n < K && !(sh.row_z[K + 1 + n] > 0.f)) d.mode = 1;
+    if (d.mode == 0)
+      d.lq = static_cast<double>(sh.row_m[K + 1 + n]) +
+             static_cast<double>(log2f(sh.row_z[K + 1 + n]));
+    sh.d = d;
+  }
+  __syncthreads();
+}
+
+// The LM-head path: one CTA per sequence decides and records the decision.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) verify_decide_kernel(const VerifyParams P) {
+  __shared__ DecideShared sh;
+  uno::launch_dependents();
+  uno::grid_dependency_wait();
+  decide_sequence<T>(P, blockIdx.x, sh, true);
+  if (threadIdx.x == 0) {
+    P.decisions[blockIdx.x] = sh.d;
+    P.draw_count[blockIdx.x] = 0;
   }
 }
 
-// ---- launch 3: the draw -------------------------------------------------------------------
+// ---- launch 2: the draw -------------------------------------------------------------------
+
+// log2(e) as a float32 and the float32 of its remainder.
+constexpr float kLog2eHi = 1.44269502162933349609375f;
+constexpr float kLog2eLo = 1.925963033500011e-08f;
+
+// The row's log2-sum-exp L as two floats, L = hi + lo to float64 accuracy.
+struct SplitL {
+  float hi, lo;
+};
+__device__ __forceinline__ SplitL split_l(double L) {
+  SplitL v;
+  v.hi = static_cast<float>(L);
+  v.lo = static_cast<float>(L - static_cast<double>(v.hi));
+  return v;
+}
+
+// Exponent argument l log2 e - L of a token in float32 (three roundings, each
+// at most 2^-24 of |argument|, and no error from log2 e itself).
+__device__ __forceinline__ float arg_of(float l, SplitL L) {
+  return fmaf(l, kLog2eLo, fmaf(l, kLog2eHi, -L.hi)) - L.lo;
+}
+
+// Weight of a token: mode 0: max(0, p - q), both exponentials skipped when
+// p <= q; mode 1: p. p = 2^(arg_p) on the SFU, the row's normalised
+// probability (up to the streaming pass's float32 normaliser).
+__device__ __forceinline__ float token_weight(int mode, SplitL Lp, SplitL Lq, float lp, float lq) {
+  const float ap = arg_of(lp, Lp);
+  if (mode) return uno::ex2(ap);
+  const float aq = arg_of(lq, Lq);
+  if (!(ap > aq)) return 0.f;
+  return fmaxf(0.f, uno::ex2(ap) - uno::ex2(aq));
+}
+
+// Chunk sums of chunks c0 + w0, c0 + w0 + wstep, ... (< c1) of the draw rows,
+// one warp per chunk: the vector path, VPL 16-byte vectors per lane and chunk,
+// kMaxVecs (chunk, vector) pairs per lane in flight per row, all loads of a
+// pass issued before any is used. A vector's weights are added in float32 as
+// a balanced tree, vectors and lanes in float64.
+template <typename T, int VPL>
+__device__ void chunk_sums_vec(const VerifyParams& P, const Decision& d, const T* rp, const T* rq,
+                               double* out, int c0, int c1, int w0, int wstep) {
+  constexpr int kVec = Elem<T>::kVec;
+  constexpr int kMaxVecs = 4;
+  constexpr int kPerPass = kMaxVecs / VPL;  // chunks per pass
+  const int lane = threadIdx.x & 31;
+  const uint4* vp = reinterpret_cast<const uint4*>(rp);
+  const uint4* vq = reinterpret_cast<const uint4*>(rq);
+  const int cvec = P.chunk_len / kVec;  // vectors per chunk
+  const int nvec_row = P.V / kVec;      // vectors per row (the last chunk may be partial)
+  const SplitL Lp = split_l(d.lp), Lq = split_l(d.mode ? 0.0 : d.lq);
+  for (int cb = c0 + w0; cb < c1; cb += wstep * kPerPass) {
+    uint4 a[kMaxVecs], bq[kMaxVecs];
+    bool in[kMaxVecs];
+#pragma unroll
+    for (int k = 0; k < kMaxVecs; ++k) {
+      const int c = cb + (k / VPL) * wstep;
+      const int vi = c * cvec + (k % VPL) * 32 + lane;
+      in[k] = (c < c1) && (vi < nvec_row);
+      a[k] = in[k] ? __ldg(vp + vi) : make_uint4(0, 0, 0, 0);
+      bq[k] = (in[k] && d.mode == 0) ? __ldg(vq + vi) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int ci = 0; ci < kPerPass; ++ci) {
+      const int c = cb + ci * wstep;
+      double t = 0.0;
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) {
+        if (!in[ci * VPL + q]) continue;
+        float fp[kVec], fq[kVec], w[kVec];
+        Elem<T>::unpack(a[ci * VPL + q], fp);
+        Elem<T>::unpack(bq[ci * VPL + q], fq);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) w[e] = token_weight(d.mode, Lp, Lq, fp[e], fq[e]);
+#pragma unroll
+        for (int st = 1; st < kVec; st *= 2) {
+#pragma unroll
+          for (int e = 0; e + st < kVec; e += 2 * st) w[e] += w[e + st];
+        }
+        t += w[0];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+      if (lane == 0 && c < c1) out[c] = t;
+    }
+  }
+}
+
+// Chunk sums of chunks c0 + w0, c0 + w0 + wstep, ... (< c1): 16-byte vectors
+// when both rows are 16-byte aligned and V and the chunk length are whole
+// vectors, otherwise scalar loads.
+template <typename T>
+__device__ void chunk_sums(const VerifyParams& P, int b, const Decision& d, const T* rp,
+                           const T* rq, int c0, int c1, int w0, int wstep) {
+  constexpr int kVec = Elem<T>::kVec;
+  const int lane = threadIdx.x & 31;
+  double* out = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
+  const int vpl = P.chunk_len / (32 * kVec);  // vectors per lane per chunk
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(rp) | reinterpret_cast<uintptr_t>(rq)) & 15) == 0 &&
+                      (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0;
+  if (vec_ok && vpl == 1) return chunk_sums_vec<T, 1>(P, d, rp, rq, out, c0, c1, w0, wstep);
+  if (vec_ok && vpl == 2) return chunk_sums_vec<T, 2>(P, d, rp, rq, out, c0, c1, w0, wstep);
+  if (vec_ok && vpl == 4) return chunk_sums_vec<T, 4>(P, d, rp, rq, out, c0, c1, w0, wstep);
+  const SplitL Lp = split_l(d.lp), Lq = split_l(d.mode ? 0.0 : d.lq);
+  for (int c = c0 + w0; c < c1; c += wstep) {
+    const int v0 = c * P.chunk_len;
+    const int v1 = min(v0 + P.chunk_len, P.V);
+    double acc = 0.0;
+    for (int v = v0 + lane; v < v1; v += 32)
+      acc += token_weight(d.mode, Lp, Lq, Elem<T>::at(rp, v), d.mode ? 0.f : Elem<T>::at(rq, v));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if (lane == 0) out[c] = acc;
+  }
+}
 
 struct DrawShared {
   double warp_tot[kWarps];
@@ -576,39 +593,40 @@ __device__ double block_exclusive_scan(double mine, DrawShared& sh) {
   return before + incl - mine;
 }
 
+template <typename T>
+__device__ __forceinline__ double weight_at(const Decision& d, SplitL Lp, SplitL Lq, const T* rp,
+                                            const T* rq, int v) {
+  return token_weight(d.mode, Lp, Lq, Elem<T>::at(rp, v), d.mode ? 0.f : Elem<T>::at(rq, v));
+}
+
 // Largest index with positive weight in chunk c (the whole CTA), or -1.
 template <typename T>
-__device__ int last_positive_in_chunk(const VerifyParams& P, const DrawRows& d, const T* rp,
+__device__ int last_positive_in_chunk(const VerifyParams& P, const Decision& d, const T* rp,
                                       const T* rq, int c, DrawShared& sh) {
+  const SplitL Lp = split_l(d.lp), Lq = split_l(d.mode ? 0.0 : d.lq);
   if (threadIdx.x == 0) sh.last_in_chunk = -1;
   __syncthreads();
   const int v0 = c * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
   for (int v = v0 + threadIdx.x; v < v1; v += kThreads)
-    if (weight<T>(d, rp, rq, v) > 0.f) atomicMax(&sh.last_in_chunk, v);
+    if (weight_at<T>(d, Lp, Lq, rp, rq, v) > 0.0) atomicMax(&sh.last_in_chunk, v);
   __syncthreads();
   return sh.last_in_chunk;
 }
 
 // Final inverse-CDF step of sequence b (the whole CTA); returns the token.
-// Thread t holds the sums of chunks [t * per, (t + 1) * per) in registers.
+// Thread t takes the sums of chunks [t * per, (t + 1) * per) (read twice).
 template <typename T>
-__device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp, const T* rq,
+__device__ int finish_draw(const VerifyParams& P, int b, Decision d, const T* rp, const T* rq,
                            DrawShared& sh) {
-  constexpr int kMaxPer = kMaxChunks / kThreads;
   const int tid = threadIdx.x;
-  float* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
+  const double* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
   const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, d.n).y);
   const int per = (P.nchunks + kThreads - 1) / kThreads;
-  const int c0 = tid * per;
-  float mine_cs[kMaxPer];
-  double mine = 0.0, before = 0.0;
+  const int c0 = min(tid * per, P.nchunks), c1 = min(c0 + per, P.nchunks);
+  double before = 0.0;
   for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k)
-      mine_cs[k] = (k < per && c0 + k < P.nchunks) ? __ldcg(cs + c0 + k) : 0.f;
-    mine = 0.0;
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) mine += static_cast<double>(mine_cs[k]);
+    double mine = 0.0;
+    for (int c = c0; c < c1; ++c) mine += __ldcg(cs + c);
     before = block_exclusive_scan(mine, sh);
     if (sh.total > 0.0 || d.mode == 1) break;
     // The residual mass is zero (possible only through rounding): draw from p_n.
@@ -629,14 +647,12 @@ __device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp
   {
     double run = before;
     int found = -1, last_pos_chunk = -1;
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-      if (k < per && c0 + k < P.nchunks) {
-        const double nxt = run + static_cast<double>(mine_cs[k]);
-        if (found < 0 && nxt > t) found = c0 + k;
-        if (mine_cs[k] > 0.f) last_pos_chunk = c0 + k;
-        if (found < 0) run = nxt;
-      }
+    for (int c = c0; c < c1; ++c) {
+      const double w = __ldcg(cs + c);
+      const double nxt = run + w;
+      if (found < 0 && nxt > t) found = c;
+      if (w > 0.0) last_pos_chunk = c;
+      if (found < 0) run = nxt;
     }
     if (found >= 0) atomicMin(&sh.chunk, found);
     if (last_pos_chunk >= 0) atomicMax(&sh.last_chunk, last_pos_chunk);
@@ -649,14 +665,18 @@ __device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp
     // Rounding left no crossing: the largest index with positive weight.
     return (sh.last_chunk >= 0) ? last_positive_in_chunk<T>(P, d, rp, rq, sh.last_chunk, sh) : -1;
   }
+  // Within the chunk, token by token from the running sum before it; if the
+  // chunk's weights end before the threshold (summation order), its last
+  // token with positive weight is taken.
+  const SplitL Lp = split_l(d.lp), Lq = split_l(d.mode ? 0.0 : d.lq);
   double carry = sh.carry;
   const int v0 = ch * P.chunk_len, v1 = min(v0 + P.chunk_len, P.V);
   for (int base = v0; base < v1; base += kThreads) {
     const int v = base + tid;
-    const float w = (v < v1) ? weight<T>(d, rp, rq, v) : 0.f;
-    const double bef = carry + block_exclusive_scan(static_cast<double>(w), sh);
-    if ((w > 0.f) && (bef + static_cast<double>(w) > t)) atomicMin(&sh.token_min, v);
-    if (w > 0.f) atomicMax(&sh.last_in_chunk, v);
+    const double w = (v < v1) ? weight_at<T>(d, Lp, Lq, rp, rq, v) : 0.0;
+    const double bef = carry + block_exclusive_scan(w, sh);
+    if ((w > 0.0) && (bef + w > t)) atomicMin(&sh.token_min, v);
+    if (w > 0.0) atomicMax(&sh.last_in_chunk, v);
     carry += sh.total;
     __syncthreads();
     if (sh.token_min != INT_MAX) break;
@@ -664,16 +684,26 @@ __device__ int finish_draw(const VerifyParams& P, int b, DrawRows d, const T* rp
   return (sh.token_min != INT_MAX) ? sh.token_min : sh.last_in_chunk;
 }
 
-template <typename T>
+// DECIDE: each CTA decides its sequence from the slab partials (the first of
+// a sequence's CTAs also writes the decision's outputs); otherwise the
+// decision launch recorded it.
+template <typename T, bool DECIDE>
 __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(const VerifyParams P) {
   __shared__ DrawShared sh;
+  __shared__ DecideShared dsh;
   uno::launch_dependents();
   uno::grid_dependency_wait();
   const int tid = threadIdx.x, warp = tid >> 5;
   const int b = blockIdx.x / P.SD, du = blockIdx.x % P.SD;
   const int K = P.K;
-  const Decision d = P.decisions[b];
-  if (d.invalid) return;  // the decision launch wrote this sequence's outputs
+  if constexpr (DECIDE) {
+    decide_sequence<T>(P, b, dsh, du == 0);
+  } else {
+    if (tid == 0) dsh.d = P.decisions[b];
+    __syncthreads();
+  }
+  const Decision d = dsh.d;
+  if (d.invalid) return;  // the decision wrote this sequence's outputs
   size_t off;
   const T* rp = row_ptr<T>(P, b, d.n, &off);
   const T* rq = (d.mode == 0) ? row_ptr<T>(P, b, K + 1 + d.n, &off) : rp;
@@ -747,7 +777,7 @@ Geometry geometry(int B, int K, int V, int dtype) {
   g.off_partials = align_up(g.off_decisions + sizeof(Decision) * static_cast<size_t>(B), 256);
   g.off_chunks =
       align_up(g.off_partials + sizeof(Partial) * static_cast<size_t>(g.stream_ctas), 256);
-  g.bytes = align_up(g.off_chunks + sizeof(float) * static_cast<size_t>(B) * g.nchunks, 256);
+  g.bytes = align_up(g.off_chunks + sizeof(double) * static_cast<size_t>(B) * g.nchunks, 256);
   return g;
 }
 
@@ -770,11 +800,13 @@ int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P
 
 template <typename T>
 int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
-  if (P.ext_p == nullptr &&
-      launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK)
-    return UNO_ERR_CUDA;
-  if (launch_pdl(verify_decide_kernel<T>, P.B, st, P) != UNO_OK) return UNO_ERR_CUDA;
-  if (launch_pdl(verify_draw_kernel<T>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  if (P.ext_p == nullptr) {
+    if (launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+    if (launch_pdl(verify_draw_kernel<T, true>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  } else {
+    if (launch_pdl(verify_decide_kernel<T>, P.B, st, P) != UNO_OK) return UNO_ERR_CUDA;
+    if (launch_pdl(verify_draw_kernel<T, false>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+  }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
@@ -831,7 +863,7 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.draw_count = reinterpret_cast<int*>(ws + g.off_counts);
   P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
   P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
-  P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
+  P.chunk_sums = reinterpret_cast<double*>(ws + g.off_chunks);
   P.q_rows = K;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return (dtype == UNO_BF16) ? launch<uint16_t>(P, g, st) : launch<float>(P, g, st);
@@ -887,7 +919,7 @@ extern "C" int uno_verify_block_head(const void* y_ar, const void* y_draft, cons
   P.draw_count = reinterpret_cast<int*>(ws + g.off_counts);
   P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
   P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
-  P.chunk_sums = reinterpret_cast<float*>(ws + g.off_chunks);
+  P.chunk_sums = reinterpret_cast<double*>(ws + g.off_chunks);
   P.q_rows = K + 1;
   P.ext_p = reinterpret_cast<const Partial*>(stats_ar);
   P.ext_q = reinterpret_cast<const Partial*>(stats_draft);

@@ -247,7 +247,9 @@ def verify_block_u(p_logits, q_logits, draft_tokens, u_acc, u_smp):
     ``row_lse`` [B, 2K+1] (p rows 0..K, then q rows 0..K-1), ``ratio``
     [B, K] = p/q at the drafts (inf where q = 0), ``accept`` [B, K] bool,
     and the draw's CDF boundaries ``cdf_prev``, ``cdf_at``, ``cdf_t``,
-    ``cdf_total`` [B] (reading 4).
+    ``cdf_total`` [B] (reading 4), with ``cdf_qres`` [B] = the q mass on the
+    residual's support, sum of q_n(v) over v with p_n(v) > q_n(v) (0 when the
+    draw uses a p row): a diagnostic for comparisons, not part of the method.
     """
     p_logits = np.asarray(p_logits, dtype=np.float64)
     q_logits = np.asarray(q_logits, dtype=np.float64)
@@ -278,6 +280,8 @@ def verify_block_u(p_logits, q_logits, draft_tokens, u_acc, u_smp):
     use_p_row = np.where(n == K, K, n)
     weights = np.where(((n == K) | resid_empty)[:, None], P[rows, use_p_row, :], resid)
     y, c_prev, c_at, c_t, c_tot = _inverse_cdf(weights, u_smp[rows, n])
+    p_n, q_n = P[rows, n_row, :], Q[rows, n_row, :]
+    q_res = np.where((n < K) & ~resid_empty, np.sum(np.where(p_n > q_n, q_n, 0.0), axis=1), 0.0)
 
     out = np.full((B, K + 1), -1, dtype=np.int64)
     cols = np.arange(K + 1)[None, :]
@@ -305,6 +309,7 @@ def verify_block_u(p_logits, q_logits, draft_tokens, u_acc, u_smp):
         "cdf_at": c_at,
         "cdf_t": c_t,
         "cdf_total": c_tot,
+        "cdf_qres": q_res,
     }
 
 

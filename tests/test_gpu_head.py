@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from lossless_decoding_b200.inputs import dualpath_inputs
-from tests.parity import VerifyReport, compare_verify, widen
+from tests.parity import VerifyReport, compare_verify, report, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -126,16 +126,16 @@ def _check_head_verify(api, B, K, V, d_in, dtype, seed, step, n_check=None, sigm
 def test_verify_head_parity(api, B, K, V, d_in, dtype):
     for seed, step in ((5, 0), (41, 9)):
         rep = _check_head_verify(api, B, K, V, d_in, dtype, seed, step)
-        assert rep.compared >= B // 2
+        report(f"LM head B={B} K={K} V={V} {dtype} seed={seed}", rep)
+        assert rep.compared >= int(np.ceil(0.9 * B)) - 1
 
 
 def test_verify_head_qwen3_lm_head(api):
     """The LM head of the batched step: 64 blocks of 17 rows, 4096 -> 151936,
-    bf16; the oracle checks 24 sequences. Over 151936 tokens the final draw
-    often lands within the tie band of a CDF boundary (the band exceeds a
-    typical token's mass), so a good part is counted rather than compared;
-    every compared sequence must match."""
-    rep = _check_head_verify(api, 64, 16, 151936, 4096, "bf16", seed=7, step=3, n_check=24,
+    bf16; the oracle checks 32 sequences, and at least 90% of them (less one)
+    must be compared token for token outside the derived near-tie band."""
+    rep = _check_head_verify(api, 64, 16, 151936, 4096, "bf16", seed=7, step=3, n_check=32,
                              sigma_w=0.03)
-    assert rep.compared >= 6
+    report("LM head B=64 K=16 V=151936 bf16", rep)
+    assert rep.compared >= 28, f"only {rep.compared} of 32 sequences compared"
     assert api.device_fault_flags() == 0

@@ -13,7 +13,7 @@ from scipy import stats
 
 import oracle
 from lossless_decoding_b200.inputs import verify_inputs
-from tests.parity import VerifyReport, compare_verify, widen
+from tests.parity import VerifyReport, compare_verify, report, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -191,15 +191,27 @@ def _sampled_full_size(api, B, K, V, dtype, dist, sigma, n_check, seed, step):
     return rep
 
 
+def _floor(n: int) -> int:
+    """Sequences that must be compared token for token out of n checked. The
+    draw band of tests/parity.py leaves about 5% of full-vocabulary draws as
+    near ties: 90% for samples of 32 and more; a few sequences fewer for the
+    small samples of single sweep points (their sum is held to 90% by
+    test_parity_verifier_sweep_compares_ninety_percent)."""
+    return int(np.ceil(0.9 * n)) if n >= 32 else n - max(1, n // 4)
+
+
 @pytest.mark.parametrize("B,K,dtype,dist,sigma,n_check", [
     (1, 16, "bf16", "normal", 1.0, 1),       # Qwen3-8B single sequence
     (64, 16, "bf16", "normal", 1.0, 64),     # batched decode B=64, K=16 (full oracle)
-    (256, 32, "f32", "gumbel", 4.0, 8),      # largest sweep point (10 GB of logits)
-    (128, 8, "bf16", "gumbel", 0.25, 16),
+    (256, 32, "f32", "gumbel", 4.0, 32),     # largest sweep point (10 GB of logits)
+    (128, 8, "bf16", "gumbel", 0.25, 32),
 ])
 def test_parity_full_vocabulary(api, B, K, dtype, dist, sigma, n_check):
     rep = _sampled_full_size(api, B, K, 151936, dtype, dist, sigma, n_check, seed=B + K, step=3)
-    assert rep.compared + rep.accept_ties + rep.draw_ties == min(n_check, B)
+    n = min(n_check, B)
+    report(f"full vocabulary B={B} K={K} {dtype} {dist} sigma={sigma}", rep)
+    assert rep.compared + rep.accept_ties + rep.draw_ties == n
+    assert rep.compared >= _floor(n), f"only {rep.compared} of {n} sequences compared"
     assert api.device_fault_flags() == 0
     torch.cuda.empty_cache()
 
@@ -219,8 +231,24 @@ def _sweep_cases():
 
 @pytest.mark.parametrize("B,K,dtype,sigma", _sweep_cases())
 def test_parity_verifier_sweep(api, B, K, dtype, sigma):
-    rep = _sampled_full_size(api, B, K, 151936, dtype, "gumbel", sigma, 2, seed=7 * B + K,
+    n = min(B, 16)
+    rep = _sampled_full_size(api, B, K, 151936, dtype, "gumbel", sigma, n, seed=7 * B + K,
                              step=B + K)
-    assert rep.compared + rep.accept_ties + rep.draw_ties == min(2, B)
+    report(f"sweep B={B} K={K} {dtype} sigma={sigma}", rep)
+    assert rep.compared + rep.accept_ties + rep.draw_ties == n
+    assert rep.compared >= _floor(n), f"only {rep.compared} of {n} sequences compared"
     assert api.device_fault_flags() == 0
     torch.cuda.empty_cache()
+
+
+def test_parity_verifier_sweep_compares_ninety_percent():
+    """Over every point of the verifier sweep run in this session, at least 90%
+    of the checked sequences are compared token for token (the rest are near
+    ties of the derived band)."""
+    from tests.parity import REPORTS
+    sweep = [r for name, r in REPORTS if name.startswith("sweep ")]
+    if len(sweep) < len(_sweep_cases()):
+        pytest.skip("the sweep did not run in full in this session")
+    rows = sum(r.rows for r in sweep)
+    compared = sum(r.compared for r in sweep)
+    assert compared >= 0.9 * rows, f"{compared} of {rows} sweep sequences compared"
