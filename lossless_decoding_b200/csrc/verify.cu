@@ -55,9 +55,10 @@ constexpr int kSlabBytes = 262144;        // target bytes streamed by one CTA
 constexpr int kMinSlabBytes = kThreads * 16;
 constexpr int kMaxK = 256;
 constexpr int kMaxRows = 2 * kMaxK + 1;
+static_assert(kMaxK <= kThreads, "the decision takes one position per thread");
 constexpr int kChunkMin = 256;            // vocabulary entries per inverse-CDF chunk
 constexpr int kMaxChunks = 4096;          // chunks per row (the chunk length grows beyond)
-constexpr int kDrawCtasPerSm = 3;
+constexpr int kDrawCtasPerSm = 4;
 constexpr int kDrawCtasTarget = 148 * kDrawCtasPerSm;  // one wave of draw CTAs
 constexpr int kSizingSms = 148;           // fixed, so the workspace size is device-independent
 constexpr float kLog2e = 1.4426950408889634f;
@@ -340,6 +341,18 @@ template <typename T>
 __device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, bool outputs) {
   const int tid = threadIdx.x;
   const int K = P.K, R = 2 * K + 1, V = P.V;
+  // Thread i < K (K <= kThreads) loads draft x_i and the logits at it first,
+  // so that these loads overlap the merge of the row statistics.
+  int x = -1;
+  float lpx = 0.f, lqx = 0.f;
+  if (tid < K) {
+    x = P.draft[static_cast<size_t>(b) * K + tid];
+    if (x >= 0 && x < V) {
+      size_t off;
+      lpx = Elem<T>::at(row_ptr<T>(P, b, tid, &off), x);
+      lqx = Elem<T>::at(row_ptr<T>(P, b, K + 1 + tid, &off), x);
+    }
+  }
   if (P.ext_p == nullptr) {
     const int S = P.S;
     for (int j = tid; j < R; j += kThreads) {
@@ -391,20 +404,15 @@ __device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, 
       P.row_lse[static_cast<size_t>(b) * R + j] = (sh.row_m[j] + log2f(sh.row_z[j])) * kLn2;
 
   // accept tests, one thread per position; first rejection by ballot
-  for (int i0 = 0; i0 < K; i0 += kThreads) {
-    const int i = i0 + tid;
+  {
+    const int i = tid;
     bool rejected = false;
     if (i < K) {
-      const int x = P.draft[static_cast<size_t>(b) * K + i];
       if (x < 0 || x >= V) {
         atomicOr(&sh.invalid, 1);
       } else {
-        size_t off;
-        const T* rp = row_ptr<T>(P, b, i, &off);
-        const T* rq = row_ptr<T>(P, b, K + 1 + i, &off);
-        const float pp = uno::ex2(fmaf(Elem<T>::at(rp, x), kLog2e, -sh.row_m[i])) / sh.row_z[i];
-        const float qq = uno::ex2(fmaf(Elem<T>::at(rq, x), kLog2e, -sh.row_m[K + 1 + i])) /
-                         sh.row_z[K + 1 + i];
+        const float pp = uno::ex2(fmaf(lpx, kLog2e, -sh.row_m[i])) / sh.row_z[i];
+        const float qq = uno::ex2(fmaf(lqx, kLog2e, -sh.row_m[K + 1 + i])) / sh.row_z[K + 1 + i];
         const uint4 w = uno::verify_block_words(P.seed, P.step, b, i);
         rejected = !(uno::uniform24(w.x) * qq < pp);
         if (outputs && P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
@@ -412,8 +420,7 @@ __device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, 
       }
     }
     const unsigned ballot = __ballot_sync(0xFFFFFFFFu, rejected);
-    if (ballot && (tid & 31) == 0)
-      atomicMin(&sh.first_reject, i0 + (tid & ~31) + __ffs(ballot) - 1);
+    if (ballot && (tid & 31) == 0) atomicMin(&sh.first_reject, (tid & ~31) + __ffs(ballot) - 1);
   }
   __syncthreads();
   const int n = sh.first_reject;
@@ -623,10 +630,17 @@ __device__ int finish_draw(const VerifyParams& P, int b, Decision d, const T* rp
   const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, d.n).y);
   const int per = (P.nchunks + kThreads - 1) / kThreads;
   const int c0 = min(tid * per, P.nchunks), c1 = min(c0 + per, P.nchunks);
+  constexpr int kKeep = 4;  // a thread's chunk sums kept in registers (more are reloaded)
+  double keep[kKeep];
   double before = 0.0;
   for (int pass = 0; pass < 2; ++pass) {
     double mine = 0.0;
-    for (int c = c0; c < c1; ++c) mine += __ldcg(cs + c);
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) {
+      keep[k] = (c0 + k < c1) ? __ldcg(cs + c0 + k) : 0.0;
+      mine += keep[k];
+    }
+    for (int c = c0 + kKeep; c < c1; ++c) mine += __ldcg(cs + c);
     before = block_exclusive_scan(mine, sh);
     if (sh.total > 0.0 || d.mode == 1) break;
     // The residual mass is zero (possible only through rounding): draw from p_n.
@@ -648,7 +662,11 @@ __device__ int finish_draw(const VerifyParams& P, int b, Decision d, const T* rp
     double run = before;
     int found = -1, last_pos_chunk = -1;
     for (int c = c0; c < c1; ++c) {
-      const double w = __ldcg(cs + c);
+      double w = 0.0;
+#pragma unroll
+      for (int k = 0; k < kKeep; ++k)
+        if (c == c0 + k) w = keep[k];
+      if (c >= c0 + kKeep) w = __ldcg(cs + c);
       const double nxt = run + w;
       if (found < 0 && nxt > t) found = c;
       if (w > 0.0) last_pos_chunk = c;
