@@ -11,13 +11,16 @@
 // Two launches per call; no CTA ever waits for another:
 //  1. verify_stream_kernel streams every logit row once. One CTA per slab
 //     (up to 256 KB of one row, a whole number of 16 KB rounds) issues 16-byte
-//     loads, four per thread in flight plus the next four prefetched, folds
-//     them into a running (reference, sum of 2^(x - reference)) in the log2
-//     domain and writes one partial per slab. Nothing else happens on this
-//     path.
+//     loads, four per thread in use plus the next four prefetched, folds them
+//     with packed float32x2 arithmetic into a running (reference, sum of
+//     2^(x - reference)) in the log2 domain and writes one partial per slab;
+//     the first slab of a drafted row also records the logit at the draft id.
+//     Slabs are left to the hardware's CTA scheduler, which hands them to SMs
+//     as they free up (SMs do not all get the same bandwidth, so a static
+//     split of the rows over one wave of CTAs ends later).
 //  2. verify_draw_kernel runs SD CTAs per sequence. Each first decides the
 //     sequence (the same decision in every one of them, so that none waits for
-//     another): it merges the slab partials of the sequence's 2K+1 rows,
+//     another): it merges the partials of the sequence's 2K+1 rows,
 //     evaluates the accept tests with Philox uniforms and finds the first
 //     rejection by ballot. It then sums, over its range of fixed-size
 //     vocabulary chunks, the weights of the final draw -- the residual
@@ -34,6 +37,7 @@
 // formed by FMAs with log2 e in two parts, so its error is three float32
 // roundings of the argument; a vector's weights are summed in float32, all
 // longer sums in float64.
+#include <atomic>
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -93,10 +97,14 @@ struct VerifyParams {
   float* p_at_draft;
   float* q_at_draft;
   float* row_lse;
-  Partial* partials;    // [B][2K+1][S]
+  Partial* partials;    // [B][2K+1][slots]
   double* chunk_sums;   // [B][nchunks] draw-weight sums of the chunks
   int* draw_count;      // [B], set to 0 before the draw launch
   Decision* decisions;  // [B] (the LM-head path: written by the decision launch)
+  // [B][2K+1]: logit of row j at its sequence's draft id (rows j != K; 0 for
+  // an id out of range), recorded by the stream launch; null without it
+  float* draft_logit = nullptr;
+  int ring = 0;  // the draw launch has a copy ring in dynamic shared memory
   // Rows of q per sequence in memory: K (q is [B][K][V]) or K+1 (q is the
   // draft-pathway output of the same B x (K+1) rows as p, bonus rows unused).
   int q_rows = 0;
@@ -237,6 +245,65 @@ __device__ __forceinline__ const T* row_ptr(const VerifyParams& P, int b, int j,
 
 // ---- launch 1: streaming ----------------------------------------------------------------
 
+// Folds two 16-byte vectors (16 bfloat16 or 8 float32 values) with packed
+// float32x2 arithmetic: the exponent arguments by fma.f32x2, 2^(.) on the SFU,
+// the balanced sum tree by add.f32x2 (fold's tree, pair by pair). Same
+// reference rule as fold.
+template <typename T>
+__device__ __forceinline__ void fold_pair(float& m, float& z, const uint4* v) {
+  constexpr bool kBf16 = sizeof(T) == 2;
+  constexpr int kP = kBf16 ? 8 : 4;  // float pairs
+  uint64_t x[kP];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+    if constexpr (kBf16) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        x[4 * k + i] =
+            uno::pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        x[2 * k + i] = uno::pack2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+    }
+  }
+  auto sum = [&](float ref) {
+    const uint64_t l2e = uno::pack2(kLog2e, kLog2e), nref = uno::pack2(-ref, -ref);
+    uint64_t e[kP];
+#pragma unroll
+    for (int i = 0; i < kP; ++i) {
+      const float2 a = uno::unpack2(uno::fma2(x[i], l2e, nref));
+      e[i] = uno::pack2(uno::ex2(a.x), uno::ex2(a.y));
+    }
+#pragma unroll
+    for (int w = 1; w < kP; w *= 2) {
+#pragma unroll
+      for (int i = 0; i + w < kP; i += 2 * w) e[i] = uno::add2(e[i], e[i + w]);
+    }
+    const float2 s = uno::unpack2(e[0]);
+    return s.x + s.y;
+  };
+  const float s = sum(m);
+  if (s < 0x1p70f) {  // false for inf and NaN
+    z += s;
+    return;
+  }
+  float gm = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kP; ++i) {
+    const float2 p = uno::unpack2(x[i]);
+    gm = fmaxf(gm, fmaxf(p.x, p.y));
+  }
+  if (gm == -INFINITY) return;
+  gm *= kLog2e;
+  if (gm > m) {
+    z = (m == -INFINITY) ? 0.f : z * uno::ex2(m - gm);
+    m = gm;
+  }
+  z += sum(m);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     verify_stream_kernel(const VerifyParams P) {
@@ -259,6 +326,14 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
   const int v0 = min(s * per, g.nvec), v1 = min(v0 + per, g.nvec);
   const uint4* vrow = reinterpret_cast<const uint4*>(row + g.head);
 
+  // The first slab's thread 0 of each drafted row also records the logit at
+  // the draft id: the id is loaded first, the logit while the first round is
+  // folded, so neither load stalls the stream.
+  const bool rec = (P.draft_logit != nullptr) && s == 0 && j != P.K && tid == 0;
+  int xq = -1;
+  float xl = 0.f;
+  if (rec) xq = __ldg(P.draft + static_cast<size_t>(b) * P.K + (j < P.K ? j : j - P.K - 1));
+
   float m = -INFINITY, z = 0.f;
   const int rounds = (v1 - v0 + kStep - 1) / kStep;  // the last one may be partial
   uint4 cur[kRound], nxt[kRound];
@@ -276,14 +351,10 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         nxt[k] = (idx < v1) ? __ldg(vrow + idx) : make_uint4(0, 0, 0, 0);
       }
     }
+    if (rec && r == 0 && xq >= 0 && xq < P.V) xl = Elem<T>::at(row, xq);
     if (base + kStep <= v1) {  // a full round: no predication
 #pragma unroll
-      for (int k = 0; k < kRound; k += 2) {
-        float f[2 * kVec];
-        Elem<T>::unpack(cur[k], f);
-        Elem<T>::unpack(cur[k + 1], f + kVec);
-        fold<2 * kVec>(m, z, f);
-      }
+      for (int k = 0; k < kRound; k += 2) fold_pair<T>(m, z, cur + k);
     } else {
 #pragma unroll
       for (int k = 0; k < kRound; ++k) {
@@ -297,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 #pragma unroll
     for (int k = 0; k < kRound; ++k) cur[k] = nxt[k];
   }
+  if (rec && rounds == 0 && xq >= 0 && xq < P.V) xl = Elem<T>::at(row, xq);
   if (s == 0 && tid < g.head) {
     const float v = Elem<T>::at(row, tid);
     fold<1>(m, z, &v);
@@ -318,6 +390,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     warp_merge(m, z);
     if (lane == 0) {
       P.partials[static_cast<size_t>(blockIdx.x)] = Partial{m, z};
+      if (rec) P.draft_logit[static_cast<size_t>(b) * R + j] = xl;
       // the draw launch counts its CTAs of this sequence from 0
       if (j == 0 && s == 0) P.draw_count[b] = 0;
     }
@@ -328,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
 
 struct DecideShared {
   float row_m[kMaxRows], row_z[kMaxRows];
+  int x[kMaxK];  // the sequence's draft ids
   int first_reject, invalid;
   Decision d;
 };
@@ -341,17 +415,24 @@ template <typename T>
 __device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, bool outputs) {
   const int tid = threadIdx.x;
   const int K = P.K, R = 2 * K + 1, V = P.V;
-  // Thread i < K (K <= kThreads) loads draft x_i and the logits at it first,
-  // so that these loads overlap the merge of the row statistics.
+  // Thread i < K (K <= kThreads) loads draft x_i and the logits at it first
+  // (recorded by the stream launch when it ran: then no load waits for x_i),
+  // and draws its Philox words, all overlapping the merge of the statistics.
   int x = -1;
   float lpx = 0.f, lqx = 0.f;
+  uint4 words = make_uint4(0, 0, 0, 0);
   if (tid < K) {
     x = P.draft[static_cast<size_t>(b) * K + tid];
-    if (x >= 0 && x < V) {
+    if (P.draft_logit != nullptr) {
+      lpx = __ldcg(P.draft_logit + static_cast<size_t>(b) * R + tid);
+      lqx = __ldcg(P.draft_logit + static_cast<size_t>(b) * R + K + 1 + tid);
+    } else if (x >= 0 && x < V) {
       size_t off;
       lpx = Elem<T>::at(row_ptr<T>(P, b, tid, &off), x);
       lqx = Elem<T>::at(row_ptr<T>(P, b, K + 1 + tid, &off), x);
     }
+    words = uno::verify_block_words(P.seed, P.step, b, tid);
+    sh.x[tid] = x;
   }
   if (P.ext_p == nullptr) {
     const int S = P.S;
@@ -413,8 +494,7 @@ __device__ void decide_sequence(const VerifyParams& P, int b, DecideShared& sh, 
       } else {
         const float pp = uno::ex2(fmaf(lpx, kLog2e, -sh.row_m[i])) / sh.row_z[i];
         const float qq = uno::ex2(fmaf(lqx, kLog2e, -sh.row_m[K + 1 + i])) / sh.row_z[K + 1 + i];
-        const uint4 w = uno::verify_block_words(P.seed, P.step, b, i);
-        rejected = !(uno::uniform24(w.x) * qq < pp);
+        rejected = !(uno::uniform24(words.x) * qq < pp);
         if (outputs && P.p_at_draft) P.p_at_draft[static_cast<size_t>(b) * K + i] = pp;
         if (outputs && P.q_at_draft) P.q_at_draft[static_cast<size_t>(b) * K + i] = qq;
       }
@@ -546,18 +626,101 @@ __device__ void chunk_sums_vec(const VerifyParams& P, const Decision& d, const T
   }
 }
 
+// Stages of a warp's copy ring for VPL vectors per lane and chunk (0: no ring).
+__host__ __device__ constexpr int ring_stages(int vpl) { return vpl == 1 ? 4 : (vpl == 2 ? 3 : 0); }
+
+// Shared-memory bytes of the draw CTA's copy ring.
+__host__ __device__ constexpr int ring_bytes(int vpl) {
+  return kWarps * ring_stages(vpl) * 2 * vpl * 32 * 16;
+}
+
+// The vector path of chunk_sums through a ring of D shared-memory stages per
+// warp, one chunk of both draw rows per stage: while a chunk's weights are
+// computed, the copies of the next D - 1 chunks are in flight (cp.async), so
+// the loads overlap the SFU work. Each lane copies and reads back only its own
+// 16-byte slots; a stage is refilled only after the lane has read it.
+template <typename T, int VPL>
+__device__ void chunk_sums_ring(const VerifyParams& P, const Decision& d, const T* rp, const T* rq,
+                                double* out, int c0, int c1, int w0, int wstep, uint4* ring) {
+  constexpr int kVec = Elem<T>::kVec;
+  constexpr int D = ring_stages(VPL);
+  constexpr int kStage = 2 * VPL * 32;  // 16-byte slots per stage and warp
+  const int lane = threadIdx.x & 31;
+  uint4* my = ring + (threadIdx.x >> 5) * (D * kStage);
+  const uint4* vp = reinterpret_cast<const uint4*>(rp);
+  const uint4* vq = reinterpret_cast<const uint4*>(rq);
+  const int cvec = P.chunk_len / kVec;
+  const int nvec_row = P.V / kVec;
+  const bool two = (d.mode == 0);
+  const int first = c0 + w0;
+  const int nk = (first < c1) ? (c1 - first + wstep - 1) / wstep : 0;
+  const SplitL Lp = split_l(d.lp), Lq = split_l(two ? d.lq : 0.0);
+  // every call commits one group per chunk slot, empty past the end, so that
+  // wait<D - 1> always refers to the chunk about to be used
+  auto issue = [&](int k) {
+    if (k < nk) {
+      const int c = first + k * wstep;
+      uint4* dst = my + (k % D) * kStage;
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) {
+        const int vi = c * cvec + q * 32 + lane;
+        if (vi < nvec_row) {
+          uno::cp_async16(dst + q * 32 + lane, vp + vi);
+          if (two) uno::cp_async16(dst + (VPL + q) * 32 + lane, vq + vi);
+        }
+      }
+    }
+    uno::cp_async_commit();
+  };
+#pragma unroll
+  for (int k = 0; k < D - 1; ++k) issue(k);
+  for (int k = 0; k < nk; ++k) {
+    issue(k + D - 1);
+    uno::cp_async_wait<D - 1>();
+    const int c = first + k * wstep;
+    const uint4* src = my + (k % D) * kStage;
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int vi = c * cvec + q * 32 + lane;
+      if (vi < nvec_row) {
+        float fp[kVec], fq[kVec], w[kVec];
+        Elem<T>::unpack(src[q * 32 + lane], fp);
+        Elem<T>::unpack(two ? src[(VPL + q) * 32 + lane] : make_uint4(0, 0, 0, 0), fq);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) w[e] = token_weight(d.mode, Lp, Lq, fp[e], fq[e]);
+#pragma unroll
+        for (int st = 1; st < kVec; st *= 2) {
+#pragma unroll
+          for (int e = 0; e + st < kVec; e += 2 * st) w[e] += w[e + st];
+        }
+        t += w[0];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+    if (lane == 0) out[c] = t;
+  }
+  uno::cp_async_wait<0>();  // nothing in flight once the ring is reused or left
+}
+
 // Chunk sums of chunks c0 + w0, c0 + w0 + wstep, ... (< c1): 16-byte vectors
 // when both rows are 16-byte aligned and V and the chunk length are whole
-// vectors, otherwise scalar loads.
+// vectors (through the copy ring when `ring` is given and the chunk is one or
+// two vectors per lane), otherwise scalar loads.
 template <typename T>
 __device__ void chunk_sums(const VerifyParams& P, int b, const Decision& d, const T* rp,
-                           const T* rq, int c0, int c1, int w0, int wstep) {
+                           const T* rq, int c0, int c1, int w0, int wstep, uint4* ring) {
   constexpr int kVec = Elem<T>::kVec;
   const int lane = threadIdx.x & 31;
   double* out = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
   const int vpl = P.chunk_len / (32 * kVec);  // vectors per lane per chunk
   const bool vec_ok = ((reinterpret_cast<uintptr_t>(rp) | reinterpret_cast<uintptr_t>(rq)) & 15) == 0 &&
                       (P.V % kVec) == 0 && (P.chunk_len % (32 * kVec)) == 0;
+  if (vec_ok && ring && vpl == 1)
+    return chunk_sums_ring<T, 1>(P, d, rp, rq, out, c0, c1, w0, wstep, ring);
+  if (vec_ok && ring && vpl == 2)
+    return chunk_sums_ring<T, 2>(P, d, rp, rq, out, c0, c1, w0, wstep, ring);
   if (vec_ok && vpl == 1) return chunk_sums_vec<T, 1>(P, d, rp, rq, out, c0, c1, w0, wstep);
   if (vec_ok && vpl == 2) return chunk_sums_vec<T, 2>(P, d, rp, rq, out, c0, c1, w0, wstep);
   if (vec_ok && vpl == 4) return chunk_sums_vec<T, 4>(P, d, rp, rq, out, c0, c1, w0, wstep);
@@ -624,7 +787,7 @@ __device__ int last_positive_in_chunk(const VerifyParams& P, const Decision& d, 
 // Thread t takes the sums of chunks [t * per, (t + 1) * per) (read twice).
 template <typename T>
 __device__ int finish_draw(const VerifyParams& P, int b, Decision d, const T* rp, const T* rq,
-                           DrawShared& sh) {
+                           DrawShared& sh, uint4* ring) {
   const int tid = threadIdx.x;
   const double* cs = P.chunk_sums + static_cast<size_t>(b) * P.nchunks;
   const float u = uno::uniform24(uno::verify_block_words(P.seed, P.step, b, d.n).y);
@@ -646,7 +809,7 @@ __device__ int finish_draw(const VerifyParams& P, int b, Decision d, const T* rp
     // The residual mass is zero (possible only through rounding): draw from p_n.
     d.mode = 1;
     rq = rp;
-    chunk_sums<T>(P, b, d, rp, rp, 0, P.nchunks, threadIdx.x >> 5, kWarps);
+    chunk_sums<T>(P, b, d, rp, rp, 0, P.nchunks, threadIdx.x >> 5, kWarps, ring);
     __threadfence();
     __syncthreads();
   }
@@ -709,6 +872,8 @@ template <typename T, bool DECIDE>
 __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(const VerifyParams P) {
   __shared__ DrawShared sh;
   __shared__ DecideShared dsh;
+  extern __shared__ __align__(16) uint4 ring_smem[];  // ring_bytes(vpl) bytes, or none
+  uint4* ring = P.ring ? ring_smem : nullptr;
   uno::launch_dependents();
   uno::grid_dependency_wait();
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -718,6 +883,7 @@ __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(c
     decide_sequence<T>(P, b, dsh, du == 0);
   } else {
     if (tid == 0) dsh.d = P.decisions[b];
+    if (tid < K) dsh.x[tid] = P.draft[static_cast<size_t>(b) * K + tid];
     __syncthreads();
   }
   const Decision d = dsh.d;
@@ -728,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(c
   const int per_cta = (P.nchunks + P.SD - 1) / P.SD;
   const int c0 = du * per_cta;
   const int c1 = min(c0 + per_cta, P.nchunks);
-  chunk_sums<T>(P, b, d, rp, rq, c0, c1, warp, kWarps);
+  chunk_sums<T>(P, b, d, rp, rq, c0, c1, warp, kWarps, ring);
   __syncthreads();
   if (tid == 0) {
     __threadfence();
@@ -739,11 +905,10 @@ __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(c
 
   // the CTA that completes the sequence picks the token and writes outputs
   __threadfence();
-  const int y = finish_draw<T>(P, b, d, rp, rq, sh);
+  const int y = finish_draw<T>(P, b, d, rp, rq, sh, ring);
   const int n = d.n;
   int32_t* out = P.out_tokens + static_cast<size_t>(b) * (K + 1);
-  const int32_t* x = P.draft + static_cast<size_t>(b) * K;
-  for (int i = tid; i <= K; i += kThreads) out[i] = (i < n) ? x[i] : ((i == n) ? y : -1);
+  for (int i = tid; i <= K; i += kThreads) out[i] = (i < n) ? dsh.x[i] : ((i == n) ? y : -1);
   if (tid == 0) P.accepted_len[b] = n;
 }
 
@@ -752,7 +917,7 @@ __global__ void __launch_bounds__(kThreads, kDrawCtasPerSm) verify_draw_kernel(c
 struct Geometry {
   int S, nchunks, chunk_len, SD;
   long long stream_ctas, draw_ctas;
-  size_t off_counts, off_decisions, off_partials, off_chunks, bytes;
+  size_t off_counts, off_decisions, off_partials, off_chunks, off_xlogit, bytes;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -795,7 +960,8 @@ Geometry geometry(int B, int K, int V, int dtype) {
   g.off_partials = align_up(g.off_decisions + sizeof(Decision) * static_cast<size_t>(B), 256);
   g.off_chunks =
       align_up(g.off_partials + sizeof(Partial) * static_cast<size_t>(g.stream_ctas), 256);
-  g.bytes = align_up(g.off_chunks + sizeof(double) * static_cast<size_t>(B) * g.nchunks, 256);
+  g.off_xlogit = align_up(g.off_chunks + sizeof(double) * static_cast<size_t>(B) * g.nchunks, 256);
+  g.bytes = align_up(g.off_xlogit + sizeof(float) * static_cast<size_t>(rows), 256);
   return g;
 }
 
@@ -803,10 +969,12 @@ Geometry geometry(int B, int K, int V, int dtype) {
 // while the previous kernel on the stream finishes (each waits for it before
 // touching global memory).
 template <typename Kern>
-int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P) {
+int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P,
+               int smem_bytes = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -816,14 +984,38 @@ int launch_pdl(Kern kern, long long grid, cudaStream_t st, const VerifyParams& P
   return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 
+// The draw kernel's dynamic shared memory: the copy ring, opted in above the
+// default 48 KB limit once per kernel instantiation and device.
+constexpr int kMaxDevices = 64;
+template <typename T, bool DECIDE>
+bool allow_draw_smem(int bytes) {
+  static std::atomic<int> allowed[kMaxDevices];  // zero-initialised (static storage)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::atomic<int>* a = (dev >= 0 && dev < kMaxDevices) ? &allowed[dev] : nullptr;
+  if (a && bytes <= a->load()) return true;
+  if (cudaFuncSetAttribute(verify_draw_kernel<T, DECIDE>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (a) a->store(bytes);
+  return true;
+}
+
 template <typename T>
-int launch(const VerifyParams& P, const Geometry& g, cudaStream_t st) {
+int launch(VerifyParams P, const Geometry& g, cudaStream_t st) {
+  const int vpl = P.chunk_len / (32 * Elem<T>::kVec);
+  const int smem = ring_bytes(vpl);
+  P.ring = smem > 0;
   if (P.ext_p == nullptr) {
+    if (!allow_draw_smem<T, true>(smem)) return UNO_ERR_CUDA;
     if (launch_pdl(verify_stream_kernel<T>, g.stream_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
-    if (launch_pdl(verify_draw_kernel<T, true>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+    if (launch_pdl(verify_draw_kernel<T, true>, g.draw_ctas, st, P, smem) != UNO_OK)
+      return UNO_ERR_CUDA;
   } else {
+    if (!allow_draw_smem<T, false>(smem)) return UNO_ERR_CUDA;
     if (launch_pdl(verify_decide_kernel<T>, P.B, st, P) != UNO_OK) return UNO_ERR_CUDA;
-    if (launch_pdl(verify_draw_kernel<T, false>, g.draw_ctas, st, P) != UNO_OK) return UNO_ERR_CUDA;
+    if (launch_pdl(verify_draw_kernel<T, false>, g.draw_ctas, st, P, smem) != UNO_OK)
+      return UNO_ERR_CUDA;
   }
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
@@ -882,6 +1074,7 @@ extern "C" int uno_verify_block(const void* p_logits, const void* q_logits,
   P.decisions = reinterpret_cast<Decision*>(ws + g.off_decisions);
   P.partials = reinterpret_cast<Partial*>(ws + g.off_partials);
   P.chunk_sums = reinterpret_cast<double*>(ws + g.off_chunks);
+  P.draft_logit = reinterpret_cast<float*>(ws + g.off_xlogit);
   P.q_rows = K;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return (dtype == UNO_BF16) ? launch<uint16_t>(P, g, st) : launch<float>(P, g, st);
