@@ -9,45 +9,58 @@
 // the accept test and the resample), so drafting, verification and
 // resampling draw independent uniforms from one stream.
 //
-// One CTA per row (b, i), one pass over the row in HBM: each warp takes
-// chunks of the row (at least kMinSteps 16-byte vectors per lane, so the warp
-// reduction is paid once per several vectors), reduces each chunk to (chunk
-// max, sum of 2^(x - chunk max)) in the log2 domain and keeps it in shared
-// memory. The CTA then rescales the chunk sums to the row maximum, takes their
-// float64 running sum, finds the chunk where u * total is crossed and scans
-// only that chunk (in L2 by then): each thread sums a contiguous segment, one
-// block scan places the segments, and the thread whose segment crosses finds
-// the token.
+// One cluster of kCluster CTAs per row (b, i), one pass over the row in HBM:
+// each warp of the cluster takes chunks of the row (at least kMinSteps 16-byte
+// vectors per lane, so the warp reduction is paid once per several vectors)
+// and streams them in rounds of kRound 16-byte vectors per lane through a
+// ring of kStages shared-memory stages (cp.async): kStages - 1 rounds are in
+// flight while one is folded into a per-lane (reference, sum of
+// 2^(x - reference)) in the log2 domain with packed float32x2 arithmetic. The
+// warp reduces each chunk to one such pair in the leading CTA's shared memory
+// (distributed shared memory), and the others leave after a cluster barrier.
+// The leader then rescales the chunk sums to the largest reference, takes
+// their float64 running sum, finds the chunk where u * total is crossed and
+// scans only that chunk (in L2 by then): each thread sums a contiguous
+// segment, one block scan places the segments, and the thread whose segment
+// crosses finds the token.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
 #include <cuda_runtime.h>
 
+#include <cooperative_groups.h>
+
+#include "logstat.cuh"
 #include "uno.h"
 #include "uno_device.cuh"
 #include "uno_host.h"
 
 namespace {
 
-constexpr int kMaxChunks = 2048;  // chunk table in shared memory (16 KB)
-constexpr int kMinSteps = 8;      // vectors per lane in a chunk, at least
+namespace cg = cooperative_groups;
 
-// Launch shapes. Many rows (a 64 x 16 block of drafts): 128-thread CTAs, 8 per
-// SM, one wave. Few rows (a tree's node rows at batch 1): 512-thread CTAs, so
-// that a handful of rows still keeps enough loads in flight. Four chunks in
-// flight per warp either way (more spill registers).
-template <int THREADS, int IN_FLIGHT, int CTAS_PER_SM>
+constexpr int kMaxChunks = 2048;  // chunk table entries (shared memory, 8 bytes each)
+constexpr int kMinSteps = 16;     // vectors per lane in a chunk, at least
+
+// Launch shapes. Many rows (a 64 x 16 block of drafts): two 128-thread CTAs
+// per row, 8 per SM, in about two waves that the hardware balances over the
+// SMs. Few rows (a tree's node rows at batch 1): four 512-thread CTAs per row,
+// so that a handful of rows still keeps enough loads in flight.
+template <int THREADS, int CTAS_PER_SM, int CLUSTER>
 struct Shape {
   static constexpr int kThreads = THREADS;
   static constexpr int kWarps = THREADS / 32;
-  static constexpr int kInFlight = IN_FLIGHT;  // chunks a warp loads before reducing them
   static constexpr int kCtasPerSm = CTAS_PER_SM;
+  static constexpr int kCluster = CLUSTER;  // CTAs per row
 };
-using Narrow = Shape<128, 4, 8>;
-using Wide = Shape<512, 4, 2>;
+using Narrow = Shape<128, 8, 2>;
+using Wide = Shape<512, 2, 4>;
+constexpr int kRound = 4;   // 16-byte vectors per lane per round (a chunk is whole rounds)
+constexpr int kStages = 3;  // ring stages per warp, one round each
 constexpr int kWideRows = 2 * 148;  // at most this many rows: the wide shape
-constexpr float kLog2e = 1.4426950408889634f;
+using uno::kLog2e;
 
 struct SampleParams {
   const void* q;       // [B][rows][V]
@@ -61,10 +74,16 @@ struct SampleParams {
   int32_t* out;        // [B][rows]
 };
 
+// Dynamic shared memory: the warps' copy rings (kStages rounds each), then the
+// chunk table: cm[nchunks] (the chunk's reference in the log2 domain, -inf
+// when empty) and cs[nchunks] (sum over the chunk of 2^(x log2 e - cm)).
+template <int kWarps>
+constexpr int ring_bytes() {
+  return kWarps * kStages * kRound * 32 * 16;
+}
+
 template <int kWarps>
 struct Shared {
-  float cm[kMaxChunks];  // chunk maximum (log2 domain), -inf when empty
-  float cs[kMaxChunks];  // sum over the chunk of 2^(x log2 e - cm)
   double warp_tot[kWarps];
   float warp_max[kWarps];
   double carry;
@@ -74,12 +93,6 @@ struct Shared {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   return v;
 }
 
@@ -115,88 +128,107 @@ __device__ __forceinline__ float w2(float x, float ref) {
 template <typename T, typename S>
 __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
     sample_drafts_kernel(const SampleParams P) {
-  constexpr int kThreads = S::kThreads, kWarps = S::kWarps, kInFlight = S::kInFlight;
+  constexpr int kThreads = S::kThreads, kWarps = S::kWarps, kCluster = S::kCluster;
   __shared__ Shared<kWarps> sh;
+  extern __shared__ __align__(16) uint4 dyn[];  // rings, then the chunk table (the leader's)
   uno::launch_dependents();
   uno::grid_dependency_wait();
   constexpr int kVec = uno::LogitRow<T>::kVec;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bi = blockIdx.x;  // b * rows + n
+  const int rank = static_cast<int>(blockIdx.x) % kCluster;  // 1-D clusters of kCluster
+  const int bi = static_cast<int>(blockIdx.x) / kCluster;    // b * rows + n
   if (P.n_rows != nullptr && bi % P.rows >= P.n_rows[bi / P.rows]) {
-    if (tid == 0) P.out[bi] = -1;  // a row not in use: the whole CTA leaves
+    if (tid == 0 && rank == 0) P.out[bi] = -1;  // a row not in use: the cluster leaves
     return;
   }
+  cg::cluster_group cluster = cg::this_cluster();
   const T* row = static_cast<const T*>(P.q) + static_cast<size_t>(bi) * P.V;
-  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   const int V = P.V, L = P.chunk_len;
+  uint4* ring = dyn + warp * (kStages * kRound * 32);
+  float* cm = reinterpret_cast<float*>(dyn + kWarps * kStages * kRound * 32);
+  float* cs = cm + P.nchunks;
 
-  // ---- pass 1: per-chunk (max, sum of 2^(x - max)) ----
-  // Each step a warp issues one 16-byte load per lane for kInFlight chunks
-  // before it reduces any of them. Every lane keeps its own reference (its
-  // running maximum, raised only when a larger value arrives) and sum; the
-  // warp combines them once per chunk.
-  for (int c0 = warp; c0 < P.nchunks; c0 += kWarps * kInFlight) {
-    float lm[kInFlight], ls[kInFlight];
+  // ---- pass 1: per-chunk (reference, sum of 2^(x - reference)) ----
+  // Warp w of the cluster (gw = rank * kWarps + w) takes chunks gw, gw + nw,
+  // ... (nw = kCluster * kWarps); a chunk is rpc rounds, a round
+  // kRound whole 16-byte vectors per lane (a load instruction of the warp
+  // reads 512 contiguous bytes). Elements outside whole vectors (the row's
+  // tail, or the whole row when it is not 16-byte aligned) are read one by
+  // one at the end of their chunk.
+  const bool aligned = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  const int nvec = aligned ? V / kVec : 0;  // whole vectors of the row
+  const uint4* vrow = reinterpret_cast<const uint4*>(row);
+  const int cvec = L / kVec;                // vectors per chunk
+  const int rpc = cvec / (32 * kRound);     // rounds per chunk
+  constexpr int nw = kCluster * kWarps;
+  const int gw = rank * kWarps + warp;
+  const int my_chunks = (gw < P.nchunks) ? (P.nchunks - gw + nw - 1) / nw : 0;
+  const int n_rounds = my_chunks * rpc;
+  int lc = gw, lr = 0;  // chunk and round of the next copies
+  // round j goes to stage j mod kStages; one commit group per round (empty
+  // past the end), so wait<kStages - 1> always means "round k has landed"
+  auto issue = [&](int j) {
+    if (j < n_rounds) {
+      uint4* dst = ring + (j % kStages) * (kRound * 32) + lane;
+      const int vb = lc * cvec + lr * (32 * kRound) + lane;
 #pragma unroll
-    for (int k = 0; k < kInFlight; ++k) {
-      lm[k] = -INFINITY;
-      ls[k] = 0.f;
-    }
-    // a chunk is L / (32 kVec) steps of one vector per lane
-    for (int s = 0; s < L; s += 32 * kVec) {
-      uint4 raw[kInFlight];
-#pragma unroll
-      for (int k = 0; k < kInFlight; ++k) {
-        const int c = c0 + k * kWarps;
-        const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
-        raw[k] = (c < P.nchunks && vec && v0 + kVec <= V)
-                     ? __ldg(reinterpret_cast<const uint4*>(row + v0))
-                     : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < kInFlight; ++k) {
-        const int c = c0 + k * kWarps;
-        const long long v0 = static_cast<long long>(c) * L + s + lane * kVec;
-        float f[kVec];  // logits as read (natural log domain)
-        if (c < P.nchunks && vec && v0 + kVec <= V) {
-          uno::LogitRow<T>::unpack(raw[k], f);
-        } else {
-#pragma unroll
-          for (int e = 0; e < kVec; ++e)
-            f[e] = (c < P.nchunks && v0 + e < V) ? uno::LogitRow<T>::at(row, v0 + e) : -INFINITY;
-        }
-        float mk = f[0];
-#pragma unroll
-        for (int e = 1; e < kVec; ++e) mk = fmaxf(mk, f[e]);
-        mk *= kLog2e;
-        if (mk > lm[k]) {  // a larger value: move the reference up
-          ls[k] *= uno::ex2(lm[k] - mk);
-          lm[k] = mk;
-        }
-        if (lm[k] > -INFINITY) {
-          float add = 0.f;
-#pragma unroll
-          for (int e = 0; e < kVec; ++e) add += w2(f[e], lm[k]);
-          ls[k] += add;
-        }
+      for (int k = 0; k < kRound; ++k)
+        if (vb + k * 32 < nvec) uno::cp_async16(dst + k * 32, vrow + vb + k * 32);
+      if (++lr == rpc) {
+        lr = 0;
+        lc += nw;
       }
     }
+    uno::cp_async_commit();
+  };
 #pragma unroll
-    for (int k = 0; k < kInFlight; ++k) {
-      const int c = c0 + k * kWarps;
-      const float m = warp_max(lm[k]);
-      const float t = warp_sum((lm[k] > -INFINITY) ? ls[k] * uno::ex2(lm[k] - m) : 0.f);
-      if (lane == 0 && c < P.nchunks) {
-        sh.cm[c] = m;
-        sh.cs[c] = (m > -INFINITY) ? t : 0.f;
+  for (int j = 0; j < kStages - 1; ++j) issue(j);
+  float lm = -INFINITY, ls = 0.f;
+  int c = gw, r = 0;  // chunk and round being folded
+  for (int k = 0; k < n_rounds; ++k) {
+    issue(k + kStages - 1);
+    uno::cp_async_wait<kStages - 1>();
+    uint4 cur[kRound];
+    {
+      const uint4* src = ring + (k % kStages) * (kRound * 32) + lane;
+#pragma unroll
+      for (int j = 0; j < kRound; ++j) cur[j] = src[j * 32];
+    }
+    const int vb = c * cvec + r * (32 * kRound) + lane;
+    if (vb + (kRound - 1) * 32 < nvec) {  // every vector of the round is whole
+#pragma unroll
+      for (int j = 0; j < kRound; j += 2) uno::fold_vecs<T, 2>(lm, ls, cur + j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kRound; ++j)
+        if (vb + j * 32 < nvec) uno::fold_vecs<T, 1>(lm, ls, cur + j);
+    }
+    if (++r == rpc) {  // the chunk is complete
+      // its elements outside whole vectors, one by one
+      const int e0 = max(c * L, nvec * kVec), e1 = min((c + 1) * L, V);
+      for (int e = e0 + lane; e < e1; e += 32) {
+        const float f = uno::LogitRow<T>::at(row, e);
+        uno::fold<1>(lm, ls, &f);
       }
+      uno::warp_merge(lm, ls);
+      if (lane == 0) {  // into the leader's table
+        *cluster.map_shared_rank(cm + c, 0) = lm;
+        *cluster.map_shared_rank(cs + c, 0) = (lm > -INFINITY) ? ls : 0.f;
+      }
+      lm = -INFINITY;
+      ls = 0.f;
+      r = 0;
+      c += nw;
     }
   }
-  __syncthreads();
+  uno::cp_async_wait<0>();
+  // the table is complete and visible to the leader (release / acquire)
+  cluster.sync();
+  if (rank != 0) return;
 
-  // ---- the row maximum and the rescaled chunk sums ----
+  // ---- the largest chunk reference M and the chunk sums rescaled to it ----
   float mx = -INFINITY;
-  for (int c = tid; c < P.nchunks; c += kThreads) mx = fmaxf(mx, sh.cm[c]);
+  for (int c = tid; c < P.nchunks; c += kThreads) mx = fmaxf(mx, cm[c]);
   mx = warp_max(mx);
   if (lane == 0) sh.warp_max[warp] = mx;
   if (tid == 0) {
@@ -221,8 +253,8 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
   double mine = 0.0;
   int last_pos_chunk = -1;
   for (int c = c_lo; c < c_hi; ++c) {
-    const double w = (sh.cm[c] > -INFINITY) ? static_cast<double>(sh.cs[c]) *
-                                                  static_cast<double>(uno::ex2(sh.cm[c] - M))
+    const double w = (cm[c] > -INFINITY) ? static_cast<double>(cs[c]) *
+                                                  static_cast<double>(uno::ex2(cm[c] - M))
                                             : 0.0;
     mine += w;
     if (w > 0.0) last_pos_chunk = c;
@@ -234,8 +266,8 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
     double run = before;
     int found = -1;
     for (int c = c_lo; c < c_hi && found < 0; ++c) {
-      const double w = (sh.cm[c] > -INFINITY) ? static_cast<double>(sh.cs[c]) *
-                                                    static_cast<double>(uno::ex2(sh.cm[c] - M))
+      const double w = (cm[c] > -INFINITY) ? static_cast<double>(cs[c]) *
+                                                    static_cast<double>(uno::ex2(cm[c] - M))
                                               : 0.0;
       if (run + w > t) found = c;
       else run += w;
@@ -291,11 +323,30 @@ bool sample_sizes_ok(int B, int K, int V, int dtype) {
          K <= 256 && V >= 1 && V <= (1 << 28) && static_cast<long long>(B) * K <= (1 << 28);
 }
 
+// Dynamic shared memory above the default 48 KB needs an opt-in, once per
+// kernel instantiation and device.
+constexpr int kMaxDevices = 64;
+template <typename T, typename S>
+bool allow_smem(int bytes) {
+  static std::atomic<int> allowed[kMaxDevices];  // zero-initialised (static storage)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::atomic<int>* a = (dev >= 0 && dev < kMaxDevices) ? &allowed[dev] : nullptr;
+  if (a && bytes <= a->load()) return true;
+  if (cudaFuncSetAttribute(sample_drafts_kernel<T, S>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (a) a->store(bytes);
+  return true;
+}
+
 template <typename T, typename S>
 int run(const uno_host::RowDraws& r, cudaStream_t st) {
   constexpr int kStep = 32 * uno::LogitRow<T>::kVec;  // elements per vector step of a warp
-  // a chunk is a whole number of warp steps and of CTA-wide segments
-  constexpr int kStepsMult = (S::kThreads > kStep) ? S::kThreads / kStep : 1;
+  // a chunk is a whole number of rounds (kRound warp steps) and of CTA-wide
+  // segments (both powers of two: the larger is a multiple of the other)
+  constexpr int kSegSteps = (S::kThreads > kStep) ? S::kThreads / kStep : 1;
+  constexpr int kStepsMult = (kSegSteps > kRound) ? kSegSteps : kRound;
   const int V = r.V;
   SampleParams P{};
   P.q = r.logits;
@@ -315,14 +366,21 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
   P.chunk_len = static_cast<int>(per_chunk * kStep);
   P.nchunks = static_cast<int>((V + P.chunk_len - 1) / P.chunk_len);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(r.B * r.rows_per_seq));
+  const int smem = ring_bytes<S::kWarps>() + 2 * P.nchunks * static_cast<int>(sizeof(float));
+  if (!allow_smem<T, S>(smem)) return UNO_ERR_CUDA;
+  cfg.gridDim = dim3(static_cast<unsigned>(r.B * r.rows_per_seq * S::kCluster));
   cfg.blockDim = dim3(S::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = S::kCluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, sample_drafts_kernel<T, S>, P) != cudaSuccess)
     return UNO_ERR_CUDA;
   return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
