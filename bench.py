@@ -1,7 +1,8 @@
 """Benchmark of one Psi-Spec decode step's hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload batched_decode_b64_k16|qwen3_8b_b1|qwen3_8b_stack_b64_k16]
+                    [--workload batched_decode_b64_k16|qwen3_8b_b1|qwen3_8b_stack_b64_k16
+                                |verifier_sweep]
 
 A step is one pass over the whole hot path for one batch:
   batched_decode_b64_k16 (default): B = 64 sequences x K = 16 drafted positions
@@ -15,6 +16,11 @@ A step is one pass over the whole hot path for one batch:
   qwen3_8b_stack_b64_k16: the whole 8B-shaped draft-verify step: 36 layers of
       dual-path projections over 64 x 17 rows (row gate: first position AR
       only), the dual-path LM head, the on-device draft sampler, the verifier.
+  verifier_sweep: the block verifier alone over every (B, K, dtype) of
+      B in {1, 8, 32, 64, 128, 256}, K in {4, 8, 16, 32}, bf16 and f32,
+      V = 151936, Gumbel logits with 20 tokens per row boosted by +8, draft
+      noise sigma = 1 (and 0.25, 4 at B = 64, K = 16, bf16): GB/s and the
+      fraction of the HBM peak per point, one step = one verifier call.
 
 The metric is verified draft rows per second (B*K per step); emitted tokens
 per second is reported beside it. Inputs are synthetic and seeded (random
@@ -552,7 +558,6 @@ class StackStep(BatchedDecode):
         T = api.dualpath_stats_tiles(M, self.V)
         self.s_ar = torch.empty(M, T, 2, dtype=torch.float32, device=dev)
         self.s_dr = torch.empty(M, T, 2, dtype=torch.float32, device=dev)
-        self.q = torch.empty(self.B, self.K, self.V, dtype=bf, device=dev)
         self.drafts = torch.empty(self.B, self.K, dtype=torch.int32, device=dev)
         need = max(api.dualpath_workspace_bytes(M, 12288, 12288, RANK, bf) * 3,
                    api.dualpath_workspace_bytes(M, H, self.V, RANK, bf))
@@ -620,10 +625,9 @@ class StackStep(BatchedDecode):
                                   y_draft=self.q_all, stats_ar=self.s_ar, stats_draft=self.s_dr,
                                   workspace=self.ws)
         mark(1)
-        # the sampler and the verifier read q as [B][K][V]: drop each block's
-        # bonus row (a torch copy, about 0.6 GB of traffic)
-        self.q.copy_(self.q_all.view(self.B, self.K + 1, self.V)[:, : self.K])
-        api.sample_drafts(self.q, self.philox_seed, seed_step, out=self.drafts)
+        # the sampler reads the first K rows of each block of K + 1 in place
+        api.sample_drafts(self.q_all.view(self.B, self.K + 1, self.V), self.philox_seed,
+                          seed_step, out=self.drafts, num_drafts=self.K)
         if ev is not None:
             ev[2].record()
         api.verify_block_head(self.p, self.q_all, self.s_ar, self.s_dr, self.drafts,
@@ -745,6 +749,11 @@ def run_reference(args):
         print(json.dumps({"impl": "reference", "unavailable": "the float64 oracle of 36 layers "
                           "and the LM head does not fit a bounded host sample"}), flush=True)
         return 0
+    if args.workload == SWEEP:
+        print(json.dumps({"impl": "reference", "unavailable": "the sweep is a set of verifier "
+                          "points, not one step a bounded oracle sample can stand for"}),
+              flush=True)
+        return 0
     n_seq = 1
     for i in range(args.warmup):
         oracle_sample(args.workload, n_seq, step=i)
@@ -767,6 +776,104 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the verifier sweep
+# ---------------------------------------------------------------------------
+
+SWEEP = "verifier_sweep"
+SWEEP_B = (1, 8, 32, 64, 128, 256)
+SWEEP_K = (4, 8, 16, 32)
+SWEEP_DTYPES = ("bf16", "f32")
+L2_BYTES = 126 * 2 ** 20
+
+
+def sweep_points():
+    pts = [(B, K, dt, 1.0) for dt in SWEEP_DTYPES for B in SWEEP_B for K in SWEEP_K]
+    pts += [(B64, K16, "bf16", 0.25), (B64, K16, "bf16", 4.0)]
+    return pts
+
+
+def verify_algorithmic_bytes(B, K, V, esize):
+    # every logit row once, the drafts, the outputs (tokens and lengths)
+    return B * (2 * K + 1) * V * esize + B * K * 4 + B * (K + 2) * 4
+
+
+def run_sweep(args):
+    world, rank, local = _dist()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from lossless_decoding_b200 import api
+    from lossless_decoding_b200.inputs import verify_inputs
+    peaks = _peaks()
+    steps = max(3, min(args.steps, 10))
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    points, tot_rows, tot_s = [], 0, 0.0
+    for (B, K, dt, sigma) in sweep_points():
+        V = QWEN3_8B_VOCAB
+        v = verify_inputs(B, K, V, dtype=dt, dist="gumbel", sigma=sigma, seed=B * 100 + K,
+                          device=dev)
+        esize = v.p_logits.element_size()
+        ws = torch.zeros(api.verify_workspace_bytes(B, K, V, v.p_logits.dtype),
+                         dtype=torch.uint8, device=dev)
+        out = api.VerifyResult(torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+                               torch.empty((B,), dtype=torch.int32, device=dev), None, None, None)
+        nbytes = verify_algorithmic_bytes(B, K, V, esize)
+        small = nbytes < 2 * L2_BYTES  # else the inputs alone exceed L2
+        for i in range(args.warmup):
+            api.verify_block(v.p_logits, v.q_logits, v.draft_tokens, seed=1234, step=i,
+                             out=out, workspace=ws)
+        ts = []
+        for i in range(steps):
+            if small:
+                flush.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            api.verify_block(v.p_logits, v.q_logits, v.draft_tokens, seed=1234,
+                             step=args.warmup + i, out=out, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(ts)
+        gbs = nbytes / t / 1e9
+        acc = float(out.accepted_len.clamp(min=0).float().mean().item())
+        points.append({"B": B, "K": K, "dtype": dt, "sigma": sigma, "us": t * 1e6,
+                       "GBps": gbs, "frac": gbs / peaks["hbm"], "rows_per_s": B * K / t,
+                       "mean_accepted": acc, "logit_bytes": B * (2 * K + 1) * V * esize,
+                       "l2_flushed": small})
+        tot_rows += B * K
+        tot_s += t
+        del v, ws, out
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    if rank == 0:
+        big = [p for p in points if p["logit_bytes"] >= 4 * L2_BYTES]
+        line = {
+            "metric": METRIC, "value": tot_rows / tot_s, "unit": UNIT, "n_gpus": 1,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / len(points),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16+f32", "data": "synthetic (seeded Gumbel logits, top-20 boosted)",
+            "config": {"workload": SWEEP, "V": QWEN3_8B_VOCAB, "points": len(points),
+                       "l2": "flushed before each timed call where a point's bytes are "
+                             "below 2x L2; larger points exceed L2 by themselves",
+                       "value": "all points' rows / the sum of their median call times"},
+            "roofline": {"kernel": "verify_stream_kernel + verify_draw_kernel", "bound": "hbm",
+                         "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac_min_large": min(p["frac"] for p in big) if big else None,
+                         "frac_median_large": (statistics.median(p["frac"] for p in big)
+                                               if big else None),
+                         "large": "points with at least 4x L2 of logits",
+                         "peak_kind": f"HBM copy, {peaks['src']}"},
+            "sweep": points, "clocks": clk, "gpu_launches": 2 * len(points) * steps,
+        }
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -933,13 +1040,16 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_decode_b64_k16")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [SWEEP],
+                    default="batched_decode_b64_k16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == SWEEP:
+        return run_sweep(args)
     return run_ours(args)
 
 

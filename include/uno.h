@@ -298,6 +298,15 @@ int uno_verify_block_head(const void* y_ar, const void* y_draft, const float* st
 int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype, uint64_t seed,
                       uint64_t step, int32_t* draft_tokens, void* stream);
 
+/* The same draws from logits laid out in blocks of block_rows >= K rows per
+ * sequence ([B, block_rows, V], for example the LM head's draft-pathway output
+ * of K + 1 rows per block): draft_tokens[b][i] ~ softmax(logits[b][i]) for
+ * i < K; rows K..block_rows-1 of each block are not read. With block_rows = K
+ * this is uno_sample_drafts. Limits as above, and K <= block_rows <= 4096,
+ * B * block_rows <= 2^28 (else UNO_ERR_SIZE). */
+int uno_sample_drafts_blocks(const void* logits, int B, int K, int block_rows, int V, int dtype,
+                             uint64_t seed, uint64_t step, int32_t* draft_tokens, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Tree sampler
  *

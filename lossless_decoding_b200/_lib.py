@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     L.uno_dualpath_linear_grouped.restype = i32
     L.uno_sample_drafts.argtypes = [vp, i32, i32, i32, i32, u64, u64, vp, vp]
     L.uno_sample_drafts.restype = i32
+    L.uno_sample_drafts_blocks.argtypes = [vp, i32, i32, i32, i32, i32, u64, u64, vp, vp]
+    L.uno_sample_drafts_blocks.restype = i32
     L.uno_dualpath_stats_tiles.argtypes = [i32, i32]
     L.uno_dualpath_stats_tiles.restype = i32
     L.uno_dualpath_linear_stats.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, vp,

@@ -390,16 +390,25 @@ def dualpath_linear_grouped(x: torch.Tensor, Ws, As, Bms, scales, *, want_ar: bo
 
 
 def sample_drafts(q_logits: torch.Tensor, seed: int, step: int, *,
-                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  out: Optional[torch.Tensor] = None,
+                  num_drafts: Optional[int] = None) -> torch.Tensor:
     """Drafted ids of the linear sampler: out[b, i] ~ softmax(q_logits[b, i]).
 
-    q_logits [B, K, V] bfloat16 or float32 on a CUDA device; returns int32
-    [B, K] (-1 for a row with no finite logit). Uniform: Philox word 2 of
-    (b, i, step) under key `seed`, next to the verifier's words 0 and 1.
+    q_logits [B, R, V] bfloat16 or float32 on a CUDA device, contiguous;
+    draws rows i < K of each block, K = num_drafts (default R; for example
+    R = K + 1 for the LM head's draft-pathway output, whose last row per block
+    is then not read). Returns int32 [B, K] (-1 for a row with no finite
+    logit). Uniform: Philox word 2 of (b, i, step) under key `seed`, next to
+    the verifier's words 0 and 1.
     """
     if q_logits.dim() != 3:
-        raise ValueError("q_logits must be [B, K, V]")
-    B, K, V = q_logits.shape
+        raise ValueError("q_logits must be [B, R, V]")
+    if not q_logits.is_contiguous():
+        raise ValueError("q_logits must be contiguous")
+    B, R, V = q_logits.shape
+    K = R if num_drafts is None else int(num_drafts)
+    if not 1 <= K <= R:
+        raise ValueError("num_drafts must be in [1, R]")
     dt = _dtype_code(q_logits)
     dev = _check_cuda(q_logits)
     if out is None:
@@ -407,11 +416,12 @@ def sample_drafts(q_logits: torch.Tensor, seed: int, step: int, *,
     if out.dtype != torch.int32 or tuple(out.shape) != (B, K):
         raise ValueError("out must be int32 [B, K]")
     _check_cuda(out)
-    st = lib.uno_sample_drafts(_ptr(q_logits), B, K, V, dt, ctypes.c_uint64(seed & (2**64 - 1)),
-                               ctypes.c_uint64(step & (2**64 - 1)), _ptr(out),
-                               _stream_handle(dev))
+    st = lib.uno_sample_drafts_blocks(_ptr(q_logits), B, K, R, V, dt,
+                                      ctypes.c_uint64(seed & (2**64 - 1)),
+                                      ctypes.c_uint64(step & (2**64 - 1)), _ptr(out),
+                                      _stream_handle(dev))
     if st != 0:
-        raise UnoError(st, "uno_sample_drafts")
+        raise UnoError(st, "uno_sample_drafts_blocks")
     return out
 
 

@@ -63,8 +63,9 @@ constexpr int kWideRows = 2 * 148;  // at most this many rows: the wide shape
 using uno::kLog2e;
 
 struct SampleParams {
-  const void* q;       // [B][rows][V]
-  int B, rows, V;      // rows: rows per sequence
+  const void* q;       // [B][seq_rows][V], rows 0..rows-1 of each block drawn
+  int B, rows, V;      // rows: rows drawn per sequence
+  int seq_rows;        // rows per sequence in memory (>= rows)
   int chunk_len;       // elements per chunk (a multiple of 32 * kVec and of kThreads)
   int nchunks;
   const int32_t* row_key;  // [B][rows] Philox position of each row (null: the row index)
@@ -142,7 +143,9 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
     return;
   }
   cg::cluster_group cluster = cg::this_cluster();
-  const T* row = static_cast<const T*>(P.q) + static_cast<size_t>(bi) * P.V;
+  const int seq = bi / P.rows;
+  const T* row = static_cast<const T*>(P.q) +
+                 (static_cast<size_t>(seq) * P.seq_rows + (bi - seq * P.rows)) * P.V;
   const int V = P.V, L = P.chunk_len;
   uint4* ring = dyn + warp * (kStages * kRound * 32);
   float* cm = reinterpret_cast<float*>(dyn + kWarps * kStages * kRound * 32);
@@ -352,6 +355,7 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
   P.q = r.logits;
   P.B = r.B;
   P.rows = r.rows_per_seq;
+  P.seq_rows = (r.seq_rows > 0) ? r.seq_rows : r.rows_per_seq;
   P.V = V;
   P.row_key = r.row_key;
   P.n_rows = r.n_rows;
@@ -395,22 +399,25 @@ int uno_host::sample_rows(const RowDraws& r, cudaStream_t st) {
   return (r.dtype == UNO_BF16) ? run<uint16_t, Narrow>(r, st) : run<float, Narrow>(r, st);
 }
 
-extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype,
-                                 uint64_t seed, uint64_t step, int32_t* draft_tokens,
-                                 void* stream) {
+extern "C" int uno_sample_drafts_blocks(const void* logits, int B, int K, int block_rows, int V,
+                                        int dtype, uint64_t seed, uint64_t step,
+                                        int32_t* draft_tokens, void* stream) {
   if (dtype != UNO_BF16 && dtype != UNO_F32) return UNO_ERR_DTYPE;
-  if (!sample_sizes_ok(B, K, V, dtype)) return UNO_ERR_SIZE;
+  if (!sample_sizes_ok(B, K, V, dtype) || block_rows < K || block_rows > 4096 ||
+      static_cast<long long>(B) * block_rows > (1LL << 28))
+    return UNO_ERR_SIZE;
   if (B == 0) return UNO_OK;
-  if (!q_logits || !draft_tokens) return UNO_ERR_NULL;
-  if (!uno_host::aligned(q_logits, dtype == UNO_BF16 ? 2 : 4) ||
+  if (!logits || !draft_tokens) return UNO_ERR_NULL;
+  if (!uno_host::aligned(logits, dtype == UNO_BF16 ? 2 : 4) ||
       !uno_host::aligned(draft_tokens, 4))
     return UNO_ERR_ALIGN;
   const int dev = uno_host::check_device();
   if (dev != UNO_OK) return dev;
   uno_host::RowDraws r{};
-  r.logits = q_logits;
+  r.logits = logits;
   r.B = B;
   r.rows_per_seq = K;
+  r.seq_rows = block_rows;
   r.V = V;
   r.dtype = dtype;
   r.word = 2;  // drafting: word 2 of the (b, i, step) block
@@ -418,4 +425,10 @@ extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int 
   r.step = step;
   r.out = draft_tokens;
   return uno_host::sample_rows(r, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int uno_sample_drafts(const void* q_logits, int B, int K, int V, int dtype,
+                                 uint64_t seed, uint64_t step, int32_t* draft_tokens,
+                                 void* stream) {
+  return uno_sample_drafts_blocks(q_logits, B, K, K, V, dtype, seed, step, draft_tokens, stream);
 }

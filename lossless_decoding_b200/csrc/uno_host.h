@@ -25,6 +25,7 @@ int check_device();
 struct RowDraws {
   const void* logits;
   int B, rows_per_seq, V, dtype;
+  int seq_rows = 0;  // rows from one sequence's block to the next (0: rows_per_seq)
   const int32_t* row_key;
   const int32_t* n_rows;
   int word;

@@ -52,3 +52,29 @@ def test_our_arm_needs_a_gpu():
         pytest.skip("a CUDA device is present")
     r = _bench("--steps", "1", "--warmup", "3", "--no-cpu-baseline")
     assert r.returncode != 0 and "CUDA device" in (r.stderr + r.stdout)
+
+
+def test_sweep_covers_the_verifier_sweep_grid():
+    """Every (B, K, dtype) of the verifier sweep at sigma = 1, plus the
+    high- and low-acceptance noise levels at B = 64, K = 16, bf16."""
+    import bench
+    pts = bench.sweep_points()
+    grid = {(B, K, dt) for B in (1, 8, 32, 64, 128, 256) for K in (4, 8, 16, 32)
+            for dt in ("bf16", "f32")}
+    assert {(B, K, dt) for B, K, dt, s in pts if s == 1.0} == grid
+    assert {s for B, K, dt, s in pts if (B, K, dt) == (64, 16, "bf16")} == {0.25, 1.0, 4.0}
+    # logits of 2K+1 rows per sequence, then the drafts and the outputs
+    assert bench.verify_algorithmic_bytes(2, 3, 10, 2) == 2 * 7 * 10 * 2 + 2 * 3 * 4 + 2 * 5 * 4
+
+
+def test_sweep_reference_arm_says_why_it_is_unavailable(capsys):
+    import bench
+    import sys
+    argv = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--workload", "verifier_sweep"]
+    try:
+        assert bench.main() == 0
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and "unavailable" in line

@@ -254,11 +254,35 @@ def test_valid_calls_without_a_device_report_an_error(lib):
                                                 fake, fake, 512, 256, 512, 32, 0, fake, need_d,
                                                 None)] in bad
     assert STATUS[lib.uno_sample_drafts(fake, 2, 4, 1000, 0, u64(0), u64(0), fake, None)] in bad
+    assert STATUS[lib.uno_sample_drafts_blocks(fake, 2, 4, 5, 1000, 0, u64(0), u64(0), fake,
+                                               None)] in bad
     need_t = lib.uno_tree_draft_workspace_bytes(2, 3, 1000, 2)
     assert STATUS[lib.uno_tree_draft(fake, 2, 3, 1000, 0, 2, 2, fake, fake, fake, fake, fake,
                                      fake, fake, need_t, None)] in bad
     assert STATUS[lib.uno_tree_verify(fake, fake, fake, fake, fake, 2, 3, 2, 1000, 0, u64(0),
                                       u64(0), fake, fake, fake, None)] in bad
+
+
+def test_sampler_argument_errors_need_no_gpu(lib):
+    """uno_sample_drafts_blocks checks dtype, sizes (block_rows >= K), the empty
+    batch, null pointers and alignment before it looks for a device."""
+    from lossless_decoding_b200._lib import STATUS
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 1)
+    u64 = ctypes.c_uint64
+
+    def s(B, K, R, V, dt, q=fake, out=fake):
+        return STATUS[lib.uno_sample_drafts_blocks(q, B, K, R, V, dt, u64(0), u64(0), out, None)]
+
+    assert s(2, 4, 5, 1000, 7) == "UNO_ERR_DTYPE"
+    assert s(2, 0, 5, 1000, 0) == "UNO_ERR_SIZE"
+    assert s(2, 4, 3, 1000, 0) == "UNO_ERR_SIZE"      # fewer rows per block than drafts
+    assert s(2, 4, 5000, 1000, 0) == "UNO_ERR_SIZE"   # block_rows above 4096
+    assert s(2, 4, 5, 0, 0) == "UNO_ERR_SIZE"
+    assert s(0, 4, 5, 1000, 0) == "UNO_OK"
+    assert s(2, 4, 5, 1000, 0, q=None) == "UNO_ERR_NULL"
+    assert s(2, 4, 5, 1000, 0, out=None) == "UNO_ERR_NULL"
+    assert s(2, 4, 5, 1000, 0, q=odd) == "UNO_ERR_ALIGN"
 
 
 def test_noalloc_checks_sizes_before_the_empty_batch(lib):

@@ -93,3 +93,19 @@ def test_chisquare_on_device(api):
     counts = np.bincount(got.cpu().numpy().reshape(-1), minlength=V)
     expected = sp_softmax(row.astype(np.float64)) * B * K
     assert chisquare(counts, expected).pvalue > 1e-4
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_blocks_of_k_plus_one_rows_read_in_place(api, dtype):
+    """Drawing the first K rows of each block of K + 1 (the LM head's
+    draft-pathway layout) gives the ids of the same rows copied out
+    contiguously, bit for bit: same rows, same counters."""
+    B, K, V = 6, 5, 3001
+    v = verify_inputs(B, K + 1, V, dtype=dtype, dist="gumbel", sigma=1.0, seed=31, device=DEV)
+    blocks = v.p_logits  # [B, K + 2, V]: any block of at least K + 1 rows works
+    R = blocks.shape[1]
+    got = api.sample_drafts(blocks, 77, 3, num_drafts=K)
+    ref = api.sample_drafts(blocks[:, :K].contiguous(), 77, 3)
+    torch.cuda.synchronize()
+    assert got.shape == (B, K) and R > K
+    assert torch.equal(got, ref)
