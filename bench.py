@@ -516,6 +516,7 @@ class StackStep(BatchedDecode):
     """
 
     name = "qwen3_8b_stack_b64_k16"
+    long_step = True  # ~20 ms of GEMMs per step: the sustained tensor peak applies
     verify_kernels = ("verify_decide_kernel + verify_draw_kernel (row statistics from the "
                       "LM head's epilogue; no streaming pass)")
 
@@ -960,12 +961,18 @@ def run_ours(args):
     gemm_kernel = "dual_kernel (T tiles, x W^T and T Bm^T, one persistent launch)"
     gemm_bytes = getattr(wl, "gemm_bytes", None)
     if gemm_bytes is None:  # tensor-core bound: FLOPs against the dense bf16 peak
+        # a step of many milliseconds of back-to-back GEMMs runs under the power
+        # cap: its peak is the sustained one; a short step takes the burst peak
+        sustained = getattr(wl, "long_step", False) and peaks.get("bf16_sustained")
+        peak_tf = peaks["bf16_sustained"] if sustained else peaks["bf16"]
+        kind = "sustained (seconds-long loop under the power cap)" if sustained else "burst"
         roof_gemm = {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops,
-                     "peak": peaks["bf16"], "unit": "TFLOP/s",
-                     "frac": gemm_tflops / peaks["bf16"],
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak_tf,
+                     "frac_burst": gemm_tflops / peaks["bf16"],
                      "frac_datasheet": gemm_tflops / DATASHEET["bf16"],
                      "traffic": measured_traffic(args.workload, "dual"),
-                     "peak_kind": f"bf16 dense burst, {peaks['src']}; datasheet 2250 TFLOP/s",
+                     "peak_kind": f"bf16 dense {kind}, {peaks['src']}; datasheet 2250 TFLOP/s",
                      "algorithmic_per_launch": wl.gemm_flops / len(wl.layers),
                      "ms_per_step": gemm_avg}
     else:  # few rows: the stream of W bounds it, bytes against the HBM peak
@@ -978,8 +985,7 @@ def run_ours(args):
                      "algorithmic_per_launch": gemm_bytes / len(wl.layers),
                      "tflops": gemm_tflops, "ms_per_step": gemm_avg}
     roof_ver = {"kernel": getattr(wl, "verify_kernels",
-                                  "verify_stream_kernel + verify_decide_kernel"
-                                  " + verify_draw_kernel"),
+                                  "verify_stream_kernel + verify_draw_kernel"),
                 "bound": "hbm", "achieved": ver_gbs,
                 "peak": peaks["hbm"], "unit": "GB/s", "frac": ver_gbs / peaks["hbm"],
                 "frac_datasheet": ver_gbs / DATASHEET["hbm"],
