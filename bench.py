@@ -76,13 +76,13 @@ def _peaks():
 # profiles/. A figure is reported only while the kernel source it was taken on
 # is unchanged (first 16 hex digits of its sha256), else traffic is null.
 MEASURED_TRAFFIC = {
-    # dual_kernel: average of the step's four launches (63.6 + 3.2, 44.1 + 0.3,
-    # 226.3 + 75.0, 130.1 + 0.1 MB read + written)
-    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "18958f12048c1c41", 135.7e6),
-    # sample_drafts_kernel over the 64 x 16 q rows: 314.9 MB read + 5.3 MB written
-    ("batched_decode_b64_k16", "draft"): ("draft_sample.cu", "9369b9644cfaf3fe", 320.2e6),
-    # stream 645.2 MB + decide 0.3 MB + draw 39.0 MB, per verifier call
-    ("batched_decode_b64_k16", "verify"): ("verify.cu", "dd3ee9362484308a", 684.5e6),
+    # dual_kernel: average of the step's four launches (63.6 + 3.2, 44.1 + 0.2,
+    # 221.5 + 71.2, 130.1 + 0.1 MB read + written)
+    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "b24445947d4d0319", 133.48e6),
+    # sample_drafts_kernel over the 64 x 16 q rows: 314.5 MB read + 3.7 MB written
+    ("batched_decode_b64_k16", "draft"): ("draft_sample.cu", "3615bc39b13f88bc", 318.13e6),
+    # stream 641.8 MB read + 0.5 MB written, draw 39.0 MB read, per verifier call
+    ("batched_decode_b64_k16", "verify"): ("verify.cu", "696e7dfc1a0a17f7", 681.36e6),
 }
 
 
