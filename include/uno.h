@@ -387,6 +387,16 @@ int uno_tree_verify(const void* p_logits, const int32_t* node_token, const int32
  * ------------------------------------------------------------------------ */
 int uno_device_fault_flags(int clear, unsigned int* flags);
 
+/* Failure-path test hook of the dual-path linear (for tests, not for use):
+ * the calls that follow in this process bound every wait of the GEMM by
+ * wait_ns nanoseconds instead of one second, and, when t_flag_skew is non-zero,
+ * make its TMA producers wait for a T-tile flag value that no tile writes (the
+ * call's value plus the skew), so that those waits run out: the kernel then
+ * sets fault bits, abandons its work (outputs undefined) and exits normally,
+ * and the context stays usable. (0, 0) restores normal operation. Always
+ * returns UNO_OK. */
+int uno_dualpath_test_hooks(uint64_t wait_ns, uint32_t t_flag_skew);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -88,6 +88,8 @@ def _load() -> ctypes.CDLL:
     L.uno_tree_verify.restype = i32
     L.uno_device_fault_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint)]
     L.uno_device_fault_flags.restype = i32
+    L.uno_dualpath_test_hooks.argtypes = [u64, ctypes.c_uint32]
+    L.uno_dualpath_test_hooks.restype = i32
     return L
 
 

@@ -68,7 +68,7 @@ constexpr int kGemmThreads = (kFirstProducer + kProducers) * 32;
 constexpr int kInsert = 6;         // main K-blocks of the next tile before an adapter
 constexpr int kPrefetch = 8;       // K-blocks of L2 prefetch ahead of the weight loads
 constexpr int kMaxSplit = 4;       // K-pieces of a split tile, at most
-constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint64_t kWaitNs = 1000000000ull;  // default limit of every bounded wait
 
 enum : unsigned { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
 
@@ -102,6 +102,9 @@ struct GemmParams {
   uint32_t idesc_t;   // instruction descriptor of the T tiles
   int t_brows;        // rows of the B box of a T-tile item (per CTA)
   uint32_t epoch;     // value a T tile's flag takes once T is stored
+  uint32_t t_wait_epoch;  // value a producer waits for on a T flag (== epoch, except
+                          // under the failure-path test hook: a value no tile writes)
+  uint64_t wait_ns;   // limit of every bounded wait (1 s; shorter under the test hook)
   int main_tiles;     // main tiles over all projections
   // The last, partial round of main tiles may be split along K so that it
   // fills the GPU: units [split_start, split_start + n_split * split_k) are
@@ -160,8 +163,16 @@ __host__ __device__ constexpr int stages_for() {
   return PAIR ? 3 : (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8));
 }
 
+// Barriers after the ring: full and empty per stage, 8 per-buffer barriers,
+// t_stored, mma_done[2]; then the TMEM address and the issuers' hand-over word.
+template <int BN, bool PAIR>
+__host__ __device__ constexpr int barrier_bytes() {
+  return (2 * stages_for<BN, PAIR>() + 8 + 1 + 2) * 8 + 4 + 4;
+}
+
 template <int BN, bool PAIR>
 __host__ __device__ constexpr int smem_bytes() {
+  static_assert(barrier_bytes<BN, PAIR>() <= 256, "barrier region");
   return stages_for<BN, PAIR>() * stage_bytes<BN, PAIR>() + 1024 /*align*/ + 256 /*barriers*/;
 }
 
@@ -282,12 +293,12 @@ __device__ __forceinline__ int ld_acquire_shared(const int* p) {
 }
 
 // Bounded wait until the other MMA issuer has handed over ring item `it`.
-__device__ bool wait_order(const int* order, int it, volatile int* abort_flag) {
+__device__ bool wait_order(const int* order, int it, volatile int* abort_flag, uint64_t limit_ns) {
   if (ld_acquire_shared(order) == it) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   for (uint32_t k = 1;; ++k) {
     if (ld_acquire_shared(order) == it) return true;
-    if ((k & 255u) == 0 && (*abort_flag || sm100::globaltimer_ns() - t0 > kWaitNs)) return false;
+    if ((k & 255u) == 0 && (*abort_flag || sm100::globaltimer_ns() - t0 > limit_ns)) return false;
   }
 }
 
@@ -317,7 +328,7 @@ __device__ __forceinline__ void arrive_at(uint32_t bar_cluster_addr) {
 
 // Bounded wait with cluster-scope acquire (barriers that a peer CTA or the
 // pair's tensor core arrives on).
-__device__ bool wait_cl(uint64_t* bar, uint32_t parity) {
+__device__ bool wait_cl(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = sm100::globaltimer_ns();
   for (uint32_t k = 0;; ++k) {
     uint32_t ok;
@@ -329,7 +340,7 @@ __device__ bool wait_cl(uint64_t* bar, uint32_t parity) {
         : "r"(sm100::smem_addr(bar)), "r"(parity)
         : "memory");
     if (ok) return true;
-    if ((k & 255u) == 255u && sm100::globaltimer_ns() - t0 > kWaitNs) return false;
+    if ((k & 255u) == 255u && sm100::globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -372,13 +383,13 @@ __device__ __forceinline__ void commit_pair(uint64_t* bar) {
 }
 
 // Bounded wait until *flag == epoch.
-__device__ bool wait_flag(const uint32_t* flag, uint32_t epoch) {
+__device__ bool wait_flag(const uint32_t* flag, uint32_t epoch, uint64_t limit_ns) {
   if (ld_acquire_u32(flag) == epoch) return true;
   const uint64_t t0 = sm100::globaltimer_ns();
   for (;;) {
     __nanosleep(64);
     if (ld_acquire_u32(flag) == epoch) return true;
-    if (sm100::globaltimer_ns() - t0 > kWaitNs) return false;
+    if (sm100::globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -418,7 +429,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* draft_full = ar_read + 2;       // [2] adapter product done
   uint64_t* acc_empty = draft_full + 2;     // [2] epilogue drained the buffer
   uint64_t* t_stored = acc_empty + 2;       // [1] epilogue warps stored a T tile
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(t_stored + 1);
+  uint64_t* mma_done = t_stored + 1;        // [2] every MMA of issuer e has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
   int* order = reinterpret_cast<int*>(tmem_holder + 1);  // next ring item to issue
   __shared__ volatile int abort_flag;
 
@@ -456,6 +468,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::mbar_init(&acc_empty[b], kEpiArrivals);
     }
     sm100::mbar_init(t_stored, kEpiArrivals);
+    sm100::mbar_init(&mma_done[0], 1);
+    sm100::mbar_init(&mma_done[1], 1);
     *order = 0;
     abort_flag = 0;
     sm100::fence_mbar_init();
@@ -590,7 +604,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t bar_pair = 0;
       auto begin_item = [&](int b_rows, int nk) -> uint8_t* {
         const int s = it % STAGES;
-        if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1)) {
+        if (it >= STAGES && !sm100::mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, p.wait_ns)) {
           set_fault(kFaultProducer, &abort_flag);
           ok = false;
           return nullptr;
@@ -669,9 +683,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ready = true;
             const uint32_t* fl = p.g[owner.g].t_flags;
             if constexpr (SWAP) {
-              for (int t = 0; t < p.nT && ready; ++t) ready = wait_flag(fl + t, p.epoch);
+              for (int t = 0; t < p.nT && ready; ++t)
+                ready = wait_flag(fl + t, p.t_wait_epoch, p.wait_ns);
             } else {
-              ready = wait_flag(fl + owner.a0 / kRows, p.epoch);
+              ready = wait_flag(fl + owner.a0 / kRows, p.t_wait_epoch, p.wait_ns);
             }
             if (!ready) {
               set_fault(kFaultProducer, &abort_flag);
@@ -698,7 +713,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // producer's items among the last STAGES (the leader's full barriers
       // count the copies of both CTAs; the pair then meets at a cluster barrier).
       for (int k = (it > STAGES ? it - STAGES : 0); leader && k < it && k <= last_mine; ++k)
-        if (k % kProducers == pr && !sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1))
+        if (k % kProducers == pr &&
+            !sm100::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1, p.wait_ns))
           set_fault(kFaultProducer, &abort_flag);
     }
   } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
@@ -726,8 +742,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // MMA overwrites the accumulator unless accumulate_first.
       auto issue = [&](uint32_t d, uint32_t idesc, bool accumulate_first, int nk) {
         const int s = it % STAGES;
-        if (!wait_order(order, it, &abort_flag) ||
-            !sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1)) {
+        if (!wait_order(order, it, &abort_flag, p.wait_ns) ||
+            !sm100::mbar_wait(&full_bar[s], (it / STAGES) & 1, p.wait_ns)) {
           fail();
           return;
         }
@@ -767,7 +783,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (kind == 1) {
             if (mine) {
               if (j == 0) {
-                if (!wait_cl(&ar_read[mo & 1], (mo >> 1) & 1)) {
+                if (!wait_cl(&ar_read[mo & 1], (mo >> 1) & 1, p.wait_ns)) {
                   fail();
                   break;
                 }
@@ -781,7 +797,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (mine) {
               if (j == 0 && li >= 1) {
                 // the other buffer is free once tile li-1 has been drained
-                if (!wait_cl(&acc_empty[pbuf], ((li - 1) >> 1) & 1)) {
+                if (!wait_cl(&acc_empty[pbuf], ((li - 1) >> 1) & 1, p.wait_ns)) {
                   fail();
                   break;
                 }
@@ -793,7 +809,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             if (mine) {
               if (j == 0 && li >= 2) {
-                if (!wait_cl(&acc_empty[buf], ((li >> 1) - 1) & 1)) {
+                if (!wait_cl(&acc_empty[buf], ((li >> 1) - 1) & 1, p.wait_ns)) {
                   fail();
                   break;
                 }
@@ -805,6 +821,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      // Before TMEM is released every MMA this thread issued must have
+      // completed, on the normal path and after an abort alike: a commit
+      // tracks all of them (with the pair it also arrives, unused, on the
+      // second CTA's barrier).
+      commit(&mma_done[e]);
+      if (!sm100::mbar_wait(&mma_done[e], 0, p.wait_ns)) set_fault(kFaultMma, &abort_flag);
+    } else if constexpr (PAIR) {
+      // the second CTA: the leader's last commits arrive here too; wait for
+      // them so that no arrival targets this CTA's shared memory after it exits
+      if (lane == 0 && !sm100::mbar_wait(&mma_done[warp - kMmaWarp0], 0, p.wait_ns))
+        set_fault(kFaultMma, &abort_flag);
     }
   } else {
     // ---- epilogue: warps 0..3, TMEM lane quarter = warp ----
@@ -1010,7 +1037,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int buf = li & 1;
       const uint32_t acc = tmem + static_cast<uint32_t>(buf * kAcc);
       const Tile x = tile_at(li);
-      const bool got = __all_sync(0xFFFFFFFFu, wait_cl(&acc_full[buf], (li >> 1) & 1));
+      const bool got = __all_sync(0xFFFFFFFFu, wait_cl(&acc_full[buf], (li >> 1) & 1, p.wait_ns));
       if (!got || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
@@ -1036,7 +1063,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
           arrive_leader(t_stored);
           if (warp == 0 && leader) {
-            if (wait_cl(t_stored, li & 1)) {
+            if (wait_cl(t_stored, li & 1, p.wait_ns)) {
               fence_proxy_async_global();
               st_release_u32(p.g[gi].t_flags + x.tt, p.epoch);
             } else {
@@ -1076,7 +1103,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) {
             arrive_leader(t_stored);  // this CTA's T tiles used phases 0 .. nt_mine-1
             if (warp == 0 && leader) {
-              if (wait_cl(t_stored, nt_mine & 1))
+              if (wait_cl(t_stored, nt_mine & 1, p.wait_ns))
                 st_release_u32(pflags + (x.piece - 1), p.epoch);
               else
                 set_fault(kFaultEpilogue, &abort_flag);
@@ -1088,7 +1115,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // piece 0: wait for the other pieces, add their partials into TMEM
         bool ready = true;
         if (lane == 0)
-          for (int q = 1; q < p.split_k && ready; ++q) ready = wait_flag(pflags + (q - 1), p.epoch);
+          for (int q = 1; q < p.split_k && ready; ++q)
+            ready = wait_flag(pflags + (q - 1), p.epoch, p.wait_ns);
         ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
         __syncwarp();  // orders lane 0's acquire before the other lanes' loads
         if (!ready) {
@@ -1142,7 +1170,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int mo = li - nt_mine;
       if (lane == 0) arrive_leader(adapter ? &ar_read[mo & 1] : &acc_empty[buf]);
       if (!adapter) continue;
-      const bool got2 = __all_sync(0xFFFFFFFFu, wait_cl(&draft_full[mo & 1], (mo >> 1) & 1));
+      const bool got2 = __all_sync(0xFFFFFFFFu, wait_cl(&draft_full[mo & 1], (mo >> 1) & 1, p.wait_ns));
       if (!got2 || abort_flag) {
         if (lane == 0) set_fault(kFaultEpilogue, &abort_flag);
         break;
@@ -1233,6 +1261,12 @@ int sm_count() {
 
 // A fresh value per call for the T-tile flags. Seeded from the clock so that
 // a workspace left over from another process is not mistaken for this call's.
+// Failure-path test hook (uno_dualpath_test_hooks): a shorter limit for every
+// bounded wait, and a skew that makes producers wait for a T-flag value no
+// tile writes. Zero: normal operation.
+std::atomic<uint64_t> g_test_wait_ns{0};
+std::atomic<uint32_t> g_test_t_skew{0};
+
 uint32_t next_epoch() {
   static std::atomic<uint32_t> counter{0};
   static std::once_flag once;
@@ -1421,6 +1455,13 @@ int run_dualpath(int n, const void* x, const void* const* W, const void* const* 
   gp.r = r;
   gp.gate = gate;
   gp.epoch = next_epoch();
+  {
+    const uint64_t w = g_test_wait_ns.load();
+    const uint32_t skew = g_test_t_skew.load();
+    gp.wait_ns = w ? w : kWaitNs;
+    gp.t_wait_epoch = gp.epoch + skew;
+    if (skew != 0 && gp.t_wait_epoch == 0) gp.t_wait_epoch = 1;  // 0 is a cleared flag
+  }
   DualMaps maps;
   const int bn = pl.swap ? bn_for(M) : 256;
   const int n_t = (r + 15) / 16 * 16;  // N of the unswapped T tiles
@@ -1600,6 +1641,12 @@ extern "C" int uno_dualpath_linear_stats(const void* x, const void* W, const voi
   if (!uno_host::aligned(stats_ar, 8) || !uno_host::aligned(stats_draft, 8)) return UNO_ERR_ALIGN;
   return dispatch(1, x, &W, &A, &Bm, &scale, gate, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,
                   workspace, workspace_bytes, stream, &stats_ar, &stats_draft);
+}
+
+extern "C" int uno_dualpath_test_hooks(uint64_t wait_ns, uint32_t t_flag_skew) {
+  g_test_wait_ns.store(wait_ns);
+  g_test_t_skew.store(t_flag_skew);
+  return UNO_OK;
 }
 
 extern "C" int uno_device_fault_flags(int clear, unsigned int* flags) {
