@@ -46,8 +46,9 @@ constexpr int kMinSteps = 16;     // vectors per lane in a chunk, at least
 
 // Launch shapes. Many rows (a 64 x 16 block of drafts): two 128-thread CTAs
 // per row, 8 per SM, in about two waves that the hardware balances over the
-// SMs. Few rows (a tree's node rows at batch 1): four 512-thread CTAs per row,
-// so that a handful of rows still keeps enough loads in flight.
+// SMs. Few rows (a tree's node rows at batch 1, a single sequence's drafts):
+// clusters of four or eight 256-thread CTAs per row, 4 per SM, so that a
+// handful of rows still keeps enough loads in flight in one wave.
 template <int THREADS, int CTAS_PER_SM, int CLUSTER>
 struct Shape {
   static constexpr int kThreads = THREADS;
@@ -56,10 +57,12 @@ struct Shape {
   static constexpr int kCluster = CLUSTER;  // CTAs per row
 };
 using Narrow = Shape<128, 8, 2>;
-using Wide = Shape<512, 2, 4>;
+using Wide = Shape<256, 4, 4>;      // at most kWideRows rows
+using Widest = Shape<256, 4, 8>;    // at most kWidestRows rows
 constexpr int kRound = 4;   // 16-byte vectors per lane per round (a chunk is whole rounds)
 constexpr int kStages = 3;  // ring stages per warp, one round each
-constexpr int kWideRows = 2 * 148;  // at most this many rows: the wide shape
+constexpr int kWideRows = 2 * 148;   // rows of the wide shape, at most
+constexpr int kWidestRows = 74;      // rows of the widest shape: one wave of 8-CTA clusters
 using uno::kLog2e;
 
 struct SampleParams {
@@ -394,7 +397,10 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
 
 int uno_host::sample_rows(const RowDraws& r, cudaStream_t st) {
   if (r.B == 0 || r.rows_per_seq == 0) return UNO_OK;
-  if (static_cast<long long>(r.B) * r.rows_per_seq <= kWideRows)
+  const long long rows = static_cast<long long>(r.B) * r.rows_per_seq;
+  if (rows <= kWidestRows)
+    return (r.dtype == UNO_BF16) ? run<uint16_t, Widest>(r, st) : run<float, Widest>(r, st);
+  if (rows <= kWideRows)
     return (r.dtype == UNO_BF16) ? run<uint16_t, Wide>(r, st) : run<float, Wide>(r, st);
   return (r.dtype == UNO_BF16) ? run<uint16_t, Narrow>(r, st) : run<float, Narrow>(r, st);
 }

@@ -9,7 +9,7 @@
 // here depth D = B - 1 (positions after the block's AR-only first token),
 // top_k and budget.
 //
-// Drafting, three launches:
+// Drafting, two launches:
 //   tree_topk_part_kernel   one CTA per (row, slab): a row of a few sequences
 //                      is split over several CTAs so that low-batch drafting
 //                      still keeps the SMs' loads in flight. Each thread keeps
@@ -18,9 +18,9 @@
 //                      of 2^(x - max)); the CTA merges the lists in top_k
 //                      argmax rounds and writes the slab's list and (max, sum)
 //                      to the workspace.
-//   tree_topk_merge_kernel  one warp per row merges its slabs and writes the
-//                      ids and log softmax(q)(id) = x - logsumexp.
-//   tree_build_kernel  one CTA per sequence: the budget best sequences by
+//   tree_build_kernel  one CTA per sequence: one warp per row merges its
+//                      slabs and writes the ids and log softmax(q)(id) =
+//                      x - logsumexp; then the budget best sequences by
 //                      joint log-probability, one position at a time (the
 //                      best budget sequences of j + 1 positions extend the
 //                      best budget of j positions); a candidate (prefix p,
@@ -34,8 +34,10 @@
 //   draws              one inverse-CDF draw per tree node from its AR row
 //                      (the sampler's row-draw kernel, uniform = word 1 of
 //                      the Philox block (b, depth, step));
-//   tree_walk_kernel   one thread per sequence: follow the draw while it is
-//                      the token of a child, emit it and stop otherwise.
+//   tree_walk_kernel   one CTA per sequence: the tree in shared memory, each
+//                      node's children located there; one thread follows the
+//                      draw while it is the token of a child, emits it and
+//                      stops otherwise.
 #include <algorithm>
 #include <climits>
 #include <cstdint>
@@ -54,9 +56,10 @@ constexpr int kTopInFlight = 4;   // 16-byte loads in flight per thread
 constexpr int kMaxTopK = 16;      // rank of a choice fits 4 bits
 constexpr int kMaxDepth = 16;     // 16 positions x 4 bits = one 64-bit tuple
 constexpr int kMaxBudget = 64;
-constexpr int kBuildThreads = 256;
+constexpr int kBuildThreads = 512;  // a warp per row for the merge (D <= 16)
 constexpr int kMaxCand = 256;     // candidates of one position step
 constexpr int kWalkThreads = 128;
+constexpr int kMaxNodes = 1 + kMaxDepth * kMaxBudget;  // nodes of a tree, at most
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -243,31 +246,59 @@ __global__ void __launch_bounds__(kTopThreads) tree_topk_part_kernel(const TopkP
   }
 }
 
-// Stage 2: one warp per row merges the slabs' lists and (max, sum) pairs and
-// writes the row's top_k ids with log softmax = x - logsumexp.
+// Stage 2 (first part of the build launch): one warp merges a row's slab
+// lists and (max, sum) pairs and writes the row's top_k ids with log softmax
+// = x - logsumexp, to global memory and to the given shared arrays.
 template <int KM>
-__global__ void __launch_bounds__(32) tree_topk_merge_kernel(const TopkParams P) {
-  uno::launch_dependents();
-  uno::grid_dependency_wait();
-  const int lane = threadIdx.x, rw = blockIdx.x;
+__device__ void merge_row(const TopkParams& P, int rw, int lane, int32_t* s_id, float* s_lq) {
   const size_t p0 = static_cast<size_t>(rw) * P.slabs;
-  float m = -INFINITY;
-  for (int sl = lane; sl < P.slabs; sl += 32) m = fmaxf(m, P.part_m[p0 + sl]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  float sum = 0.f;
-  for (int sl = lane; sl < P.slabs; sl += 32) {
-    const float ms = P.part_m[p0 + sl];
-    if (ms > -INFINITY) sum += P.part_s[p0 + sl] * uno::ex2(ms - m);
+  // the slabs' (max, sum) pairs: a lane merges its slabs (at most two when
+  // there are 64), then the warp
+  float m = -INFINITY, sum = 0.f;
+  for (int sl = lane; sl < P.slabs; sl += 64) {
+    const bool two = sl + 32 < P.slabs;
+    const float m1 = __ldcg(P.part_m + p0 + sl), s1 = __ldcg(P.part_s + p0 + sl);
+    const float m2 = two ? __ldcg(P.part_m + p0 + sl + 32) : -INFINITY;
+    const float s2 = two ? __ldcg(P.part_s + p0 + sl + 32) : 0.f;
+    const float mm = fmaxf(m, fmaxf(m1, m2));
+    if (mm > -INFINITY) {
+      sum = ((m > -INFINITY) ? sum * uno::ex2(m - mm) : 0.f) +
+            ((m1 > -INFINITY) ? s1 * uno::ex2(m1 - mm) : 0.f) +
+            ((m2 > -INFINITY) ? s2 * uno::ex2(m2 - mm) : 0.f);
+      m = mm;
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+    const float s2 = __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    const float mm = fmaxf(m, m2);
+    if (mm > -INFINITY) {
+      sum = ((m > -INFINITY) ? sum * uno::ex2(m - mm) : 0.f) +
+            ((m2 > -INFINITY) ? s2 * uno::ex2(m2 - mm) : 0.f);
+      m = mm;
+    }
+  }
   const float lse = (m > -INFINITY) ? (m + log2f(sum)) * kLn2 : -INFINITY;
 
   TopList<KM> top;
   top.init();
   const int n = P.slabs * P.top_k;
-  for (int c = lane; c < n; c += 32) top.offer(P.part_val[p0 * P.top_k + c], P.part_id[p0 * P.top_k + c]);
+  const float* pv = P.part_val + p0 * P.top_k;
+  const int32_t* pi = P.part_id + p0 * P.top_k;
+  constexpr int kBatch = 8;  // loads issued before any is used
+  for (int c0 = lane; c0 < n; c0 += 32 * kBatch) {
+    float v[kBatch];
+    int id[kBatch];
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) {
+      const int c = c0 + 32 * e;
+      v[e] = (c < n) ? __ldcg(pv + c) : -INFINITY;
+      id[e] = (c < n) ? __ldcg(pi + c) : INT_MAX;
+    }
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) top.offer(v[e], id[e]);
+  }
   int32_t* out_i = P.ids + static_cast<size_t>(rw) * P.top_k;
   float* out_l = P.logq + static_cast<size_t>(rw) * P.top_k;
   for (int r = 0; r < P.top_k; ++r) {
@@ -285,15 +316,17 @@ __global__ void __launch_bounds__(32) tree_topk_merge_kernel(const TopkParams P)
     const bool found = bv > -INFINITY;
     if (found && top.i[0] == bi) top.pop();
     if (lane == 0) {
-      out_i[r] = found ? bi : -1;
-      out_l[r] = found ? bv - lse : -INFINITY;
+      const int id = found ? bi : -1;
+      const float lq = found ? bv - lse : -INFINITY;
+      out_i[r] = id;
+      out_l[r] = lq;
+      s_id[r] = id;
+      s_lq[r] = lq;
     }
   }
 }
 
 struct BuildParams {
-  const int32_t* ids;  // [B][D][top_k]
-  const float* logq;   // [B][D][top_k]
   int B, D, top_k, budget, N;
   int32_t* node_token;   // [B][N]
   int32_t* node_parent;  // [B][N]
@@ -305,23 +338,43 @@ __device__ __forceinline__ unsigned long long prefix_of(unsigned long long t, in
   return t >> (4 * (kMaxDepth - j));  // the first j ranks (1 <= j <= kMaxDepth)
 }
 
-__global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const BuildParams P) {
+// One CTA per sequence: the merge of its D rows' slab lists (stage 2), then
+// the kept set and its prefix tree.
+template <int KM>
+__global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkParams TP,
+                                                                   const BuildParams P) {
   __shared__ float k_score[2][kMaxBudget];
   __shared__ unsigned long long k_tup[2][kMaxBudget];
   __shared__ float c_score[kMaxCand];
   __shared__ unsigned long long c_tup[kMaxCand];
   __shared__ float s_lq[kMaxDepth][kMaxTopK];
+  __shared__ int32_t s_ids[kMaxDepth][kMaxTopK];
   __shared__ int s_avail[kMaxDepth];
+  // s_coff[a][p]: first candidate slot of prefix p when a choices are available
+  // (prefix p owns min(a, budget / (p + 1)) slots); s_coff[a][nk] = their number
+  __shared__ int s_coff[kMaxTopK + 1][kMaxBudget + 1];
+  __shared__ int s_cap[kMaxBudget];  // budget / (p + 1)
   __shared__ unsigned char s_rep[kMaxDepth][kMaxBudget];
+  __shared__ int s_cnt[kMaxDepth + 1];
   __shared__ int s_off[kMaxDepth + 2];
+  __shared__ int s_final[2];  // buffer and size of the final kept set
   uno::launch_dependents();
   uno::grid_dependency_wait();
-  const int b = blockIdx.x, tid = threadIdx.x;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int D = P.D, k = P.top_k, budget = P.budget;
-  const float* lq = P.logq + static_cast<size_t>(b) * D * k;
-  const int32_t* ids = P.ids + static_cast<size_t>(b) * D * k;
-  // every position's log-probabilities in one round trip
-  for (int e = tid; e < D * k; e += kBuildThreads) s_lq[e / k][e % k] = lq[e];
+  for (int q = tid; q < budget; q += kBuildThreads) s_cap[q] = budget / (q + 1);
+  // the D rows' merges, one warp per row
+  for (int j = warp; j < D; j += kBuildThreads / 32)
+    merge_row<KM>(TP, b * D + j, lane, s_ids[j], s_lq[j]);
+  __syncthreads();
+  for (int a = tid; a <= k; a += kBuildThreads) {
+    int off = 0;
+    for (int q = 0; q < budget; ++q) {
+      s_coff[a][q] = off;
+      off += min(a, s_cap[q]);
+    }
+    s_coff[a][budget] = off;
+  }
   if (tid == 0) {
     k_score[0][0] = 0.f;  // the empty prefix
     k_tup[0][0] = 0ull;
@@ -333,46 +386,62 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const BuildPa
     s_avail[tid] = a;
   }
   __syncthreads();
-  int cur = 0, nk = 1;
-  for (int j = 0; j < D; ++j) {
-    const int avail = s_avail[j];
-    // candidates (p, s) with (p + 1)(s + 1) <= budget: prefix p owns a run of
-    // min(avail, budget / (p + 1)) slots starting at the sum of the runs before
-    int nc = 0, off = 0;
-    for (int p = 0; p < nk; ++p) {
-      const int c = min(avail, budget / (p + 1));
-      if (p < tid) off += c;
-      nc += c;
-    }
-    if (tid < nk) {
-      const float ps = k_score[cur][tid];
-      const unsigned long long pt = k_tup[cur][tid];
-      const int cnt = min(avail, budget / (tid + 1));
-      for (int s = 0; s < cnt; ++s) {
-        c_score[off + s] = ps + s_lq[j][s];
-        c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << (4 * (kMaxDepth - 1 - j)));
+  // The kept set, position by position, in warp 0 alone (the steps are
+  // short and dependent: warp-synchronous, no CTA barrier between them).
+  if (warp == 0) {
+    int cur = 0, nk = 1;
+    for (int j = 0; j < D; ++j) {
+      const int avail = s_avail[j];
+      // candidates (p, s) with (p + 1)(s + 1) <= budget: prefix p owns a run
+      // of min(avail, budget / (p + 1)) slots from s_coff[avail][p]
+      const int nc = s_coff[avail][nk];
+      const unsigned long long shift = 4ull * (kMaxDepth - 1 - j);
+      for (int p = lane; p < nk; p += 32) {
+        const int off = s_coff[avail][p];
+        const int cnt = s_coff[avail][p + 1] - off;
+        const float ps = k_score[cur][p];
+        const unsigned long long pt = k_tup[cur][p];
+        for (int s = 0; s < cnt; ++s) {
+          c_score[off + s] = ps + s_lq[j][s];
+          c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << shift);
+        }
       }
-    }
-    __syncthreads();
-    const int nxt = cur ^ 1;
-    const int keep = min(budget, nc);
-    for (int c = tid; c < nc; c += kBuildThreads) {
-      const float sc = c_score[c];
-      const unsigned long long tu = c_tup[c];
-      int rank = 0;
-      for (int o = 0; o < nc; ++o) {
-        const float so = c_score[o];
-        rank += (so > sc || (so == sc && c_tup[o] < tu)) ? 1 : 0;
+      __syncwarp();
+      const int nxt = cur ^ 1;
+      const int keep = min(budget, nc);
+      // rank of candidate c = the candidates ahead of it (lane c mod 32)
+      for (int c = lane; c < nc; c += 32) {
+        const float sc = c_score[c];
+        const unsigned long long tu = c_tup[c];
+        int a0 = 0, a1 = 0;
+        int o = 0;
+        for (; o + 1 < nc; o += 2) {  // two independent comparisons per step
+          const float s0 = c_score[o], s1 = c_score[o + 1];
+          const unsigned long long t0 = c_tup[o], t1 = c_tup[o + 1];
+          a0 += (s0 > sc || (s0 == sc && t0 < tu)) ? 1 : 0;
+          a1 += (s1 > sc || (s1 == sc && t1 < tu)) ? 1 : 0;
+        }
+        if (o < nc) {
+          const float s0 = c_score[o];
+          a0 += (s0 > sc || (s0 == sc && c_tup[o] < tu)) ? 1 : 0;
+        }
+        const int rank = a0 + a1;
+        if (rank < keep) {
+          k_score[nxt][rank] = sc;
+          k_tup[nxt][rank] = tu;
+        }
       }
-      if (rank < keep) {
-        k_score[nxt][rank] = sc;
-        k_tup[nxt][rank] = tu;
-      }
+      __syncwarp();
+      cur = nxt;
+      nk = keep;
     }
-    __syncthreads();
-    cur = nxt;
-    nk = keep;
+    if (lane == 0) {
+      s_final[0] = cur;
+      s_final[1] = nk;
+    }
   }
+  __syncthreads();
+  const int cur = s_final[0], nk = s_final[1];
 
   // ---- the prefix tree of the kept sequences ----
   int32_t* tok = P.node_token + static_cast<size_t>(b) * P.N;
@@ -392,13 +461,18 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const BuildPa
     s_rep[j - 1][m] = rep ? 1 : 0;
   }
   __syncthreads();
+  // nodes per depth, one warp per depth, then their offsets
+  for (int j = warp + 1; j <= D; j += kBuildThreads / 32) {
+    int c = 0;
+    for (int m = lane; m < nk; m += 32) c += s_rep[j - 1][m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+    if (lane == 0) s_cnt[j] = c;
+  }
+  __syncthreads();
   if (tid == 0) {
     s_off[1] = 1;
-    for (int j = 1; j <= D; ++j) {
-      int cnt = 0;
-      for (int m = 0; m < nk; ++m) cnt += s_rep[j - 1][m];
-      s_off[j + 1] = s_off[j] + cnt;
-    }
+    for (int j = 1; j <= D; ++j) s_off[j + 1] = s_off[j] + s_cnt[j];
     P.n_nodes[b] = s_off[D + 1];
   }
   __syncthreads();  // also orders the padding stores before the node stores
@@ -414,7 +488,7 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const BuildPa
     const unsigned long long t = k_tup[cur][m];
     const int id = node_id(j, prefix_of(t, j));
     const int s = static_cast<int>((t >> (4 * (kMaxDepth - j))) & 15ull);  // rank at position j-1
-    tok[id] = ids[(j - 1) * k + s];
+    tok[id] = s_ids[j - 1][s];
     par[id] = (j == 1) ? 0 : node_id(j - 1, prefix_of(t, j - 1));
     dep[id] = j;
   }
@@ -430,26 +504,50 @@ struct WalkParams {
   int32_t* acc;  // [B]
 };
 
+// One CTA per sequence: the tree (draws, tokens, parents) comes into shared
+// memory in one round trip, each node's children are located there (first
+// child and count), and one thread walks.
 __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(const WalkParams P) {
+  __shared__ int32_t s_draw[kMaxNodes], s_tok[kMaxNodes], s_par[kMaxNodes];
+  __shared__ int s_first[kMaxNodes], s_nchild[kMaxNodes];
   uno::launch_dependents();
   uno::grid_dependency_wait();
-  const int b = blockIdx.x * kWalkThreads + threadIdx.x;
-  if (b >= P.B) return;
+  const int b = blockIdx.x, tid = threadIdx.x;
   const size_t base = static_cast<size_t>(b) * P.N;
-  const int32_t* draw = P.draw + base;
-  const int32_t* tok = P.node_token + base;
-  const int32_t* par = P.node_parent + base;
   const int n = min(max(P.n_nodes[b], 1), P.N);
+  for (int c = tid; c < n; c += kWalkThreads) {
+    s_draw[c] = P.draw[base + c];
+    s_tok[c] = P.node_token[base + c];
+    s_par[c] = P.node_parent[base + c];
+    s_first[c] = INT_MAX;
+    s_nchild[c] = 0;
+  }
+  __syncthreads();
+  for (int c = 1 + tid; c < n; c += kWalkThreads) {
+    const int pa = s_par[c];
+    if (pa >= 0 && pa < c) {
+      atomicMin(&s_first[pa], c);
+      atomicAdd(&s_nchild[pa], 1);
+    }
+  }
+  __syncthreads();
+  if (tid != 0) return;
   int32_t* out = P.out + static_cast<size_t>(b) * (P.D + 1);
   int node = 0, acc = -1;
   for (int j = 0; j <= P.D; ++j) {
-    const int y = draw[node];
+    const int y = s_draw[node];
     if (y < 0) break;  // a row with no distribution on the walk: invalid
     out[j] = y;
     int child = -1;
-    if (j < P.D)
-      for (int c = node + 1; c < n && child < 0; ++c)
-        if (par[c] == node && tok[c] == y) child = c;
+    if (j < P.D) {
+      // the node's children in index order: the first with the drawn token
+      int left = s_nchild[node];
+      for (int c = s_first[node]; left > 0 && c < n && child < 0; ++c) {
+        if (s_par[c] != node) continue;
+        --left;
+        if (s_tok[c] == y) child = c;
+      }
+    }
     if (child < 0) {
       acc = j;
       break;
@@ -471,6 +569,22 @@ bool tree_sizes_ok(int B, int D, int V, int top_k, int budget) {
   if (top_k < 1 || top_k > kMaxTopK || budget < 1 || budget > kMaxBudget) return false;
   const long long N = 1 + static_cast<long long>(D) * budget;
   return static_cast<long long>(B) * D <= (1 << 28) && static_cast<long long>(B) * N <= (1 << 28);
+}
+
+template <typename Kern, typename Params, typename Params2>
+int launch_pdl2(Kern kern, dim3 grid, dim3 block, const Params& p, const Params2& p2,
+                cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p, p2) != cudaSuccess) return UNO_ERR_CUDA;
+  return (cudaGetLastError() == cudaSuccess) ? UNO_OK : UNO_ERR_CUDA;
 }
 
 template <typename Kern, typename Params>
@@ -519,21 +633,23 @@ TopkPlan topk_plan(long long rows, int V, int top_k) {
   return pl;
 }
 
+// The two drafting launches: the slabs' top-k lists, then per sequence the
+// merge of its rows and the tree.
 template <typename T, int KM>
-int launch_topk_km(const TopkParams& tp, cudaStream_t st) {
+int launch_draft_km(const TopkParams& tp, const BuildParams& bp, cudaStream_t st) {
   const int rc = launch_pdl(tree_topk_part_kernel<T, KM>,
                             dim3(static_cast<unsigned>(tp.rows * tp.slabs)), dim3(kTopThreads),
                             tp, st);
   if (rc != UNO_OK) return rc;
-  return launch_pdl(tree_topk_merge_kernel<KM>, dim3(static_cast<unsigned>(tp.rows)), dim3(32),
-                    tp, st);
+  return launch_pdl2(tree_build_kernel<KM>, dim3(static_cast<unsigned>(bp.B)),
+                     dim3(kBuildThreads), tp, bp, st);
 }
 
 template <typename T>
-int launch_topk(const TopkParams& tp, cudaStream_t st) {
-  if (tp.top_k <= 4) return launch_topk_km<T, 4>(tp, st);
-  if (tp.top_k <= 8) return launch_topk_km<T, 8>(tp, st);
-  return launch_topk_km<T, 16>(tp, st);
+int launch_draft(const TopkParams& tp, const BuildParams& bp, cudaStream_t st) {
+  if (tp.top_k <= 4) return launch_draft_km<T, 4>(tp, bp, st);
+  if (tp.top_k <= 8) return launch_draft_km<T, 8>(tp, bp, st);
+  return launch_draft_km<T, 16>(tp, bp, st);
 }
 
 }  // namespace
@@ -585,12 +701,10 @@ extern "C" int uno_tree_draft(const void* q_logits, int B, int D, int V, int dty
   tp.part_s = reinterpret_cast<float*>(ws + pl.s_off);
   tp.ids = topk_ids;
   tp.logq = topk_logq;
-  const int rc = (dtype == UNO_BF16) ? launch_topk<uint16_t>(tp, st) : launch_topk<float>(tp, st);
-  if (rc != UNO_OK) return rc;
-  BuildParams bp{topk_ids, topk_logq, B, D, top_k, budget, 1 + D * budget,
-                 node_token, node_parent, node_depth, n_nodes};
-  return launch_pdl(tree_build_kernel, dim3(static_cast<unsigned>(B)), dim3(kBuildThreads), bp,
-                    st);
+  BuildParams bp{B, D, top_k, budget, 1 + D * budget, node_token, node_parent, node_depth,
+                 n_nodes};
+  return (dtype == UNO_BF16) ? launch_draft<uint16_t>(tp, bp, st)
+                             : launch_draft<float>(tp, bp, st);
 }
 
 extern "C" int uno_tree_verify(const void* p_logits, const int32_t* node_token,
@@ -629,7 +743,5 @@ extern "C" int uno_tree_verify(const void* p_logits, const int32_t* node_token,
   int rc = uno_host::sample_rows(r, st);
   if (rc != UNO_OK) return rc;
   WalkParams wp{node_draw, node_token, node_parent, n_nodes, B, D, N, out_tokens, accepted_len};
-  return launch_pdl(tree_walk_kernel, dim3(static_cast<unsigned>((B + kWalkThreads - 1) /
-                                                                 kWalkThreads)),
-                    dim3(kWalkThreads), wp, st);
+  return launch_pdl(tree_walk_kernel, dim3(static_cast<unsigned>(B)), dim3(kWalkThreads), wp, st);
 }
