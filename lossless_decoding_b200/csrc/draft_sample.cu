@@ -14,11 +14,12 @@
 // vectors per lane, so the warp reduction is paid once per several vectors)
 // and streams them in rounds of kRound 16-byte vectors per lane through a
 // ring of kStages shared-memory stages (cp.async): kStages - 1 rounds are in
-// flight while one is folded into a per-lane (reference, sum of
-// 2^(x - reference)) in the log2 domain with packed float32x2 arithmetic. The
-// warp reduces each chunk to one such pair in the leading CTA's shared memory
+// flight while one is folded into a per-lane (running maximum, sum of
+// 2^(x - maximum)) in the log2 domain with packed float32x2 arithmetic. The
+// warp reduces each chunk to one such pair (the lanes' sums rescaled to the
+// warp's maximum and added in float64) in the leading CTA's shared memory
 // (distributed shared memory), and the others leave after a cluster barrier.
-// The leader then rescales the chunk sums to the largest reference, takes
+// The leader then rescales the chunk sums to the largest maximum, takes
 // their float64 running sum, finds the chunk where u * total is crossed and
 // scans only that chunk (in L2 by then): each thread sums a contiguous
 // segment, one block scan places the segments, and the thread whose segment
@@ -79,8 +80,8 @@ struct SampleParams {
 };
 
 // Dynamic shared memory: the warps' copy rings (kStages rounds each), then the
-// chunk table: cm[nchunks] (the chunk's reference in the log2 domain, -inf
-// when empty) and cs[nchunks] (sum over the chunk of 2^(x log2 e - cm)).
+// chunk table: cs[nchunks] (float64: sum over the chunk of 2^(x log2 e - cm))
+// and cm[nchunks] (the chunk's maximum times log2 e, -inf when empty).
 template <int kWarps>
 constexpr int ring_bytes() {
   return kWarps * kStages * kRound * 32 * 16;
@@ -151,8 +152,8 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
                  (static_cast<size_t>(seq) * P.seq_rows + (bi - seq * P.rows)) * P.V;
   const int V = P.V, L = P.chunk_len;
   uint4* ring = dyn + warp * (kStages * kRound * 32);
-  float* cm = reinterpret_cast<float*>(dyn + kWarps * kStages * kRound * 32);
-  float* cs = cm + P.nchunks;
+  double* cs = reinterpret_cast<double*>(dyn + kWarps * kStages * kRound * 32);
+  float* cm = reinterpret_cast<float*>(cs + P.nchunks);
 
   // ---- pass 1: per-chunk (reference, sum of 2^(x - reference)) ----
   // Warp w of the cluster (gw = rank * kWarps + w) takes chunks gw, gw + nw,
@@ -203,23 +204,32 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
     const int vb = c * cvec + r * (32 * kRound) + lane;
     if (vb + (kRound - 1) * 32 < nvec) {  // every vector of the round is whole
 #pragma unroll
-      for (int j = 0; j < kRound; j += 2) uno::fold_vecs<T, 2>(lm, ls, cur + j);
+      for (int j = 0; j < kRound; j += 2) uno::fold_vecs_max<T, 2>(lm, ls, cur + j);
     } else {
 #pragma unroll
       for (int j = 0; j < kRound; ++j)
-        if (vb + j * 32 < nvec) uno::fold_vecs<T, 1>(lm, ls, cur + j);
+        if (vb + j * 32 < nvec) uno::fold_vecs_max<T, 1>(lm, ls, cur + j);
     }
     if (++r == rpc) {  // the chunk is complete
       // its elements outside whole vectors, one by one
       const int e0 = max(c * L, nvec * kVec), e1 = min((c + 1) * L, V);
       for (int e = e0 + lane; e < e1; e += 32) {
-        const float f = uno::LogitRow<T>::at(row, e);
-        uno::fold<1>(lm, ls, &f);
+        uno::fold_one_max(lm, ls, uno::LogitRow<T>::at(row, e));
       }
-      uno::warp_merge(lm, ls);
+      // the warp's pair: the largest reference, each lane's sum rescaled to
+      // it once, in float64 (32 exact-ish exponentials per chunk)
+      float mm = lm;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, o));
+      double zd = (lm > -INFINITY)
+                      ? static_cast<double>(ls) *
+                            exp2(static_cast<double>(lm) - static_cast<double>(mm))
+                      : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zd += __shfl_xor_sync(0xFFFFFFFFu, zd, o);
       if (lane == 0) {  // into the leader's table
-        *cluster.map_shared_rank(cm + c, 0) = lm;
-        *cluster.map_shared_rank(cs + c, 0) = (lm > -INFINITY) ? ls : 0.f;
+        *cluster.map_shared_rank(cm + c, 0) = mm;
+        *cluster.map_shared_rank(cs + c, 0) = (mm > -INFINITY) ? zd : 0.0;
       }
       lm = -INFINITY;
       ls = 0.f;
@@ -259,9 +269,9 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
   double mine = 0.0;
   int last_pos_chunk = -1;
   for (int c = c_lo; c < c_hi; ++c) {
-    const double w = (cm[c] > -INFINITY) ? static_cast<double>(cs[c]) *
-                                                  static_cast<double>(uno::ex2(cm[c] - M))
-                                            : 0.0;
+    const double w = (cm[c] > -INFINITY)
+                         ? cs[c] * exp2(static_cast<double>(cm[c]) - static_cast<double>(M))
+                         : 0.0;
     mine += w;
     if (w > 0.0) last_pos_chunk = c;
   }
@@ -272,9 +282,9 @@ __global__ void __launch_bounds__(S::kThreads, S::kCtasPerSm)
     double run = before;
     int found = -1;
     for (int c = c_lo; c < c_hi && found < 0; ++c) {
-      const double w = (cm[c] > -INFINITY) ? static_cast<double>(cs[c]) *
-                                                    static_cast<double>(uno::ex2(cm[c] - M))
-                                              : 0.0;
+      const double w = (cm[c] > -INFINITY)
+                           ? cs[c] * exp2(static_cast<double>(cm[c]) - static_cast<double>(M))
+                           : 0.0;
       if (run + w > t) found = c;
       else run += w;
     }
@@ -373,7 +383,8 @@ int run(const uno_host::RowDraws& r, cudaStream_t st) {
   P.chunk_len = static_cast<int>(per_chunk * kStep);
   P.nchunks = static_cast<int>((V + P.chunk_len - 1) / P.chunk_len);
   cudaLaunchConfig_t cfg = {};
-  const int smem = ring_bytes<S::kWarps>() + 2 * P.nchunks * static_cast<int>(sizeof(float));
+  const int smem = ring_bytes<S::kWarps>() +
+                   P.nchunks * static_cast<int>(sizeof(double) + sizeof(float));
   if (!allow_smem<T, S>(smem)) return UNO_ERR_CUDA;
   cfg.gridDim = dim3(static_cast<unsigned>(r.B * r.rows_per_seq * S::kCluster));
   cfg.blockDim = dim3(S::kThreads);

@@ -128,6 +128,70 @@ __device__ __forceinline__ void fold_vecs(float& m, float& z, const uint4* v) {
   z += sum(m);
 }
 
+// The same fold with m kept at the running maximum (times log2 e) instead of a
+// lazy reference: the group's maximum is taken first and m moves up to it
+// before the sum, so every exponent argument is <= 0. Costs one more max per
+// value; in return a weight's error from its argument's rounding is at most
+// about 2^-24 ln 2 |argument| 2^argument of the maximum's weight, which keeps
+// a sampler's chunk sums (not only their ratios) accurate to a few float32
+// roundings.
+template <typename T, int NV>
+__device__ __forceinline__ void fold_vecs_max(float& m, float& z, const uint4* v) {
+  constexpr bool kBf16 = sizeof(T) == 2;
+  constexpr int kP = (kBf16 ? 4 : 2) * NV;  // float pairs
+  uint64_t x[kP];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+    if constexpr (kBf16) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        x[4 * k + i] = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        x[2 * k + i] = pack2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+    }
+  }
+  float gm = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kP; ++i) {
+    const float2 p = unpack2(x[i]);
+    gm = fmaxf(gm, fmaxf(p.x, p.y));
+  }
+  if (gm == -INFINITY) return;  // nothing finite in the group
+  gm *= kLog2e;
+  if (gm > m) {
+    z = (m == -INFINITY) ? 0.f : z * ex2(m - gm);
+    m = gm;
+  }
+  const uint64_t l2e = pack2(kLog2e, kLog2e), nref = pack2(-m, -m);
+  uint64_t e[kP];
+#pragma unroll
+  for (int i = 0; i < kP; ++i) {
+    const float2 a = unpack2(fma2(x[i], l2e, nref));
+    e[i] = pack2(ex2(a.x), ex2(a.y));
+  }
+#pragma unroll
+  for (int w = 1; w < kP; w *= 2) {
+#pragma unroll
+    for (int i = 0; i + w < kP; i += 2 * w) e[i] = add2(e[i], e[i + w]);
+  }
+  const float2 s = unpack2(e[0]);
+  z += s.x + s.y;
+}
+
+// One value, m kept at the running maximum (times log2 e).
+__device__ __forceinline__ void fold_one_max(float& m, float& z, float x) {
+  if (!(x > -INFINITY)) return;
+  const float g = x * kLog2e;
+  if (g > m) {
+    z = (m == -INFINITY) ? 0.f : z * ex2(m - g);
+    m = g;
+  }
+  z += ex2(fmaf(x, kLog2e, -m));
+}
+
 template <typename T>
 __device__ __forceinline__ void fold_pair(float& m, float& z, const uint4* v) {
   fold_vecs<T, 2>(m, z, v);

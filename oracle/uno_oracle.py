@@ -401,8 +401,13 @@ def sample_drafts_u(q_logits, u):
     w = np.where(np.isfinite(rows), np.exp(rows - m[:, None]), 0.0)
     idx, c_prev, c_at, t, total = _inverse_cdf(w, np.asarray(u, dtype=np.float64).reshape(-1))
     idx = np.where(finite, idx, -1).astype(np.int32)
+    # sqrt(sum of squared weights): the scale at which uncorrelated per-token
+    # relative errors of a float32 implementation move the CDF (diagnostic,
+    # for near-tie accounting only)
+    spread = np.sqrt(np.sum(w * w, axis=1))
     details = {"c_prev": c_prev.reshape(B, K), "c_at": c_at.reshape(B, K),
-               "threshold": t.reshape(B, K), "total": total.reshape(B, K)}
+               "threshold": t.reshape(B, K), "total": total.reshape(B, K),
+               "spread": spread.reshape(B, K)}
     return idx.reshape(B, K), details
 
 

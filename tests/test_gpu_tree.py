@@ -18,7 +18,7 @@ import torch
 
 import oracle
 from lossless_decoding_b200.inputs import verify_inputs
-from tests.parity import TAU_ABS, TAU_REL, widen
+from tests.parity import TAU_DRAFT, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -156,7 +156,7 @@ def _check_walk(api, ref, p, seed, step, D, budget):
             j = int(ref["node_depth"][b, c])
             ids, det = oracle.sample_drafts_u(pw[b, c][None, None], u[b, j][None, None])
             tie = (min(det["threshold"] - det["c_prev"], det["c_at"] - det["threshold"])
-                   < TAU_ABS + TAU_REL * det["total"]).item() and ids[0, 0] >= 0
+                   < TAU_DRAFT * det["spread"]).item() and ids[0, 0] >= 0
             ties_at[b, c] = tie
             if not tie:
                 assert draw[b, c] == ids[0, 0], (b, c, draw[b, c], ids[0, 0])
