@@ -296,11 +296,31 @@ class BatchedDecode:
         nbytes = self.v.q_logits.numel() * self.v.q_logits.element_size() + ids.numel() * 4
         gbs = nbytes / (us / 1e6) / 1e9
         peak = _peaks()["hbm"]
+        # the verifier's calls back to back on the step's inputs: as in the
+        # step, each call's stream launch sets up during the previous kernel
+        # (the per-launch breakdown puts events between launches, which
+        # serialises that set-up)
+        for i in range(3):
+            self.api.verify_block(self.v.p_logits, self.v.q_logits, self.v.draft_tokens,
+                                  seed=self.philox_seed, step=i, out=self.out, workspace=self.vws)
+        a.record(stream)
+        for i in range(reps):
+            self.api.verify_block(self.v.p_logits, self.v.q_logits, self.v.draft_tokens,
+                                  seed=self.philox_seed, step=100 + i, out=self.out,
+                                  workspace=self.vws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        us_v = a.elapsed_time(b) * 1e3 / reps
+        gbs_v = self.verify_bytes / (us_v / 1e6) / 1e9
         return {"draft_sampler": {"kernel": "sample_drafts_kernel", "us": us, "achieved": gbs,
                                   "unit": "GB/s", "peak": peak, "frac": gbs / peak,
                                   "algorithmic_bytes": nbytes,
                                   "traffic": measured_traffic(self.name, "draft"),
-                                  "rows": f"{self.B}x{self.K} rows of {self.V}"}}
+                                  "rows": f"{self.B}x{self.K} rows of {self.V}"},
+                "verifier_back_to_back": {"kernels": "verify_stream_kernel + verify_draw_kernel",
+                                          "us": us_v, "achieved": gbs_v, "unit": "GB/s",
+                                          "peak": peak, "frac": gbs_v / peak,
+                                          "calls": reps, "algorithmic_bytes": self.verify_bytes}}
 
     def make_events(self):
         n = len(self.layers)
