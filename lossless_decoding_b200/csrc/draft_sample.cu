@@ -43,7 +43,7 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kMaxChunks = 2048;  // chunk table entries (shared memory, 8 bytes each)
-constexpr int kMinSteps = 16;     // vectors per lane in a chunk, at least
+constexpr int kMinSteps = 8;      // vectors per lane in a chunk, at least (2 rounds)
 
 // Launch shapes. Many rows (a 64 x 16 block of drafts): two 128-thread CTAs
 // per row, 8 per SM, in about two waves that the hardware balances over the

@@ -7,7 +7,7 @@ replays, in numpy float32, the roundings the device's sampler makes on rows
 shaped like the full-vocabulary test workloads, with the SFU's 2^(.) error
 injected at its measured largest relative size (1.46e-7):
 
-  * pass 1, per chunk (4096 bfloat16 or 2048 float32 logits) and per lane:
+  * pass 1, per chunk (2048 bfloat16 or 1024 float32 logits) and per lane:
     the reference m kept at the running maximum (each group of two vectors
     moves it up to its own maximum first, rescaling the sum by an SFU
     2^(m - gm)), the exponent argument x log2 e - m by one fused multiply-add,
@@ -35,7 +35,7 @@ from tests.parity import TAU_DRAFT, widen
 F32 = np.float32
 LOG2E = F32(1.4426950408889634)
 SFU_REL = 1.46e-7
-LANES, ROUNDS, KV = 32, 4, 4   # a chunk: ROUNDS rounds of KV 16-byte vectors per lane
+LANES, ROUNDS, KV = 32, 2, 4   # a chunk: ROUNDS rounds of KV 16-byte vectors per lane
 
 
 def _sfu(a, rng):
