@@ -240,20 +240,24 @@ int uno_dualpath_linear_gated(const void* x, const void* W, const void* A, const
  * Framework": drafting uses theta_AR + theta_Delta, verification theta_AR
  * alone). uno_dualpath_linear_stats is uno_dualpath_linear_gated (same
  * arguments, same outputs bit for bit) that also writes, for every output
- * row and every 256-column tile, the softmax partial of the values it
- * stored: m = max(value) * log2(e) and z = sum of 2^(value * log2(e) - m)
- * (float pairs). uno_verify_block_head then verifies without reading every
+ * row, the softmax partials of the values it stored, each over a part of the
+ * row: m = max(value) * log2(e) and z = sum of 2^(value * log2(e) - m)
+ * (float pairs; a part with no values is (-inf, 0)). uno_verify_block_head then verifies without reading every
  * logit again: it merges those partials instead of streaming the rows and
  * reads only the logits at the drafted ids and the one p (and q) row that
  * the final draw needs per sequence.
  *
- * uno_dualpath_stats_tiles(M, d_out) = ceil(d_out / 256) when M > 256 (the
- *   statistics come from the CTA-pair layout), else 0.
+ * uno_dualpath_stats_tiles(M, d_out) = T, the partials per row: for M > 256
+ *   (CTA pairs, one per 256-column tile) ceil(d_out / 256), the partial of
+ *   tile t covering columns [256 t, 256 t + 256); for 1 <= M <= 256 (swapped
+ *   operands, one partial per CTA, which accumulates over every column tile
+ *   it computes) 148, slots of CTAs the launch does not start holding
+ *   (-inf, 0); 0 when M < 1 or d_out < 1.
  * uno_dualpath_linear_stats: as uno_dualpath_linear_gated, plus
  *   stats_ar     [M, T, 2] f32 out (T = uno_dualpath_stats_tiles), or null;
  *                needs y_ar
  *   stats_draft  [M, T, 2] f32 out, or null; needs y_draft
- *   M must exceed 256 (UNO_ERR_SIZE otherwise).
+ *   A row's logsumexp is the merge of its T partials, whatever the layout.
  * uno_verify_block_head: as uno_verify_block, with
  *   y_ar         [B, K+1, V] dtype: p, row i of sequence b = LM-head row
  *                b * (K+1) + i

@@ -228,8 +228,9 @@ def dualpath_linear(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm: torch
 
 
 def dualpath_stats_tiles(M: int, d_out: int) -> int:
-    """Column tiles of the row statistics of ``dualpath_linear_stats`` (0 when
-    M <= 256: not available)."""
+    """Softmax partials per row written by ``dualpath_linear_stats``: one per
+    256-column tile when M > 256, one per CTA (148) when M <= 256, 0 for an
+    empty problem."""
     return int(lib.uno_dualpath_stats_tiles(M, d_out))
 
 
@@ -241,9 +242,10 @@ def dualpath_linear_stats(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm:
                           stats_draft: Optional[torch.Tensor] = None,
                           workspace: Optional[torch.Tensor] = None):
     """The LM head: ``dualpath_linear`` (both outputs) that also writes each
-    output row's softmax partials per 256-column tile, float32 [M, T, 2] as
-    (max * log2 e, sum of 2^(x log2 e - that)). M must exceed 256. Returns
-    (y_ar, y_draft, stats_ar, stats_draft)."""
+    output row's softmax partials, float32 [M, T, 2] as (max * log2 e, sum
+    of 2^(x log2 e - that)), each over a part of the row (T =
+    ``dualpath_stats_tiles``; an empty part is (-inf, 0)). Returns (y_ar,
+    y_draft, stats_ar, stats_draft)."""
     if x.dim() != 2 or W.dim() != 2 or A.dim() != 2 or Bm.dim() != 2:
         raise ValueError("expected 2-D x, W, A, Bm")
     M, d_in = x.shape
@@ -255,7 +257,7 @@ def dualpath_linear_stats(x: torch.Tensor, W: torch.Tensor, A: torch.Tensor, Bm:
         raise TypeError("x, W, A and Bm must share a dtype")
     T = dualpath_stats_tiles(M, d_out)
     if T == 0:
-        raise ValueError("row statistics need M > 256")
+        raise ValueError("row statistics need M >= 1 and d_out >= 1")
     dt = _dtype_code(x)
     dev = _check_cuda(x, W, A, Bm)
     if y_ar is None:

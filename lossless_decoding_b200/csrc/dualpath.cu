@@ -170,10 +170,18 @@ __host__ __device__ constexpr int barrier_bytes() {
   return (2 * stages_for<BN, PAIR>() + 8 + 1 + 2) * 8 + 4 + 4;
 }
 
+// One CTA's running row statistics in the swapped layout: per epilogue warp,
+// y_ar and y_draft, BN rows of (m, z).
+template <int BN, bool PAIR>
+__host__ __device__ constexpr int swap_stat_bytes() {
+  return PAIR ? 0 : 4 * 2 * BN * 8;
+}
+
 template <int BN, bool PAIR>
 __host__ __device__ constexpr int smem_bytes() {
   static_assert(barrier_bytes<BN, PAIR>() <= 256, "barrier region");
-  return stages_for<BN, PAIR>() * stage_bytes<BN, PAIR>() + 1024 /*align*/ + 256 /*barriers*/;
+  return stages_for<BN, PAIR>() * stage_bytes<BN, PAIR>() + 1024 /*align*/ + 256 /*barriers*/ +
+         swap_stat_bytes<BN, PAIR>();
 }
 
 __device__ __forceinline__ void set_fault(unsigned bit, volatile int* abort_flag) {
@@ -432,6 +440,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* mma_done = t_stored + 1;        // [2] every MMA of issuer e has completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
   int* order = reinterpret_cast<int*>(tmem_holder + 1);  // next ring item to issue
+  // swapped layout with row statistics: [4 epilogue warps][2 outputs][BN] (m, z)
+  float2* srs = reinterpret_cast<float2*>(smem + STAGES * kStage + 256);
+  const bool swap_stats = SWAP && (p.g[0].stats_ar != nullptr || p.g[0].stats_draft != nullptr);
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -842,6 +853,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       else sm100::mbar_arrive(bar);
     };
     const int rr = quarter * 32 + lane;
+    // Swapped layout: one lane holds one output column for 32 rows. The
+    // statistics of this warp's 32 columns for rows cbase..cbase+31 (sv[e] =
+    // the stored value of row cbase + e, -inf where there is none) are reduced
+    // across the lanes by recursive halving: at offset h a lane keeps the half
+    // of its rows selected by bit h of its lane index and merges the partner's
+    // pairs for them, so after offsets 16..1 lane l holds row cbase + l (31
+    // merges, 62 shuffles). It is then merged into the CTA's running pair for
+    // that row (this warp's own slot). Pairs (m, z) are in the log2 domain as
+    // everywhere: m = max value times log2 e, z = sum of 2^(v log2 e - m).
+    // The pair with the larger reference keeps its sum; only the other one's
+    // is rescaled (one 2^x per merge; 2^-inf = 0 covers an empty pair, and
+    // two empty pairs stay (-inf, 0)).
+    auto merge_mz = [](float& m, float& z, float m2, float z2) {
+      const bool first = m >= m2;
+      const float hi = first ? m : m2, lo = first ? m2 : m;
+      const float zhi = first ? z : z2, zlo = first ? z2 : z;
+      z = fmaf(zlo, uno::ex2(lo == -INFINITY ? -INFINITY : lo - hi), zhi);
+      m = hi;
+    };
+    auto swap_row_stats = [&](float* sv, int out, int cbase) {
+      constexpr float kL2e = 1.4426950408889634f;
+      const bool b16 = (lane & 16) != 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {  // single values: (v log2 e, 1)
+        const float keep = b16 ? sv[i + 16] : sv[i];
+        const float send = b16 ? sv[i] : sv[i + 16];
+        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+        float m = keep * kL2e, z = (keep > -INFINITY) ? 1.f : 0.f;
+        merge_mz(m, z, recv * kL2e, (recv > -INFINITY) ? 1.f : 0.f);
+        sv[i] = m;
+        sv[16 + i] = z;
+      }
+#pragma unroll
+      for (int h = 8; h >= 1; h >>= 1) {  // pairs (sv[i], sv[16 + i]), i < 2h
+        const bool bit = (lane & h) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+          float m = bit ? sv[i + h] : sv[i];
+          float z = bit ? sv[16 + i + h] : sv[16 + i];
+          const float sm = bit ? sv[i] : sv[i + h];
+          const float sz = bit ? sv[16 + i] : sv[16 + i + h];
+          const float rm = __shfl_xor_sync(0xFFFFFFFFu, sm, h);
+          const float rz = __shfl_xor_sync(0xFFFFFFFFu, sz, h);
+          merge_mz(m, z, rm, rz);
+          sv[i] = m;
+          sv[16 + i] = z;
+        }
+      }
+      float2* slot = srs + (quarter * 2 + out) * BN + cbase + lane;
+      float2 a = *slot;
+      merge_mz(a.x, a.y, sv[0], sv[16]);
+      *slot = a;
+    };
+    if (swap_stats)
+      for (int q = 0; q < 2 * BN; q += 32)
+        srs[quarter * 2 * BN + q + lane] = make_float2(-INFINITY, 0.f);
     // outputs of the projection of the tile being drained
     T* ya = nullptr;
     T* yd = nullptr;
@@ -852,7 +919,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // unswapped, the B rows swapped); a closed row stores T = 0.
     auto drain = [&](uint32_t acc, int a0, int b0, T* y, int ld, int nrows, int ncol,
                      float mul, const uint8_t* gate = nullptr, float2* stats = nullptr,
-                     int stats_tiles = 0) {
+                     int stats_tiles = 0, int stat_out = 0) {
       if (!y) return;
       const uint32_t tq = acc + (static_cast<uint32_t>(quarter * 32) << 16);
       const int arow = a0 + rr;
@@ -893,6 +960,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (brow + e < nrows)
                 store_one<T>(y + static_cast<size_t>(brow + e) * ld + arow, f[e]);
+          }
+          if (stats) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              f[e] = (arow < ld && brow + e < nrows) ? stored_value<T>(f[e]) : -INFINITY;
+            swap_row_stats(f, stat_out, c);
           }
         }
       }
@@ -1020,6 +1093,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int e = 0; e < 32; ++e)
                 if (brow + e < p.M) store_one<T>(y + static_cast<size_t>(brow + e) * ncols + arow, f[e]);
+            }
+            if (st2[pass]) {
+              float sv[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                sv[e] = (arow < ncols && brow + e < p.M) ? stored_value<T>(f[e]) : -INFINITY;
+              swap_row_stats(sv, pass, c);
             }
           }
         }
@@ -1164,7 +1244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       drain(acc, x.a0 + my_rows, x.b0, ya, ncols, p.M, BN, 1.f, nullptr, p.g[gi].stats_ar,
-            p.g[gi].stats_tiles);
+            p.g[gi].stats_tiles, 0);
       sm100::tc_fence_before();
       __syncwarp();
       const int mo = li - nt_mine;
@@ -1177,10 +1257,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       sm100::tc_fence_after();
       drain(acc, x.a0 + my_rows, x.b0, yd, ncols, p.M, BN, 1.f, nullptr, p.g[gi].stats_draft,
-            p.g[gi].stats_tiles);
+            p.g[gi].stats_tiles, 1);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(&acc_empty[buf]);
+    }
+    if (swap_stats) {
+      // this CTA's pair per row: the four warps' pairs merged, written to its
+      // slot (slot = CTA index; CTA 0 marks the slots of absent CTAs empty)
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+      if (quarter == 0) {
+        const int T_ = p.g[0].stats_tiles;
+        for (int out = 0; out < 2; ++out) {
+          float2* st = out ? p.g[0].stats_draft : p.g[0].stats_ar;
+          if (!st) continue;
+          for (int cb = 0; cb < BN; cb += 32) {
+            const int row = cb + lane;
+            float m = -INFINITY, z = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float2 v = srs[(w * 2 + out) * BN + row];
+              merge_mz(m, z, v.x, v.y);
+            }
+            if (row < p.M && static_cast<int>(blockIdx.x) < T_)
+              st[static_cast<size_t>(row) * T_ + blockIdx.x] = make_float2(m, z);
+          }
+          if (blockIdx.x == 0)
+            for (int sl = static_cast<int>(gridDim.x); sl < T_; ++sl)
+              for (int row = lane; row < p.M; row += 32)
+                st[static_cast<size_t>(row) * T_ + sl] = make_float2(-INFINITY, 0.f);
+        }
+      }
     }
   }
 
@@ -1327,7 +1434,12 @@ int launch_dual(const DualMaps& maps, const GemmParams& p, cudaStream_t st) {
     attr_done.fetch_or(bit, std::memory_order_relaxed);
   }
   const long long units0 = static_cast<long long>(p.nT) * p.ngroups + p.main_tiles;
-  const long long resident = PAIR ? max_pairs(kern, bytes) : sm_count();
+  long long resident = PAIR ? max_pairs(kern, bytes) : sm_count();
+  // the swapped layout's row statistics have one slot per CTA: the launch
+  // (and the split plan below, which assumes every CTA is resident) uses at
+  // most that many CTAs
+  if (SWAP && (p.g[0].stats_ar || p.g[0].stats_draft) && resident > p.g[0].stats_tiles)
+    resident = p.g[0].stats_tiles;
   // Split the last, partial round of main tiles along K over the CTAs (or
   // pairs) it would leave idle: 3 or 4 pieces, each of at least 2 K-blocks.
   // (Two pieces do not pay for the hand-off of the fp32 partial: measured on
@@ -1476,7 +1588,9 @@ int run_dualpath(int n, const void* x, const void* const* W, const void* const* 
     a.y_draft = y_draft[g];
     a.stats_ar = stats_ar ? reinterpret_cast<float2*>(stats_ar[g]) : nullptr;
     a.stats_draft = stats_draft ? reinterpret_cast<float2*>(stats_draft[g]) : nullptr;
-    a.stats_tiles = (d_out[g] + 255) / 256;
+    // row statistics: one pair per 256-column tile (CTA pairs), or per CTA
+    // (swapped layout: each CTA accumulates over all of its tiles)
+    a.stats_tiles = pl.swap ? kSizingSms : (d_out[g] + 255) / 256;
     a.t_buf = ws;
     a.t_flags = reinterpret_cast<uint32_t*>(ws + pl.t_bytes);
     ws += pl.t_bytes + pl.flag_bytes;
@@ -1626,8 +1740,11 @@ extern "C" int uno_dualpath_linear_grouped(int n, const void* x, const void* con
 }
 
 extern "C" int uno_dualpath_stats_tiles(int M, int d_out) {
-  if (M <= 256 || d_out < 1) return 0;  // row statistics come from the CTA-pair layout
-  return (d_out + 255) / 256;
+  if (M < 1 || d_out < 1) return 0;
+  // CTA pairs (M > 256): one pair per 256-column tile; swapped layout: one
+  // per CTA of the launch (at most kSizingSms CTAs; absent ones write empty
+  // pairs)
+  return (M <= 256) ? kSizingSms : (d_out + 255) / 256;
 }
 
 extern "C" int uno_dualpath_linear_stats(const void* x, const void* W, const void* A,
@@ -1636,7 +1753,6 @@ extern "C" int uno_dualpath_linear_stats(const void* x, const void* W, const voi
                                          float* stats_draft, int M, int d_in, int d_out, int r,
                                          int dtype, void* workspace, size_t workspace_bytes,
                                          void* stream) {
-  if (M <= 256) return UNO_ERR_SIZE;
   if ((stats_ar && !y_ar) || (stats_draft && !y_draft)) return UNO_ERR_NULL;
   if (!uno_host::aligned(stats_ar, 8) || !uno_host::aligned(stats_draft, 8)) return UNO_ERR_ALIGN;
   return dispatch(1, x, &W, &A, &Bm, &scale, gate, &y_ar, &y_draft, M, d_in, &d_out, r, dtype,

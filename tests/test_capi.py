@@ -202,11 +202,12 @@ def test_head_argument_errors_need_no_gpu(lib):
     odd = ctypes.c_void_p(4096 + 4)
     u64 = ctypes.c_uint64
     assert lib.uno_dualpath_stats_tiles(1088, 151936) == 594
-    assert lib.uno_dualpath_stats_tiles(256, 151936) == 0
+    # swapped operands (M <= 256): one partial per CTA of the launch
+    assert lib.uno_dualpath_stats_tiles(256, 151936) == 148
+    assert lib.uno_dualpath_stats_tiles(17, 151936) == 148
+    assert lib.uno_dualpath_stats_tiles(0, 151936) == 0
+    assert lib.uno_dualpath_stats_tiles(17, 0) == 0
     st = lib.uno_dualpath_linear_stats
-    # statistics need the CTA-pair layout (M > 256)
-    assert STATUS[st(fake, fake, fake, fake, 2.0, None, fake, fake, fake, fake, 256, 4096, 4096,
-                     128, 0, fake, 1 << 30, None)] == "UNO_ERR_SIZE"
     # statistics of an output that is not written
     assert STATUS[st(fake, fake, fake, fake, 2.0, None, None, fake, fake, fake, 1088, 4096, 4096,
                      128, 0, fake, 1 << 30, None)] == "UNO_ERR_NULL"
@@ -252,6 +253,10 @@ def test_valid_calls_without_a_device_report_an_error(lib):
                                           32, 0, fake, need_d, None)] in bad
     assert STATUS[lib.uno_dualpath_linear_stats(fake, fake, fake, fake, 2.0, None, fake, fake,
                                                 fake, fake, 512, 256, 512, 32, 0, fake, need_d,
+                                                None)] in bad
+    need_s = lib.uno_dualpath_workspace_bytes(17, 256, 512, 32, 0)
+    assert STATUS[lib.uno_dualpath_linear_stats(fake, fake, fake, fake, 2.0, None, fake, fake,
+                                                fake, fake, 17, 256, 512, 32, 0, fake, need_s,
                                                 None)] in bad
     assert STATUS[lib.uno_sample_drafts(fake, 2, 4, 1000, 0, u64(0), u64(0), fake, None)] in bad
     assert STATUS[lib.uno_sample_drafts_blocks(fake, 2, 4, 5, 1000, 0, u64(0), u64(0), fake,

@@ -75,11 +75,38 @@ def test_stats_match_outputs(api, M, d_in, d_out, dtype):
         assert np.allclose(stn[..., 0], want_m, rtol=1e-6, atol=0)
 
 
-def test_stats_entry_refuses_small_batches(api):
-    d = _head(200, 256, 512, 32, "bf16", seed=3)
-    assert api.dualpath_stats_tiles(200, 512) == 0
-    with pytest.raises(ValueError):
-        api.dualpath_linear_stats(d.x, d.W, d.A, d.Bm, d.scale)
+@pytest.mark.parametrize("M,d_in,d_out,dtype", [
+    (17, 256, 1000, "bf16"),       # one block of 17 rows: BN = 32, ragged column tile
+    (200, 512, 3000, "f32"),       # BN = 256, the TF32 path
+    (68, 1024, 151936, "bf16"),    # four blocks over the full vocabulary: every CTA busy
+])
+def test_swapped_stats_match_outputs(api, M, d_in, d_out, dtype):
+    """Small batches (swapped operands): one partial per CTA, merged over the
+    CTA's column tiles; slots of CTAs the launch did not start are empty."""
+    d = _head(M, d_in, d_out, 64, dtype, seed=M + d_out)
+    gate = torch.ones(M, dtype=torch.uint8, device=DEV)
+    gate[::17] = 0
+    y_ar, y_dr, s_ar, s_dr = api.dualpath_linear_stats(d.x, d.W, d.A, d.Bm, d.scale, gate=gate)
+    ref_ar, ref_dr = api.dualpath_linear(d.x, d.W, d.A, d.Bm, d.scale, gate=gate)
+    torch.cuda.synchronize()
+    assert torch.equal(y_ar, ref_ar) and torch.equal(y_dr, ref_dr)
+    T = api.dualpath_stats_tiles(M, d_out)
+    assert T == 148 and tuple(s_ar.shape) == (M, T, 2)
+    for y, st in ((y_ar, s_ar), (y_dr, s_dr)):
+        yw = widen(y)
+        stn = st.cpu().numpy()
+        _, lse = oracle.softmax_rows(yw)
+        got = _lse_from_stats(stn)
+        assert np.abs(got - lse).max() < 2e-5 * max(1.0, np.abs(lse).max())
+        # every reference is the largest stored value of some of the row's
+        # columns (times log2 e); together they reach the row's maximum
+        m = stn[..., 0]
+        z = stn[..., 1]
+        empty = m == -np.inf
+        assert np.all(z[empty] == 0) and np.all(z[~empty] >= 1 - 1e-6)
+        want_top = (yw.max(axis=1) * LOG2E).astype(np.float32)
+        assert np.allclose(m.max(axis=1), want_top, rtol=1e-6, atol=0)
+    assert api.device_fault_flags() == 0
 
 
 def _check_head_verify(api, B, K, V, d_in, dtype, seed, step, n_check=None, sigma_w=0.05):
@@ -122,12 +149,25 @@ def _check_head_verify(api, B, K, V, d_in, dtype, seed, step, n_check=None, sigm
 @pytest.mark.parametrize("B,K,V,d_in,dtype", [
     (32, 8, 3000, 256, "bf16"),
     (20, 15, 5000, 512, "f32"),     # the TF32 path, V not a multiple of 256
+    (12, 8, 5000, 256, "f32"),      # 108 rows, swapped, TF32
 ])
 def test_verify_head_parity(api, B, K, V, d_in, dtype):
     for seed, step in ((5, 0), (41, 9)):
         rep = _check_head_verify(api, B, K, V, d_in, dtype, seed, step)
         report(f"LM head B={B} K={K} V={V} {dtype} seed={seed}", rep)
         assert rep.compared >= int(np.ceil(0.9 * B)) - 1
+
+
+def test_verify_head_single_sequence(api):
+    """One sequence (17 rows, swapped operands) over eight steps: at least
+    seven of the eight blocks compared token for token."""
+    tot = np.zeros(5, dtype=np.int64)
+    for step in range(8):
+        r = _check_head_verify(api, 1, 16, 20000, 512, "bf16", seed=11, step=step)
+        tot += np.array([r.rows, r.compared, r.accept_ties, r.draw_ties, r.invalid])
+    rep = VerifyReport(*[int(t) for t in tot])
+    report("LM head B=1 K=16 V=20000 bf16, 8 steps", rep)
+    assert rep.compared >= 7
 
 
 def test_verify_head_qwen3_lm_head(api):
