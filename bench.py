@@ -429,7 +429,7 @@ def tree_measure(api, stream, B, D, top_k, budget, V, reps=20, sets=4):
             "draft_us": us_d, "draft_gbs": bytes_d / (us_d / 1e6) / 1e9,
             "verify_us": us_v, "verify_gbs": bytes_v / (us_v / 1e6) / 1e9,
             "verify_rows_in_use": rows, "peak_gbs": peak,
-            "kernels": "tree_topk_part_kernel + tree_topk_merge_kernel + tree_build_kernel; "
+            "kernels": "tree_topk_part_kernel + tree_build_kernel (slab lists merged there); "
                        "sample_drafts_kernel (node rows) + tree_walk_kernel"}
 
 

@@ -357,7 +357,6 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
   __shared__ unsigned char s_rep[kMaxDepth][kMaxBudget];
   __shared__ int s_cnt[kMaxDepth + 1];
   __shared__ int s_off[kMaxDepth + 2];
-  __shared__ int s_final[2];  // buffer and size of the final kept set
   uno::launch_dependents();
   uno::grid_dependency_wait();
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -386,62 +385,61 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
     s_avail[tid] = a;
   }
   __syncthreads();
-  // The kept set, position by position, in warp 0 alone (the steps are
-  // short and dependent: warp-synchronous, no CTA barrier between them).
-  if (warp == 0) {
-    int cur = 0, nk = 1;
-    for (int j = 0; j < D; ++j) {
-      const int avail = s_avail[j];
-      // candidates (p, s) with (p + 1)(s + 1) <= budget: prefix p owns a run
-      // of min(avail, budget / (p + 1)) slots from s_coff[avail][p]
-      const int nc = s_coff[avail][nk];
-      const unsigned long long shift = 4ull * (kMaxDepth - 1 - j);
-      for (int p = lane; p < nk; p += 32) {
-        const int off = s_coff[avail][p];
-        const int cnt = s_coff[avail][p + 1] - off;
-        const float ps = k_score[cur][p];
-        const unsigned long long pt = k_tup[cur][p];
-        for (int s = 0; s < cnt; ++s) {
-          c_score[off + s] = ps + s_lq[j][s];
-          c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << shift);
+  // The kept set, position by position, by the whole CTA: per step the
+  // candidates are written (one thread per kept prefix), then ranked, a
+  // barrier after each. A candidate's rank (the candidates ahead of it) is
+  // counted by kRankLanes threads, each comparing it with every kRankLanes-th
+  // candidate, and summed by shuffles within the group, so a step costs a few
+  // comparisons per thread instead of one pass over all candidates.
+  constexpr int kRankLanes = 8;
+  constexpr int kRankGroups = kBuildThreads / kRankLanes;
+  const int sub = tid & (kRankLanes - 1);
+  int cur = 0, nk = 1;
+  for (int j = 0; j < D; ++j) {
+    const int avail = s_avail[j];
+    // candidates (p, s) with (p + 1)(s + 1) <= budget: prefix p owns a run
+    // of min(avail, budget / (p + 1)) slots from s_coff[avail][p]
+    const int nc = s_coff[avail][nk];
+    const unsigned long long shift = 4ull * (kMaxDepth - 1 - j);
+    for (int p = tid; p < nk; p += kBuildThreads) {
+      const int off = s_coff[avail][p];
+      const int cnt = s_coff[avail][p + 1] - off;
+      const float ps = k_score[cur][p];
+      const unsigned long long pt = k_tup[cur][p];
+      for (int s = 0; s < cnt; ++s) {
+        c_score[off + s] = ps + s_lq[j][s];
+        c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << shift);
+      }
+    }
+    __syncthreads();
+    const int nxt = cur ^ 1;
+    const int keep = min(budget, nc);
+    // every thread runs the same iterations (the shuffles need whole warps)
+    for (int base = 0; base < nc; base += kRankGroups) {
+      const int c = base + tid / kRankLanes;
+      const bool mine = c < nc;
+      int ahead = 0;
+      float sc = 0.f;
+      unsigned long long tu = 0ull;
+      if (mine) {
+        sc = c_score[c];
+        tu = c_tup[c];
+        for (int o = sub; o < nc; o += kRankLanes) {
+          const float so = c_score[o];
+          ahead += (so > sc || (so == sc && c_tup[o] < tu)) ? 1 : 0;
         }
       }
-      __syncwarp();
-      const int nxt = cur ^ 1;
-      const int keep = min(budget, nc);
-      // rank of candidate c = the candidates ahead of it (lane c mod 32)
-      for (int c = lane; c < nc; c += 32) {
-        const float sc = c_score[c];
-        const unsigned long long tu = c_tup[c];
-        int a0 = 0, a1 = 0;
-        int o = 0;
-        for (; o + 1 < nc; o += 2) {  // two independent comparisons per step
-          const float s0 = c_score[o], s1 = c_score[o + 1];
-          const unsigned long long t0 = c_tup[o], t1 = c_tup[o + 1];
-          a0 += (s0 > sc || (s0 == sc && t0 < tu)) ? 1 : 0;
-          a1 += (s1 > sc || (s1 == sc && t1 < tu)) ? 1 : 0;
-        }
-        if (o < nc) {
-          const float s0 = c_score[o];
-          a0 += (s0 > sc || (s0 == sc && c_tup[o] < tu)) ? 1 : 0;
-        }
-        const int rank = a0 + a1;
-        if (rank < keep) {
-          k_score[nxt][rank] = sc;
-          k_tup[nxt][rank] = tu;
-        }
+#pragma unroll
+      for (int w = kRankLanes / 2; w > 0; w >>= 1) ahead += __shfl_xor_sync(0xFFFFFFFFu, ahead, w);
+      if (mine && sub == 0 && ahead < keep) {
+        k_score[nxt][ahead] = sc;
+        k_tup[nxt][ahead] = tu;
       }
-      __syncwarp();
-      cur = nxt;
-      nk = keep;
     }
-    if (lane == 0) {
-      s_final[0] = cur;
-      s_final[1] = nk;
-    }
+    __syncthreads();
+    cur = nxt;
+    nk = keep;
   }
-  __syncthreads();
-  const int cur = s_final[0], nk = s_final[1];
 
   // ---- the prefix tree of the kept sequences ----
   int32_t* tok = P.node_token + static_cast<size_t>(b) * P.N;
