@@ -406,6 +406,7 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
       const int cnt = s_coff[avail][p + 1] - off;
       const float ps = k_score[cur][p];
       const unsigned long long pt = k_tup[cur][p];
+#pragma unroll 4
       for (int s = 0; s < cnt; ++s) {
         c_score[off + s] = ps + s_lq[j][s];
         c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << shift);
@@ -424,6 +425,7 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
       if (mine) {
         sc = c_score[c];
         tu = c_tup[c];
+#pragma unroll 4
         for (int o = sub; o < nc; o += kRankLanes) {
           const float so = c_score[o];
           ahead += (so > sc || (so == sc && c_tup[o] < tu)) ? 1 : 0;
