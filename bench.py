@@ -487,11 +487,43 @@ class SingleSequence(BatchedDecode):
             ev[3].record()
 
     def extra_measurements(self, stream, reps=20):
-        """The tree sampler at this workload's batch: a block of 16 (D = 15
-        positions after the AR-only first token), top-4 per position, the 16
-        best sequences kept (241 node rows)."""
-        return {"tree_sampler": tree_measure(self.api, stream, B=self.B, D=self.K - 1, top_k=4,
+        """The LM head alone at exactly 16 rows (the K draft positions) and at
+        the step's 17, timed over back-to-back calls (W, 1.24 GB, is larger
+        than L2); and the tree sampler at this workload's batch: a block of 16
+        (D = 15 positions after the AR-only first token), top-4 per position,
+        the 16 best sequences kept (241 node rows)."""
+        return {"lm_head_alone": self.lm_head_alone(stream, reps),
+                "tree_sampler": tree_measure(self.api, stream, B=self.B, D=self.K - 1, top_k=4,
                                              budget=16, V=self.V, reps=reps)}
+
+    def lm_head_alone(self, stream, reps):
+        api = self.api
+        _, _, (d,), (y_ar,), (y_dr,), ws = self.layers[0]
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        peak = _peaks()["hbm"]
+        out = {}
+        for rows in (16, self.M):
+            x, ya, yd = d.x[:rows], y_ar[:rows], y_dr[:rows]
+            need = api.dualpath_workspace_bytes(rows, QWEN3_8B_HIDDEN, self.V, RANK,
+                                                torch.bfloat16)
+            w = ws if ws.numel() >= need else torch.empty(need, dtype=torch.uint8,
+                                                           device=ws.device)
+            for _ in range(3):
+                api.dualpath_linear(x, d.W, d.A, d.Bm, d.scale, y_ar=ya, y_draft=yd, workspace=w)
+            a.record(stream)
+            for _ in range(reps):
+                api.dualpath_linear(x, d.W, d.A, d.Bm, d.scale, y_ar=ya, y_draft=yd, workspace=w)
+            b.record(stream)
+            torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / reps
+            nbytes = ((d.W.numel() + d.A.numel() + d.Bm.numel() + rows * QWEN3_8B_HIDDEN) * 2
+                      + 2 * rows * self.V * 2)
+            gbs = nbytes / (us / 1e6) / 1e9
+            out[f"rows_{rows}"] = {"us": us, "achieved": gbs, "unit": "GB/s", "peak": peak,
+                                   "frac": gbs / peak, "algorithmic_bytes": nbytes,
+                                   "calls": reps}
+        return out
 
     def host_inputs(self):
         _, x, *_ = self.layers[0]
