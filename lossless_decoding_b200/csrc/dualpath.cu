@@ -171,10 +171,11 @@ __host__ __device__ constexpr int barrier_bytes() {
 }
 
 // One CTA's running row statistics in the swapped layout: per epilogue warp,
-// y_ar and y_draft, BN rows of (m, z).
+// y_ar and y_draft, BN rows of (m, z); then per epilogue warp a 32 x 33 float
+// scratch for the transpose of a 32-row chunk.
 template <int BN, bool PAIR>
 __host__ __device__ constexpr int swap_stat_bytes() {
-  return PAIR ? 0 : 4 * 2 * BN * 8;
+  return PAIR ? 0 : 4 * 2 * BN * 8 + 4 * 32 * 33 * 4;  // + the warps' transpose scratch
 }
 
 template <int BN, bool PAIR>
@@ -183,6 +184,10 @@ __host__ __device__ constexpr int smem_bytes() {
   return stages_for<BN, PAIR>() * stage_bytes<BN, PAIR>() + 1024 /*align*/ + 256 /*barriers*/ +
          swap_stat_bytes<BN, PAIR>();
 }
+static_assert(smem_bytes<256, false>() <= 232448 && smem_bytes<128, false>() <= 232448 &&
+                  smem_bytes<64, false>() <= 232448 && smem_bytes<32, false>() <= 232448 &&
+                  smem_bytes<256, true>() <= 232448,
+              "dynamic shared memory per CTA (227 KB)");
 
 __device__ __forceinline__ void set_fault(unsigned bit, volatile int* abort_flag) {
   atomicOr(&g_fault_flags, bit);
@@ -855,11 +860,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int rr = quarter * 32 + lane;
     // Swapped layout: one lane holds one output column for 32 rows. The
     // statistics of this warp's 32 columns for rows cbase..cbase+31 (sv[e] =
-    // the stored value of row cbase + e, -inf where there is none) are reduced
-    // across the lanes by recursive halving: at offset h a lane keeps the half
-    // of its rows selected by bit h of its lane index and merges the partner's
-    // pairs for them, so after offsets 16..1 lane l holds row cbase + l (31
-    // merges, 62 shuffles). It is then merged into the CTA's running pair for
+    // the stored value of row cbase + e, -inf where there is none) go through
+    // the warp's 32 x 33 shared-memory scratch (the pad makes both the column
+    // writes and the row reads conflict-free), so that lane l holds row
+    // cbase + l's 32 values; it folds them (their maximum, then one 2^x per
+    // value against it) and merges the pair into the CTA's running pair for
     // that row (this warp's own slot). Pairs (m, z) are in the log2 domain as
     // everywhere: m = max value times log2 e, z = sum of 2^(v log2 e - m).
     // The pair with the larger reference keeps its sum; only the other one's
@@ -872,39 +877,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       z = fmaf(zlo, uno::ex2(lo == -INFINITY ? -INFINITY : lo - hi), zhi);
       m = hi;
     };
-    auto swap_row_stats = [&](float* sv, int out, int cbase) {
+    float* sxp = reinterpret_cast<float*>(srs + 4 * 2 * BN) + quarter * 32 * 33;
+    auto swap_row_stats = [&](const float* sv, int out, int cbase) {
       constexpr float kL2e = 1.4426950408889634f;
-      const bool b16 = (lane & 16) != 0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {  // single values: (v log2 e, 1)
-        const float keep = b16 ? sv[i + 16] : sv[i];
-        const float send = b16 ? sv[i] : sv[i + 16];
-        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-        float m = keep * kL2e, z = (keep > -INFINITY) ? 1.f : 0.f;
-        merge_mz(m, z, recv * kL2e, (recv > -INFINITY) ? 1.f : 0.f);
-        sv[i] = m;
-        sv[16 + i] = z;
-      }
+      for (int e = 0; e < 32; ++e) sxp[e * 33 + lane] = sv[e];
+      __syncwarp();
+      float v[32];
 #pragma unroll
-      for (int h = 8; h >= 1; h >>= 1) {  // pairs (sv[i], sv[16 + i]), i < 2h
-        const bool bit = (lane & h) != 0;
+      for (int c = 0; c < 32; ++c) v[c] = sxp[lane * 33 + c];
+      __syncwarp();  // the next chunk may overwrite the scratch
+      float mx = v[0];
 #pragma unroll
-        for (int i = 0; i < h; ++i) {
-          float m = bit ? sv[i + h] : sv[i];
-          float z = bit ? sv[16 + i + h] : sv[16 + i];
-          const float sm = bit ? sv[i] : sv[i + h];
-          const float sz = bit ? sv[16 + i] : sv[16 + i + h];
-          const float rm = __shfl_xor_sync(0xFFFFFFFFu, sm, h);
-          const float rz = __shfl_xor_sync(0xFFFFFFFFu, sz, h);
-          merge_mz(m, z, rm, rz);
-          sv[i] = m;
-          sv[16 + i] = z;
-        }
-      }
+      for (int c = 1; c < 32; ++c) mx = fmaxf(mx, v[c]);
+      if (mx == -INFINITY) return;  // no stored value in this row's 32 columns
+      const float ml = mx * kL2e;
+      float zp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 32; ++c) zp[c & 3] += uno::ex2(fmaf(v[c], kL2e, -ml));
       float2* slot = srs + (quarter * 2 + out) * BN + cbase + lane;
-      float2 a = *slot;
-      merge_mz(a.x, a.y, sv[0], sv[16]);
-      *slot = a;
+      float2 acc = *slot;
+      merge_mz(acc.x, acc.y, ml, (zp[0] + zp[1]) + (zp[2] + zp[3]));
+      *slot = acc;
     };
     if (swap_stats)
       for (int q = 0; q < 2 * BN; q += 32)
