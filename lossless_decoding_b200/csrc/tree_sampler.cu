@@ -354,6 +354,9 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
   // (prefix p owns min(a, budget / (p + 1)) slots); s_coff[a][nk] = their number
   __shared__ int s_coff[kMaxTopK + 1][kMaxBudget + 1];
   __shared__ int s_cap[kMaxBudget];  // budget / (p + 1)
+  // s_slot_p[a][c]: the prefix that owns candidate slot c when a choices are
+  // available (so each candidate is written by its own thread)
+  __shared__ unsigned char s_slot_p[kMaxTopK + 1][kMaxCand];
   __shared__ unsigned char s_rep[kMaxDepth][kMaxBudget];
   __shared__ int s_cnt[kMaxDepth + 1];
   __shared__ int s_off[kMaxDepth + 2];
@@ -374,6 +377,11 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
     }
     s_coff[a][budget] = off;
   }
+  __syncthreads();
+  for (int w = tid; w < (k + 1) * budget; w += kBuildThreads) {
+    const int a = w / budget, q = w - a * budget;
+    for (int c = s_coff[a][q]; c < s_coff[a][q + 1]; ++c) s_slot_p[a][c] = static_cast<unsigned char>(q);
+  }
   if (tid == 0) {
     k_score[0][0] = 0.f;  // the empty prefix
     k_tup[0][0] = 0ull;
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
   }
   __syncthreads();
   // The kept set, position by position, by the whole CTA: per step the
-  // candidates are written (one thread per kept prefix), then ranked, a
+  // candidates are written (one thread per candidate slot), then ranked, a
   // barrier after each. A candidate's rank (the candidates ahead of it) is
   // counted by kRankLanes threads, each comparing it with every kRankLanes-th
   // candidate, and summed by shuffles within the group, so a step costs a few
@@ -401,16 +409,11 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
     // of min(avail, budget / (p + 1)) slots from s_coff[avail][p]
     const int nc = s_coff[avail][nk];
     const unsigned long long shift = 4ull * (kMaxDepth - 1 - j);
-    for (int p = tid; p < nk; p += kBuildThreads) {
-      const int off = s_coff[avail][p];
-      const int cnt = s_coff[avail][p + 1] - off;
-      const float ps = k_score[cur][p];
-      const unsigned long long pt = k_tup[cur][p];
-#pragma unroll 4
-      for (int s = 0; s < cnt; ++s) {
-        c_score[off + s] = ps + s_lq[j][s];
-        c_tup[off + s] = pt | (static_cast<unsigned long long>(s) << shift);
-      }
+    for (int c = tid; c < nc; c += kBuildThreads) {
+      const int p = s_slot_p[avail][c];
+      const int sl = c - s_coff[avail][p];
+      c_score[c] = k_score[cur][p] + s_lq[j][sl];
+      c_tup[c] = k_tup[cur][p] | (static_cast<unsigned long long>(sl) << shift);
     }
     __syncthreads();
     const int nxt = cur ^ 1;
@@ -425,10 +428,11 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
       if (mine) {
         sc = c_score[c];
         tu = c_tup[c];
-#pragma unroll 4
-        for (int o = sub; o < nc; o += kRankLanes) {
+#pragma unroll 8
+        for (int o = sub; o < nc; o += kRankLanes) {  // branch-free: both loads always
           const float so = c_score[o];
-          ahead += (so > sc || (so == sc && c_tup[o] < tu)) ? 1 : 0;
+          const unsigned long long to = c_tup[o];
+          ahead += static_cast<int>((so > sc) | ((so == sc) & (to < tu)));
         }
       }
 #pragma unroll
