@@ -146,10 +146,11 @@ __global__ void __launch_bounds__(kTopThreads) tree_topk_part_kernel(const TopkP
   TopList<KM> top;
   top.init();
   float lm = -INFINITY, ls = 0.f;  // running max (log2 domain) and sum of 2^(x log2 e - lm)
-  auto take = [&](const float* f, int n, long long x0) {
-    float mk = f[0];
-    for (int e = 1; e < n; ++e) mk = fmaxf(mk, f[e]);
-    mk *= kLog2e;
+  // folds n values into (lm, ls); returns their maximum
+  auto stat = [&](const float* f, int n) {
+    float mx = f[0];
+    for (int e = 1; e < n; ++e) mx = fmaxf(mx, f[e]);
+    const float mk = mx * kLog2e;
     if (mk > lm) {
       ls *= uno::ex2(lm - mk);
       lm = mk;
@@ -159,29 +160,67 @@ __global__ void __launch_bounds__(kTopThreads) tree_topk_part_kernel(const TopkP
       for (int e = 0; e < n; ++e) add += uno::ex2(fmaf(f[e], kLog2e, -lm));
       ls += add;
     }
-    for (int e = 0; e < n; ++e) top.offer(f[e], static_cast<int>(x0 + e));
+    return mx;
   };
-  for (long long base = v_lo + tid; base < v_hi; base += kTopThreads * kTopInFlight) {
+  // A value below the warp's threshold cannot be among the slab's top_k:
+  // top_k values at least that large have been seen (the threshold is the
+  // top_k-th largest of the lanes' round maxima, one per lane, and only
+  // grows). Offering only values at or above it keeps most of the list
+  // insertions -- chains of dependent compares that also split the warp --
+  // out of the stream; the kept set and its order are unchanged.
+  float thr = -INFINITY;
+  auto kth_of_lanes = [&](float x) {
+    float kth = -INFINITY;
+    for (int r = 0; r < P.top_k; ++r) {
+      float m = x;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      kth = m;
+      if (!(m > -INFINITY)) break;  // the same in every lane
+      const unsigned holders = __ballot_sync(0xFFFFFFFFu, x == m);
+      if (lane == __ffs(holders) - 1) x = -INFINITY;  // one lane gives up its value
+    }
+    return kth;
+  };
+  // rounds of kTopInFlight vectors per thread; every thread runs every round
+  // (the threshold's shuffles need whole warps)
+  for (long long r0 = v_lo; r0 < v_hi; r0 += kTopThreads * kTopInFlight) {
     uint4 raw[kTopInFlight];
 #pragma unroll
     for (int k = 0; k < kTopInFlight; ++k) {
-      const long long vi = base + static_cast<long long>(k) * kTopThreads;
+      const long long vi = r0 + tid + static_cast<long long>(k) * kTopThreads;
       raw[k] = (vi < v_hi) ? __ldg(reinterpret_cast<const uint4*>(row) + vi)
                            : make_uint4(0u, 0u, 0u, 0u);
     }
+    float rmax = -INFINITY;
 #pragma unroll
     for (int k = 0; k < kTopInFlight; ++k) {
-      const long long vi = base + static_cast<long long>(k) * kTopThreads;
+      const long long vi = r0 + tid + static_cast<long long>(k) * kTopThreads;
       if (vi < v_hi) {
         float f[kVec];
         R::unpack(raw[k], f);
-        take(f, kVec, vi * kVec);
+        rmax = fmaxf(rmax, stat(f, kVec));
+      }
+    }
+    // (top_k rounds of shuffles per round: they cost more than they save at
+    // top_k 16, measured; such lists take every value)
+    if (P.top_k <= 8) thr = fmaxf(thr, kth_of_lanes(rmax));
+#pragma unroll
+    for (int k = 0; k < kTopInFlight; ++k) {
+      const long long vi = r0 + tid + static_cast<long long>(k) * kTopThreads;
+      if (vi < v_hi) {
+        float f[kVec];
+        R::unpack(raw[k], f);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e)
+          if (f[e] >= thr) top.offer(f[e], static_cast<int>(vi * kVec + e));
       }
     }
   }
   for (long long v = tail0 + tid; v < e1; v += kTopThreads) {
     const float f = R::at(row, v);
-    take(&f, 1, v);
+    stat(&f, 1);
+    top.offer(f, static_cast<int>(v));
   }
 
   // ---- the slab's (max, sum) ----
