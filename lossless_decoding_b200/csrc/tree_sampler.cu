@@ -291,6 +291,23 @@ __global__ void __launch_bounds__(kTopThreads) tree_topk_part_kernel(const TopkP
 template <int KM>
 __device__ void merge_row(const TopkParams& P, int rw, int lane, int32_t* s_id, float* s_lq) {
   const size_t p0 = static_cast<size_t>(rw) * P.slabs;
+  // the slabs' candidates, a batch of loads at a time; the first batch is in
+  // flight while the (max, sum) pairs are merged
+  const int n = P.slabs * P.top_k;
+  const float* pv = P.part_val + p0 * P.top_k;
+  const int32_t* pi = P.part_id + p0 * P.top_k;
+  constexpr int kBatch = 8;
+  float v[kBatch];
+  int id[kBatch];
+  auto load_batch = [&](int c0) {
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) {
+      const int c = c0 + 32 * e;
+      v[e] = (c < n) ? __ldcg(pv + c) : -INFINITY;
+      id[e] = (c < n) ? __ldcg(pi + c) : INT_MAX;
+    }
+  };
+  load_batch(lane);
   // the slabs' (max, sum) pairs: a lane merges its slabs (at most two when
   // there are 64), then the warp
   float m = -INFINITY, sum = 0.f;
@@ -322,19 +339,8 @@ __device__ void merge_row(const TopkParams& P, int rw, int lane, int32_t* s_id, 
 
   TopList<KM> top;
   top.init();
-  const int n = P.slabs * P.top_k;
-  const float* pv = P.part_val + p0 * P.top_k;
-  const int32_t* pi = P.part_id + p0 * P.top_k;
-  constexpr int kBatch = 8;  // loads issued before any is used
   for (int c0 = lane; c0 < n; c0 += 32 * kBatch) {
-    float v[kBatch];
-    int id[kBatch];
-#pragma unroll
-    for (int e = 0; e < kBatch; ++e) {
-      const int c = c0 + 32 * e;
-      v[e] = (c < n) ? __ldcg(pv + c) : -INFINITY;
-      id[e] = (c < n) ? __ldcg(pi + c) : INT_MAX;
-    }
+    if (c0 != lane) load_batch(c0);
 #pragma unroll
     for (int e = 0; e < kBatch; ++e) top.offer(v[e], id[e]);
   }
@@ -500,7 +506,8 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
     const int j = w / nk + 1, m = w - (j - 1) * nk;
     const unsigned long long pre = prefix_of(k_tup[cur][m], j);
     bool rep = true;
-    for (int m2 = 0; m2 < m && rep; ++m2) rep = prefix_of(k_tup[cur][m2], j) != pre;
+#pragma unroll 4
+    for (int m2 = 0; m2 < m; ++m2) rep &= prefix_of(k_tup[cur][m2], j) != pre;
     s_rep[j - 1][m] = rep ? 1 : 0;
   }
   __syncthreads();
@@ -521,8 +528,9 @@ __global__ void __launch_bounds__(kBuildThreads) tree_build_kernel(const TopkPar
   __syncthreads();  // also orders the padding stores before the node stores
   auto node_id = [&](int j, unsigned long long pre) {  // node of a depth-j prefix
     int rank = 0;
+#pragma unroll 4
     for (int m2 = 0; m2 < nk; ++m2)
-      rank += (s_rep[j - 1][m2] && prefix_of(k_tup[cur][m2], j) < pre) ? 1 : 0;
+      rank += static_cast<int>((s_rep[j - 1][m2] != 0) & (prefix_of(k_tup[cur][m2], j) < pre));
     return s_off[j] + rank;
   };
   for (int w = tid; w < D * nk; w += kBuildThreads) {
