@@ -8,7 +8,6 @@ independence of the draft word from the accept and draw words, and the
 edge cases (V = 1, a row with no finite logit).
 """
 import numpy as np
-import pytest
 from scipy.special import softmax as sp_softmax
 from scipy.stats import chisquare
 
