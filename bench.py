@@ -76,9 +76,9 @@ def _peaks():
 # summaries in profiles/. A figure is reported only while the kernel source it was taken on
 # is unchanged (first 16 hex digits of its sha256), else traffic is null.
 MEASURED_TRAFFIC = {
-    # dual_kernel: average of the step's four launches (63.6 + 5.3, 44.1 + 0.1,
-    # 223.2 + 74.1, 130.1 + 0.4 MB read + written)
-    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "815b2e0103670a69", 135.24e6),
+    # dual_kernel: average of the step's four launches (63.6 + 3.2, 44.1 + 0.0,
+    # 224.0 + 74.2, 130.1 + 0.1 MB read + written)
+    ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "33fb88aa9ae18da6", 134.84e6),
     # sample_drafts_kernel over the 64 x 16 q rows: 313.0 MB read + 3.6 MB written
     ("batched_decode_b64_k16", "draft"): ("draft_sample.cu", "9c3a8c794d39d5b7", 316.59e6),
     # stream 641.9 MB read + 0.1 MB written, draw 39.0 MB read, per verifier call
