@@ -15,9 +15,11 @@
 //                      still keeps the SMs' loads in flight. Each thread keeps
 //                      a sorted register list of its best logits (larger
 //                      first, ties to the smaller id) and a running (max, sum
-//                      of 2^(x - max)); the CTA merges the lists in top_k
-//                      argmax rounds and writes the slab's list and (max, sum)
-//                      to the workspace.
+//                      of 2^(x - max)); only logits at or above a warp
+//                      threshold (the top_k-th largest lane maximum so far)
+//                      are offered to the lists. The CTA merges the lists in
+//                      top_k argmax rounds and writes the slab's list and
+//                      (max, sum) to the workspace.
 //   tree_build_kernel  one CTA per sequence: one warp per row merges its
 //                      slabs and writes the ids and log softmax(q)(id) =
 //                      x - logsumexp; then the budget best sequences by
