@@ -81,8 +81,8 @@ MEASURED_TRAFFIC = {
     ("batched_decode_b64_k16", "dual"): ("dualpath.cu", "33fb88aa9ae18da6", 134.84e6),
     # sample_drafts_kernel over the 64 x 16 q rows: 313.0 MB read + 3.6 MB written
     ("batched_decode_b64_k16", "draft"): ("draft_sample.cu", "9c3a8c794d39d5b7", 316.59e6),
-    # stream 641.9 MB read + 0.1 MB written, draw 39.0 MB read, per verifier call
-    ("batched_decode_b64_k16", "verify"): ("verify.cu", "696e7dfc1a0a17f7", 681.00e6),
+    # stream 641.8 MB read + 3.4 MB written, draw 39.0 MB read, per verifier call
+    ("batched_decode_b64_k16", "verify"): ("verify.cu", "85a3dfdf71983495", 684.24e6),
 }
 
 
